@@ -1,0 +1,203 @@
+"""Scalar CPU oracle for block-scaled microscaling quantization.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's
+CPU-baseline leg use it; the product package never imports it.  The numeric
+work happens in ``mxq_oracle.c`` (IEEE double, its own rounding routines);
+this module only moves numpy arrays in and out of it.
+
+Arrays of floating-point elements are passed as their raw bit patterns:
+uint16 for bf16 / f16, uint32 for f32.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+DTYPES = {"bf16": 0, "f16": 1, "f32": 2}
+FORMATS = {"fp8": 0, "mxfp4": 1, "nvfp4": 2}
+_BITS = {"bf16": np.uint16, "f16": np.uint16, "f32": np.uint32}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        d, i, i64, p = ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+        L.orc_e2m1_value.restype = d
+        L.orc_e2m1_value.argtypes = [i]
+        L.orc_e2m1_code.restype = i
+        L.orc_e2m1_code.argtypes = [d]
+        for name in ("orc_round_bf16", "orc_round_f16", "orc_round_f32", "orc_round_e4m3"):
+            getattr(L, name).restype = d
+            getattr(L, name).argtypes = [d]
+        L.orc_encode_e4m3.restype = ctypes.c_uint8
+        L.orc_encode_e4m3.argtypes = [d]
+        L.orc_decode_e4m3.restype = d
+        L.orc_decode_e4m3.argtypes = [ctypes.c_uint8]
+        L.orc_decode_array.argtypes = [p, i, i64, p]
+        L.orc_round_array.argtypes = [p, i, i64, p]
+        L.orc_mx_scale_exp.restype = i
+        L.orc_mx_scale_exp.argtypes = [d]
+        L.orc_mx_quantize.restype = i
+        L.orc_mx_quantize.argtypes = [p, i, i64, i64, p, p]
+        L.orc_mx_dequantize.restype = i
+        L.orc_mx_dequantize.argtypes = [p, p, i64, i64, p, i]
+        L.orc_cache_scale_exp.restype = i
+        L.orc_cache_scale_exp.argtypes = [d, i]
+        L.orc_cache_element.restype = d
+        L.orc_cache_element.argtypes = [d, i, i]
+        L.orc_quantize_cache.restype = i
+        L.orc_quantize_cache.argtypes = [p, p, i, i64, i64, i, i]
+        L.orc_check_offs.restype = i
+        L.orc_check_offs.argtypes = [p, i64, i64]
+        L.orc_grouped_mm.restype = i
+        L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---- scalar helpers -------------------------------------------------------
+
+def e2m1_value(code):
+    return lib().orc_e2m1_value(int(code))
+
+
+def e2m1_code(v):
+    return lib().orc_e2m1_code(float(v))
+
+
+def round_bf16(v):
+    return lib().orc_round_bf16(float(v))
+
+
+def round_f16(v):
+    return lib().orc_round_f16(float(v))
+
+
+def round_f32(v):
+    return lib().orc_round_f32(float(v))
+
+
+def round_e4m3(v):
+    return lib().orc_round_e4m3(float(v))
+
+
+def encode_e4m3(v):
+    return lib().orc_encode_e4m3(float(v))
+
+
+def decode_e4m3(b):
+    return lib().orc_decode_e4m3(int(b))
+
+
+def mx_scale_exp(amax):
+    return lib().orc_mx_scale_exp(float(amax))
+
+
+def cache_scale_exp(amax, fmt):
+    return lib().orc_cache_scale_exp(float(amax), FORMATS[fmt])
+
+
+def cache_element(x, k, fmt):
+    return lib().orc_cache_element(float(x), int(k), FORMATS[fmt])
+
+
+# ---- array helpers --------------------------------------------------------
+
+def decode(bits, dtype):
+    """Bit patterns of `dtype` -> float64 values."""
+    b = _c(bits, _BITS[dtype])
+    out = np.empty(b.shape, np.float64)
+    lib().orc_decode_array(_ptr(b), DTYPES[dtype], b.size, _ptr(out))
+    return out
+
+
+def round_to(values, dtype):
+    """float64 values -> bit patterns of `dtype` (nearest-even)."""
+    v = _c(values, np.float64)
+    out = np.empty(v.shape, _BITS[dtype])
+    lib().orc_round_array(_ptr(v), DTYPES[dtype], v.size, _ptr(out))
+    return out
+
+
+def mx_quantize(x_bits, dtype="bf16"):
+    """x [..., K] -> (packed uint8 [..., K/2], scales uint8 [..., K/32])."""
+    x = _c(x_bits, _BITS[dtype])
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    packed = np.empty(x.shape[:-1] + (K // 2,), np.uint8)
+    scales = np.empty(x.shape[:-1] + (K // 32,), np.uint8)
+    rc = lib().orc_mx_quantize(_ptr(x), DTYPES[dtype], rows, K, _ptr(packed), _ptr(scales))
+    if rc != 0:
+        raise ValueError("oracle mx_quantize: bad arguments (K %% 32 != 0?) rc=%d" % rc)
+    return packed, scales
+
+
+def mx_dequantize(packed, scales, dtype="bf16"):
+    """packed [..., K/2], scales [..., K/32] -> bits of dtype [..., K]."""
+    p = _c(packed, np.uint8)
+    s = _c(scales, np.uint8)
+    K = p.shape[-1] * 2
+    rows = p.size // p.shape[-1] if p.shape[-1] else 0
+    out = np.empty(p.shape[:-1] + (K,), _BITS[dtype])
+    rc = lib().orc_mx_dequantize(_ptr(p), _ptr(s), rows, K, _ptr(out), DTYPES[dtype])
+    if rc != 0:
+        raise ValueError("oracle mx_dequantize: bad arguments rc=%d" % rc)
+    return out
+
+
+def quantize_cache(x_bits, fmt, block_size, dtype="bf16"):
+    """Fake quantization of x [..., C]; returns bits of the same dtype."""
+    x = _c(x_bits, _BITS[dtype])
+    C = x.shape[-1]
+    rows = x.size // C if C else 0
+    out = np.empty_like(x)
+    rc = lib().orc_quantize_cache(_ptr(x), _ptr(out), DTYPES[dtype], rows, C, FORMATS[fmt],
+                                  int(block_size))
+    if rc != 0:
+        raise ValueError("oracle quantize_cache: bad arguments rc=%d" % rc)
+    return out
+
+
+def check_offs(offs, T):
+    o = _c(offs, np.int32)
+    return lib().orc_check_offs(_ptr(o), o.size, int(T)) == 0
+
+
+def grouped_mm(a_bits, packed, scales, offs, transpose_w=False, rows=None):
+    """Exact-sum (double) grouped GEMM on the listed rows (default: all).
+
+    a_bits: bf16 bits [T, Kin]; packed [E, N, K/2]; scales [E, N, K/32];
+    offs int32 [E] (inclusive prefix sums of the expert row counts).
+    Returns float64 [len(rows), Nout], not rounded.
+    """
+    a = _c(a_bits, np.uint16)
+    p = _c(packed, np.uint8)
+    s = _c(scales, np.uint8)
+    o = _c(offs, np.int32)
+    E, N, Kh = p.shape
+    K = 2 * Kh
+    T = a.shape[0]
+    if rows is None:
+        rows = np.arange(T, dtype=np.int64)
+    r = _c(rows, np.int64)
+    nout = K if transpose_w else N
+    out = np.zeros((r.size, nout), np.float64)
+    rc = lib().orc_grouped_mm(_ptr(a), _ptr(p), _ptr(s), _ptr(o), T, E, N, K,
+                              1 if transpose_w else 0, _ptr(r), r.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle grouped_mm: rc=%d" % rc)
+    return out
+

@@ -1,0 +1,489 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against something it does not compute from its
+own tables: values the pages print (tests/golden/, each with its citation),
+brute force over every bf16 bit pattern, library casts (torch, numpy), closed
+forms and invariants of the method.  A plausible slip in the oracle - a wrong
+midpoint, a tie broken the wrong way, a swapped nibble, an off-by-one in a
+scale exponent, a dropped sign, a transposed GEMM operand - fails at least
+one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as gen
+from conftest import read_golden
+
+# The eight E2M1 magnitudes as the page prints them (codes 0..7).
+PAGE_TABLE = {int(i): float(v) for i, v in read_golden("e2m1_table.txt")}
+T8 = np.array([PAGE_TABLE[i] for i in range(8)])
+MIDPOINTS = [float(v) for v in read_golden("e2m1_midpoints.txt")[0]]
+
+
+def all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f32 = (bits.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(f32)
+    vals = f32.astype(np.float64)
+    return bits[keep], vals[keep]
+
+
+def bruteforce_e2m1_mag(a):
+    """Index of the nearest of T8 to a >= 0; on a tie the even index."""
+    d = np.abs(a[:, None] - T8[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    idx = np.where(cand, np.arange(8)[None, :], 99)
+    even = np.where(cand & (np.arange(8)[None, :] % 2 == 0), np.arange(8)[None, :], 99)
+    return np.where(even.min(axis=1) < 99, even.min(axis=1), idx.min(axis=1))
+
+
+def e4m3_candidates():
+    """(value, code) of the 127 non-negative finite E4M3 numbers, built from
+    the format definition (bias 7, 3 mantissa bits, S.1111.111 is NaN)."""
+    out = [(m * 2.0 ** -9, m) for m in range(8)]
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            out.append(((8 + m) * 2.0 ** (e - 10), (e << 3) | m))
+    return np.array([v for v, _ in out]), np.array([c for _, c in out])
+
+
+def bruteforce_e4m3(vals):
+    cv, cc = e4m3_candidates()
+    a = np.abs(vals)
+    d = np.abs(a[:, None] - cv[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    even = cand & (cc[None, :] % 2 == 0)
+    pick = np.where(even.any(axis=1), np.argmax(even, axis=1), np.argmax(cand, axis=1))
+    r = cv[pick]
+    r = np.where(a > 448.0, 448.0, r)
+    return np.copysign(r, vals)
+
+
+# ---------------------------------------------------------------- E2M1 table
+
+def test_table_matches_page():
+    for i, v in PAGE_TABLE.items():
+        assert oracle.e2m1_value(i) == v, i
+    # index 8 prints as 0.0: a positive zero
+    assert math.copysign(1.0, oracle.e2m1_value(8)) == 1.0
+
+
+def test_table_sign_half():
+    # codes 8..15 carry the sign bit of 0..7 (codes 13..15 are not printed)
+    for c in range(1, 8):
+        assert oracle.e2m1_value(c + 8) == -T8[c]
+
+
+def test_midpoints_are_means_of_neighbours():
+    assert len(MIDPOINTS) == 7
+    for i, m in enumerate(MIDPOINTS):
+        assert m == (T8[i] + T8[i + 1]) / 2
+
+
+@pytest.mark.parametrize("row", read_golden("e2m1_ties.txt"))
+def test_tie_rule_from_page(row):
+    tie, want = float(row[0]), float(row[1])
+    assert oracle.e2m1_value(oracle.e2m1_code(tie)) == want
+    assert oracle.e2m1_value(oracle.e2m1_code(-tie)) == -want
+
+
+def test_e2m1_code_bruteforce_every_bf16():
+    _, vals = all_finite_bf16()
+    # distances are exact in double only while |v| < 2^40; beyond, the
+    # nearest magnitude is 6 (code 7) by definition
+    big = np.abs(vals) >= 2.0**40
+    mag = np.where(big, 7, bruteforce_e2m1_mag(np.where(big, 0.0, np.abs(vals))))
+    want = mag | np.where(vals < 0, 8, 0)
+    got = np.array([oracle.e2m1_code(v) for v in vals])
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (vals[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e2m1_sign_reading():
+    # -0.0 carries no sign bit; a tiny negative keeps it (nibble 8)
+    assert oracle.e2m1_code(-0.0) == 0
+    assert oracle.e2m1_code(-1e-30) == 8
+    assert oracle.e2m1_code(-7.0) == 15
+
+
+# ------------------------------------------------------- binary formats
+
+def test_e4m3_rounding_bruteforce_every_bf16():
+    _, vals = all_finite_bf16()
+    vals = vals[np.abs(vals) < 1e6]
+    want = bruteforce_e4m3(vals)
+    got = np.array([oracle.round_e4m3(v) for v in vals])
+    assert np.array_equal(np.signbit(got), np.signbit(want))
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (vals[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e4m3_rounding_matches_torch_cast():
+    _, vals = all_finite_bf16()
+    vals = vals[np.abs(vals) <= 448.0]
+    t = torch.from_numpy(vals.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64)
+    got = np.array([oracle.round_e4m3(v) for v in vals])
+    assert np.array_equal(got, t.numpy())
+
+
+def test_e4m3_encode_decode_all_bytes():
+    cv, cc = e4m3_candidates()
+    byval = dict(zip(cc.tolist(), cv.tolist()))
+    for b in range(256):
+        mag = b & 0x7F
+        if mag == 0x7F:
+            assert math.isnan(oracle.decode_e4m3(b))
+            continue
+        v = oracle.decode_e4m3(b)
+        assert abs(v) == byval[mag]
+        assert math.copysign(1.0, v) == (-1.0 if b & 0x80 else 1.0)
+        assert oracle.encode_e4m3(v) == b
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 2**32, 200000, dtype=np.uint64).astype(np.uint32)
+    edge = np.array([0x00000001, 0x00008000, 0x00007FFF, 0x00018000, 0x007FFFFF, 0x00800000,
+                     0x7F7F7FFF, 0x7F7F8000, 0x7F7FFFFF, 0x3F808000, 0x3F818000, 0x80000001,
+                     0xFF7F8000, 0x00000000, 0x80000000], np.uint32)
+    bits = np.concatenate([bits, edge])
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.round_to(f.astype(np.float64), "bf16")
+    assert np.array_equal(got, want)
+
+
+def test_f16_rounding_matches_numpy():
+    rng = np.random.default_rng(2)
+    v = np.concatenate([
+        rng.standard_normal(100000) * 10.0 ** rng.uniform(-9, 5, 100000),
+        np.array([65504.0, 65519.99, 65520.0, 2.0**-24, 2.0**-25, 3 * 2.0**-26, 2.0**-14,
+                  -0.0, 0.0, 1 + 2.0**-11, 1 + 3 * 2.0**-11])])
+    with np.errstate(over="ignore"):
+        want = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.round_to(v, "f16"), want)
+
+
+def test_f32_rounding_matches_numpy():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal(100000) * 10.0 ** rng.uniform(-45, 38, 100000)
+    v = np.concatenate([v, [2.0**-149, 2.0**-150, 3 * 2.0**-151, 3.4028235677973366e38]])
+    with np.errstate(over="ignore"):
+        want = v.astype(np.float32).view(np.uint32)
+    assert np.array_equal(oracle.round_to(v, "f32"), want)
+
+
+# ------------------------------------------------------- MXFP4 pack / unpack
+
+def full_table():
+    return np.array([PAGE_TABLE.get(c, -T8[c - 8] if c >= 8 else None) for c in range(16)])
+
+
+def test_every_byte_decodes_low_nibble_first():
+    tab = full_table()
+    packed = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    scales = np.full((1, 16), 127, np.uint8)
+    out = oracle.decode(oracle.mx_dequantize(packed, scales, "f32"), "f32")[0]
+    b = np.arange(256)
+    assert np.array_equal(out[0::2], tab[b & 15])
+    assert np.array_equal(out[1::2], tab[b >> 4])
+
+
+def test_scale_byte_is_power_of_two():
+    for s in range(256):
+        packed = np.full((1, 16), 0x22, np.uint8)  # two codes 2 (= 1.0)
+        scales = np.array([[s]], np.uint8)
+        out = oracle.decode(oracle.mx_dequantize(packed, scales, "f32"), "f32")[0]
+        if s == 255:
+            assert np.isnan(out).all()
+        else:
+            assert (out == math.ldexp(1.0, s - 127)).all(), s
+
+
+def test_every_byte_round_trips():
+    # byte b beside a 0x77 byte (two 6.0s) so the block max is 6 and the
+    # derived scale is 2^0 again
+    for b in range(256):
+        packed = np.zeros((1, 16), np.uint8)
+        packed[0, 0] = b
+        packed[0, 1] = 0x77
+        scales = np.array([[127]], np.uint8)
+        x = oracle.mx_dequantize(packed, scales, "bf16")
+        p2, s2 = oracle.mx_quantize(x, "bf16")
+        assert s2[0, 0] == 127
+        lo, hi = b & 15, b >> 4
+        lo, hi = (0 if lo == 8 else lo), (0 if hi == 8 else hi)  # +0.0 re-encodes as nibble 0
+        assert p2[0, 0] == lo | (hi << 4), b
+        assert p2[0, 1] == 0x77
+
+
+def test_dequant_quant_dequant_is_identity():
+    # the value-exact round trip quantize_mxfp4 promises for exactly
+    # representable inputs, over every scale byte that stays finite in bf16
+    rng = np.random.default_rng(4)
+    rows = 253
+    packed = rng.integers(0, 256, (rows, 64), dtype=np.uint8)
+    scales = np.repeat(np.arange(rows, dtype=np.uint8)[:, None], 4, axis=1)
+    x = oracle.mx_dequantize(packed, scales, "bf16")
+    p2, s2 = oracle.mx_quantize(x, "bf16")
+    x2 = oracle.mx_dequantize(p2, s2, "bf16")
+    assert np.array_equal(oracle.decode(x2, "bf16"), oracle.decode(x, "bf16"))
+
+
+def test_scale_rule_floor_log2_minus_2():
+    x = gen.mixed_blocks(64, 256).view(torch.int16).numpy().view(np.uint16)
+    vals = oracle.decode(x, "bf16").reshape(-1, 32)
+    _, s = oracle.mx_quantize(x, "bf16")
+    s = s.reshape(-1).astype(int)
+    for blk, byte in zip(vals, s):
+        amax = np.abs(blk).max()
+        if amax == 0:
+            assert byte == 0
+            continue
+        e = byte - 127
+        fl = math.frexp(amax)[1] - 1  # floor(log2 amax)
+        assert e == max(fl - 2, -127)
+        if e > -127:
+            assert 2.0 ** (e + 2) <= amax < 2.0 ** (e + 3)
+
+
+def test_forced_rows_closed_form():
+    x = gen.mx_small().view(torch.int16).numpy().view(np.uint16)
+    p, s = oracle.mx_quantize(x, "bf16")
+    # row 0 all zero: scale byte 0, codes 0
+    assert (p[0] == 0).all() and (s[0] == 0).all()
+    # row 1 all 1.75: floor(log2 1.75) - 2 = -2 -> byte 125; 1.75/2^-2 = 7 saturates to 6 (code 7)
+    assert (s[1] == 125).all() and (p[1] == 0x77).all()
+    # row 2: block max exactly 2 -> e = -1 (byte 126); the +-2 element is 4.0 = code 6 (+8 if negative)
+    assert (s[2] == 126).all()
+    xv = oracle.decode(x[2], "bf16")
+    codes = np.stack([p[2] & 15, p[2] >> 4], axis=1).reshape(-1)
+    two = np.abs(xv) == 2.0
+    assert two.sum() == 8
+    assert np.array_equal(codes[two], np.where(xv[two] < 0, 14, 6))
+    # row 3 all 2^-3: e = -5 (byte 122); 2^-3 / 2^-5 = 4 -> code 6
+    assert (s[3] == 122).all() and (p[3] == 0x66).all()
+
+
+def test_mx_quantize_bruteforce_tiny():
+    rng = np.random.default_rng(5)
+    tab = full_table()
+    for trial in range(200):
+        v = rng.standard_normal(32) * 10.0 ** rng.uniform(-3, 3)
+        bits = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        xv = oracle.decode(bits, "bf16")
+        p, s = oracle.mx_quantize(bits.reshape(1, 32), "bf16")
+        amax = np.abs(xv).max()
+        e = max(math.frexp(amax)[1] - 1 - 2, -127)
+        assert s[0, 0] == e + 127
+        scaled = xv / 2.0 ** e
+        codes = np.stack([p[0] & 15, p[0] >> 4], axis=1).reshape(-1)
+        for j in range(32):
+            d = np.abs(scaled[j] - tab)
+            cands = np.nonzero(d == d.min())[0]
+            # among equally near codes: the sign must follow v<0, ties go to the even magnitude
+            cands = [c for c in cands if (c >= 8) == (scaled[j] < 0) or tab[c] == 0]
+            mags = sorted({c & 7 for c in cands}, key=lambda m: (m % 2, m))
+            want = mags[0] | (8 if scaled[j] < 0 else 0)
+            assert codes[j] == want, (trial, j, scaled[j])
+
+
+def test_effective_bits_ratio(facts):
+    x = gen.normal_bf16(9, (4, 7168)).view(torch.int16).numpy().view(np.uint16)
+    p, s = oracle.mx_quantize(x, "bf16")
+    assert s.nbytes * 16 == p.nbytes  # MXFP4: 8 scale bits per 32 values of 4 bits
+    assert facts["r1_fp4_scale_bytes"] * 8 == facts["r1_fp4_packed_bytes"]
+    assert facts["expert_cols"] / 2 == facts["expert_packed_cols"]
+    assert facts["expert_cols"] / facts["nvfp4_block_size"] == facts["expert_nvfp4_scale_cols"]
+    assert 4 + 8 / facts["nvfp4_block_size"] == facts["nvfp4_effective_bits"]
+
+
+# ----------------------------------------------------- quantize_cache
+
+QMAX = {"fp8": 448.0, "mxfp4": 6.0, "nvfp4": 6.0}
+CLAMP = {"fp8": (-126, 127), "mxfp4": (-126, 127), "nvfp4": (-9, 8)}
+
+
+def independent_scale_exp(amax, fmt):
+    lo, hi = CLAMP[fmt]
+    if amax == 0:
+        return lo
+    k = -300
+    while QMAX[fmt] * 2.0 ** k < amax:  # exact: powers of two times 448 or 6
+        k += 1
+    return min(max(k, lo), hi)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "mxfp4", "nvfp4"])
+def test_cache_scale_is_power_of_two_ceiling(fmt):
+    _, vals = all_finite_bf16()
+    amaxes = np.unique(np.abs(vals))
+    for a in amaxes[::7]:
+        assert oracle.cache_scale_exp(a, fmt) == independent_scale_exp(a, fmt), a
+    q = QMAX[fmt]
+    assert oracle.cache_scale_exp(q, fmt) == 0
+    assert oracle.cache_scale_exp(np.nextafter(q, 10 * q), fmt) == 1
+    assert oracle.cache_scale_exp(q / 2, fmt) == -1
+
+
+def cache_bruteforce(xv, fmt, B):
+    """Fake quantization by nearest-grid search: for each group the scale is
+    the least power of two with 2^k*qmax >= amax; each value goes to the
+    nearest grid point (ties: even code), zero magnitudes are +0 for the fp4
+    formats and keep their sign for fp8; then nearest-even to bf16."""
+    out = np.empty_like(xv)
+    cv, cc = e4m3_candidates()
+    for r in range(xv.shape[0]):
+        for c0 in range(0, xv.shape[1], B):
+            blk = xv[r, c0:c0 + B]
+            k = independent_scale_exp(np.abs(blk).max(), fmt)
+            v = blk / 2.0 ** k
+            if fmt == "fp8":
+                q = bruteforce_e4m3(v)
+            else:
+                mag = bruteforce_e2m1_mag(np.abs(v))
+                q = np.where(mag == 0, 0.0, np.copysign(T8[mag], v))
+            out[r, c0:c0 + B] = q * 2.0 ** k
+    f32 = out.astype(np.float32)  # exact: at most 4 significant bits, >= 2^-135
+    assert np.array_equal(f32.astype(np.float64), out)
+    return torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("fmt,B", [("fp8", 128), ("fp8", 32), ("mxfp4", 32), ("nvfp4", 16),
+                                   ("nvfp4", 7)])
+def test_cache_matches_nearest_grid_bruteforce(fmt, B):
+    x = torch.cat([gen.kv_cache((1, 6, 256)).view(6, 256), gen.mixed_blocks(6, 256)])
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    got = oracle.quantize_cache(bits, fmt, B)
+    want = cache_bruteforce(oracle.decode(bits, "bf16"), fmt, B)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("fmt,B", [("fp8", 32), ("mxfp4", 32), ("nvfp4", 16)])
+def test_cache_tail_group_is_zero_padded(fmt, B):
+    # a final partial group behaves as if zero-padded to a full group
+    x = gen.kv_cache((1, 5, 48)).view(5, 48).clone()
+    x[:, 40:] = 0.0
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    full = oracle.quantize_cache(bits, fmt, B)
+    part = oracle.quantize_cache(np.ascontiguousarray(bits[:, :40]), fmt, B)
+    assert np.array_equal(part, full[:, :40])
+
+
+@pytest.mark.parametrize("fmt,B", [("fp8", 128), ("mxfp4", 32), ("nvfp4", 16)])
+def test_cache_is_idempotent(fmt, B):
+    x = torch.cat([gen.kv_cache((1, 16, 512)).view(16, 512), gen.mixed_blocks(16, 512)])
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    once = oracle.quantize_cache(bits, fmt, B)
+    twice = oracle.quantize_cache(once, fmt, B)
+    assert np.array_equal(once, twice)
+
+
+def test_cache_fp8_matches_torch_cast():
+    x = gen.kv_cache((1, 32, 256)).view(32, 256)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    xv = oracle.decode(bits, "bf16")
+    want = np.empty_like(xv)
+    for r in range(32):
+        for c0 in range(0, 256, 32):
+            blk = xv[r, c0:c0 + 32]
+            k = independent_scale_exp(np.abs(blk).max(), "fp8")
+            q = torch.from_numpy((blk / 2.0 ** k).astype(np.float32)).to(torch.float8_e4m3fn)
+            want[r, c0:c0 + 32] = q.to(torch.float64).numpy() * 2.0 ** k
+    w = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    got = oracle.quantize_cache(bits, "fp8", 32)
+    assert np.array_equal(got, w.view(np.uint16))
+
+
+def test_cache_clamps():
+    # nvfp4: a block of ~1e-40 values takes the 2^-9 floor and rounds to +0
+    tiny = torch.full((1, 16), 1e-40, dtype=torch.bfloat16).view(torch.int16).numpy()
+    out = oracle.quantize_cache(tiny.view(np.uint16), "nvfp4", 16)
+    assert (out == 0).all()
+    # nvfp4: a block with max 1e4 takes the 2^8 ceiling and saturates at 6*256
+    big = torch.tensor([[1e4] + [1.0] * 15], dtype=torch.bfloat16).view(torch.int16).numpy()
+    out = oracle.decode(oracle.quantize_cache(big.view(np.uint16), "nvfp4", 16), "bf16")
+    assert out[0, 0] == 1536.0
+    # fp8: tiny values keep the sign of zero
+    neg = torch.tensor([[-1e-30, 1.0] + [0.0] * 30], dtype=torch.bfloat16).view(torch.int16)
+    out = oracle.decode(oracle.quantize_cache(neg.numpy().view(np.uint16), "fp8", 32), "bf16")
+    assert out[0, 0] == 0.0 and math.copysign(1.0, out[0, 0]) == -1.0
+    # mxfp4: tiny negatives become +0
+    out = oracle.decode(oracle.quantize_cache(neg.numpy().view(np.uint16), "mxfp4", 32), "bf16")
+    assert out[0, 0] == 0.0 and math.copysign(1.0, out[0, 0]) == 1.0
+
+
+# ----------------------------------------------------- grouped GEMM
+
+def small_moe(T=7, counts=(3, 0, 4), N=5, K=64, seed=11):
+    E = len(counts)
+    offs = np.cumsum(counts).astype(np.int32)
+    assert offs[-1] == T
+    packed, scales = gen.random_packed(E, N, K, 118, 130, workload=seed)
+    a = gen.normal_bf16(seed, (T, K)).view(torch.int16).numpy().view(np.uint16)
+    return a, packed.numpy(), scales.numpy(), offs
+
+
+def dense_weights(packed, scales):
+    E = packed.shape[0]
+    return np.stack([oracle.decode(oracle.mx_dequantize(packed[e], scales[e], "f32"), "f32")
+                     for e in range(E)])
+
+
+def test_grouped_mm_forward_matches_numpy():
+    a, packed, scales, offs = small_moe()
+    W = dense_weights(packed, scales)
+    av = oracle.decode(a, "bf16")
+    got = oracle.grouped_mm(a, packed, scales, offs)
+    lo = 0
+    for e, hi in enumerate(offs):
+        want = av[lo:hi] @ W[e].T
+        np.testing.assert_allclose(got[lo:hi], want, rtol=1e-12, atol=1e-300)
+        lo = hi
+
+
+def test_grouped_mm_dgrad_matches_numpy():
+    a, packed, scales, offs = small_moe()
+    N = packed.shape[1]
+    g = gen.normal_bf16(12, (7, N)).view(torch.int16).numpy().view(np.uint16)
+    W = dense_weights(packed, scales)
+    gv = oracle.decode(g, "bf16")
+    got = oracle.grouped_mm(g, packed, scales, offs, transpose_w=True)
+    lo = 0
+    for e, hi in enumerate(offs):
+        np.testing.assert_allclose(got[lo:hi], gv[lo:hi] @ W[e], rtol=1e-12, atol=1e-300)
+        lo = hi
+
+
+def test_grouped_mm_one_hot_rows_pick_weights():
+    _, packed, scales, offs = small_moe()
+    W = dense_weights(packed, scales)
+    K = packed.shape[2] * 2
+    T = int(offs[-1])
+    a = np.zeros((T, K), np.float32)
+    ks = [(3 * t + 1) % K for t in range(T)]
+    for t, k in enumerate(ks):
+        a[t, k] = 1.0
+    bits = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.grouped_mm(bits, packed, scales, offs)
+    expert = np.searchsorted(offs, np.arange(T), side="right")
+    for t in range(T):
+        assert np.array_equal(got[t], W[expert[t], :, ks[t]])
+
+
+def test_grouped_mm_rejects_bad_offs():
+    a, packed, scales, _ = small_moe()
+    with pytest.raises(ValueError):
+        oracle.grouped_mm(a, packed, scales, np.array([3, 2, 7], np.int32))
+    with pytest.raises(ValueError):
+        oracle.grouped_mm(a, packed, scales, np.array([3, 3, 6], np.int32))
+    assert oracle.check_offs(np.array([0, 0, 7], np.int32), 7)
