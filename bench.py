@@ -1,0 +1,449 @@
+#!/usr/bin/env python3
+"""Benchmark of the block-scaled quantization hot path on B200.
+
+One step is one pass of every hot-path operation over synthetic inputs that
+are resident in HBM:
+  1. mx_quantize     expert weights bf16 [64, 2048, 7168] -> packed + E8M0 scales
+  2. grouped GEMM    forward  x bf16 [32768, 7168] . deq(W)^T, W [32, 2048, 7168]
+  3. grouped GEMM    backward grad_out bf16 [32768, 2048] . deq(W)
+  4. quantize_cache  KV-like bf16 [4, 8192, 512]: fp8 (block 128), mxfp4 (32), nvfp4 (16)
+  5. mx_dequantize   the packed weights of step 1 back to bf16 [64, 2048, 7168]
+Every kernel reads inputs last touched more than L2's 126 MB of traffic
+earlier (the 2.4 GB pack/unpack passes and the GEMMs sit between reuses).
+
+Printed metric: quant/dequant HBM GB/s = algorithmic bytes of steps 1, 4, 5
+over their summed device time (CUDA events on the launching stream), with
+the grouped-GEMM TFLOP/s beside it.  `--impl reference` times the scalar
+CPU oracle instead, on a bounded sample of the same workload.
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload (weak
+scaling, no data exchange); timings are the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "quant/dequant HBM GB/s (% of ~8 TB/s); MXFP4 grouped-GEMM TFLOPS (% of peak)"
+
+# Workload sizes.
+W_SHAPE = (64, 2048, 7168)
+KV_SHAPE = (4, 8192, 512)
+CACHE_RUNS = (("fp8", 128), ("mxfp4", 32), ("nvfp4", 16))
+T, E, N, K = 32768, 32, 2048, 7168
+
+
+def algorithmic_bytes():
+    w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
+    kv = KV_SHAPE[0] * KV_SHAPE[1] * KV_SHAPE[2]
+    return {
+        # read bf16, write packed nibbles + one scale byte per 32
+        "mx_quantize": w * 2 + w // 2 + w // 32,
+        "mx_dequantize": w // 2 + w // 32 + w * 2,
+        # read and write bf16
+        "quantize_cache": kv * 4,
+    }
+
+
+def gemm_flops():
+    return 2.0 * T * N * K
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(name):
+    p = os.path.join(ROOT, "nvfp4_quantization_amax_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key, src):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    ent = t.get(kernel_key)
+    if not ent or ent.get("source_sha") != source_hash(src):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------- clocks
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+def gpu_id(torch, dev):
+    """nvidia-smi -i selector for a torch device (its UUID)."""
+    u = str(torch.cuda.get_device_properties(dev).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", "-i", str(self.index),
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                mask = int(parts[3], 16)
+            except ValueError:
+                continue
+            for bit, name in REASON_BITS.items():
+                if mask & bit and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = sorted(sm)[len(sm) // 2:] if len(sm) > 3 else sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU arm
+
+class Step:
+    """Device-resident inputs and outputs of one step, and the step itself."""
+
+    def __init__(self, torch, mxq, gen, dev):
+        self.torch, self.mxq = torch, mxq
+        self.W = gen.expert_weights(*W_SHAPE, device=dev)
+        self.P, self.S = mxq.mx_quantize(self.W)
+        self.Wout = torch.empty_like(self.W)
+        self.kv = [gen.kv_cache(KV_SHAPE, device=dev, seed_base=10 * i) for i in range(3)]
+        self.kv_out = [torch.empty_like(k) for k in self.kv]
+        W5 = gen.expert_weights(E, N, K, device=dev, workload=5)
+        self.P5, self.S5 = mxq.mx_quantize(W5)
+        del W5
+        self.x = gen.normal_bf16(gen.seed_for(5, 3), (T, K), device=dev)
+        self.g = gen.normal_bf16(gen.seed_for(5, 4), (T, N), device=dev)
+        counts = gen.expert_counts(T, E, device=dev)
+        self.offs = torch.cumsum(counts, 0).to(torch.int32)
+        self.y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        self.gx = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.names = ["mx_quantize", "gemm_fwd", "gemm_dgrad", "qc_fp8", "qc_mxfp4", "qc_nvfp4",
+                      "mx_dequantize"]
+
+    def run(self, ev=None):
+        m = self.mxq
+        calls = [
+            lambda: m.mx_quantize(self.W, self.P, self.S),
+            lambda: m.mxfp4_grouped_mm(self.x, self.P5, self.S5, self.offs, False, self.y,
+                                       self.status),
+            lambda: m.mxfp4_grouped_mm(self.g, self.P5, self.S5, self.offs, True, self.gx,
+                                       self.status),
+        ] + [
+            (lambda i=i, f=f, b=b: m.quantize_cache(self.kv[i], f, b, self.kv_out[i]))
+            for i, (f, b) in enumerate(CACHE_RUNS)
+        ] + [lambda: m.mx_dequantize(self.P, self.S, self.torch.bfloat16, self.Wout)]
+        for i, c in enumerate(calls):
+            if ev is not None:
+                ev[i][0].record()
+            c()
+            if ev is not None:
+                ev[i][1].record()
+
+
+def time_e2e(torch, mxq, step, steps):
+    """Same metric through the public API with host (pinned) buffers: every
+    call copies its inputs host->device and its result device->host."""
+    hW = step.W.cpu().pin_memory()
+    hP, hS = step.P.cpu().pin_memory(), step.S.cpu().pin_memory()
+    hkv = [k.cpu().pin_memory() for k in step.kv]
+    h2d = hW.numel() * 2 + hP.numel() + hS.numel() + sum(k.numel() * 2 for k in hkv)
+    d2h = hP.numel() + hS.numel() + hW.numel() * 2 + sum(k.numel() * 2 for k in hkv)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        mxq.mx_quantize(hW)
+        for k, (f, b) in zip(hkv, CACHE_RUNS):
+            mxq.quantize_cache(k, f, b)
+        mxq.mx_dequantize(hP, hS, torch.bfloat16)
+    torch.cuda.synchronize()
+    dt = (time.perf_counter() - t0) / steps
+    return dt, h2d, d2h
+
+
+def run_gpu(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_quantization_amax_b200 as mxq
+    import synthetic as gen
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    step = Step(torch, mxq, gen, dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in step.names]
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError("grouped GEMM reported status %d" % int(step.status.item()))
+
+    per = {n: [] for n in step.names}
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id(torch, dev)) as clk:
+        start.record()
+        for _ in range(args.steps):
+            step.run(ev)
+            torch.cuda.synchronize()  # read this step's events
+            for n, (a, b) in zip(step.names, ev):
+                per[n].append(a.elapsed_time(b))
+        stop.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
+    if world > 1:
+        t = torch.tensor([total_ms] + [kern_ms[n] for n in step.names], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t[0])
+        kern_ms = {n: float(v) for n, v in zip(step.names, t[1:])}
+
+    e2e_dt, h2d, d2h = time_e2e(torch, mxq, step, max(1, min(args.steps, 3)))
+    if world > 1:
+        t = torch.tensor([e2e_dt], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_dt = float(t[0])
+
+    if rank == 0:
+        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary())
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks):
+    peaks, peak_src = load_peaks()
+    ab = algorithmic_bytes()
+    qd_bytes = ab["mx_quantize"] + ab["mx_dequantize"] + 3 * ab["quantize_cache"]
+    qd_ms = kern_ms["mx_quantize"] + kern_ms["mx_dequantize"] + \
+        sum(kern_ms[n] for n in ("qc_fp8", "qc_mxfp4", "qc_nvfp4"))
+    gbs = qd_bytes / (qd_ms * 1e-3) / 1e9 * world
+    gemm_ms = kern_ms["gemm_fwd"] + kern_ms["gemm_dgrad"]
+    tflops = 2 * gemm_flops() / (gemm_ms * 1e-3) / 1e12 * world
+    kernels = {}
+    for n, ms in kern_ms.items():
+        if n.startswith("gemm"):
+            tf = gemm_flops() / (ms * 1e-3) / 1e12
+            kernels[n] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                          "frac": round(tf / peaks["bf16_tflops"], 4)}
+        else:
+            b = ab["quantize_cache"] if n.startswith("qc_") else ab[n]
+            g = b / (ms * 1e-3) / 1e9
+            kernels[n] = {"ms": round(ms, 4), "gbs": round(g, 1),
+                          "frac": round(g / peaks["hbm_gbs"], 4)}
+    dominant = max(kern_ms, key=kern_ms.get)
+    if dominant.startswith("gemm"):
+        ach = gemm_flops() / (kern_ms[dominant] * 1e-3) / 1e12
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": round(ach, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / peaks["bf16_tflops"], 4),
+                "traffic": profiled_traffic(dominant, "grouped_mm_tc.cu"),
+                "peak_source": peak_src + " bf16 burst"}
+    else:
+        b = ab["quantize_cache"] if dominant.startswith("qc_") else ab[dominant]
+        ach = b / (kern_ms[dominant] * 1e-3) / 1e9
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": round(ach, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "traffic": profiled_traffic(dominant, "elementwise.cu"),
+                "peak_source": peak_src + " copy"}
+    e2e_gbs = qd_bytes / e2e_dt / 1e9 * world
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 / Box-Muller inputs of the configured shapes)",
+        "config": {
+            "workload": "mx_quantize + mx_dequantize of expert weights bf16 [64,2048,7168]; "
+                        "quantize_cache fp8/128, mxfp4/32, nvfp4/16 of KV bf16 [4,8192,512]; "
+                        "MXFP4 grouped GEMM fwd + dgrad, x [32768,7168], W [32,2048,7168], "
+                        "multinomial expert counts",
+            "hbm_fraction_nominal_8tbs": round(gbs / world / 8000.0, 4),
+            "l2": "no flush; every kernel's inputs were last touched >126 MB of traffic earlier",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "gemm": {"value": round(tflops, 1), "unit": "TFLOP/s",
+                 "frac_of_measured_burst": round(tflops / world / peaks["bf16_tflops"], 4),
+                 "frac_of_measured_sustained":
+                     round(tflops / world / peaks["bf16_tflops_sustained"], 4),
+                 "frac_of_nominal_2250": round(tflops / world / 2250.0, 4)},
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 7 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------ CPU oracle arm
+
+def cpu_baseline(budget_s):
+    """The scalar oracle, as it stands, on a bounded sample of the same
+    workload (single thread).  Returns GB/s over the same algorithmic bytes
+    per element as the GPU metric, plus the oracle's grouped-GEMM GFLOP/s."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synthetic as gen
+
+    per = max(budget_s / 4.0, 0.5)
+    done = {}
+
+    def timed(fn, bytes_per_call):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= per:
+                return n * bytes_per_call, dt, n
+
+    W = gen.expert_weights(1, 16, 7168).view(16, 7168)
+    wb = W.view(torch.int16).numpy().view(np.uint16)
+    pk, sc = oracle.mx_quantize(wb)
+    kv = gen.kv_cache((1, 64, 512)).view(64, 512).view(torch.int16).numpy().view(np.uint16)
+    e_w = 16 * 7168
+    b1, t1, n1 = timed(lambda: oracle.mx_quantize(wb), e_w * 2 + e_w // 2 + e_w // 32)
+    b2, t2, n2 = timed(lambda: oracle.mx_dequantize(pk, sc), e_w // 2 + e_w // 32 + e_w * 2)
+    e_kv = 64 * 512
+
+    def qc():
+        for f, b in CACHE_RUNS:
+            oracle.quantize_cache(kv, f, b)
+    b3, t3, n3 = timed(qc, 3 * e_kv * 4)
+    done["gbs"] = (b1 + b2 + b3) / (t1 + t2 + t3) / 1e9
+    # grouped GEMM: 2 rows of one expert, forward (includes dequantizing W_e)
+    Wg = gen.expert_weights(1, 256, 7168, workload=5)
+    pg, sg = oracle.mx_quantize(Wg.view(torch.int16).numpy().view(np.uint16))
+    pg, sg = pg.reshape(1, 256, 3584), sg.reshape(1, 256, 224)
+    a = gen.normal_bf16(3, (8, 7168)).view(torch.int16).numpy().view(np.uint16)
+    offs = np.array([8], np.int32)
+    t0 = time.perf_counter()
+    oracle.grouped_mm(a, pg, sg, offs, rows=np.arange(8))
+    gdt = time.perf_counter() - t0
+    done["gemm_gflops"] = 2.0 * 8 * 256 * 7168 / gdt / 1e9
+    return {"value": round(done["gbs"], 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "gemm_gflops": round(done["gemm_gflops"], 4),
+            "sample": ("mx_quantize %dx and mx_dequantize %dx of [16,7168] weight rows, "
+                       "quantize_cache (3 formats) %dx of [64,512] KV rows, ~%.0f s total; "
+                       "GEMM: 8 rows x 256 outputs x 7168" % (n1, n2, n3, t1 + t2 + t3))}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; the loop keeps the contract's shape
+    cb = cpu_baseline(max(4.0, min(30.0, 2.0 * args.steps)))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "bounded sample of the GPU arm's "
+                                                        "workload on the scalar CPU oracle"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_gpu(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

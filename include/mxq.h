@@ -1,0 +1,151 @@
+/*
+ * mxq.h - C ABI of libmxq.so: block-scaled microscaling quantization on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named as device buffers are CUDA device pointers owned by the
+ *    caller.  The library allocates nothing and keeps no pointer after a
+ *    call returns.
+ *  - Tensors are dense and row-major.  Leading dimensions are flattened into
+ *    `rows` (rows = numel / last_dim).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call is asynchronous on that stream; the library never
+ *    synchronizes.
+ *  - Return value: MXQ_OK (0) or a negative mxq_status.  Argument errors are
+ *    detected on the host before anything is launched and leave every output
+ *    untouched.  MXQ_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *  - Element dtypes are mxq_dtype values; floating-point results are rounded
+ *    to nearest-even with subnormals kept and overflow to +-infinity.
+ *  - Inputs are expected to be finite; NaN/Inf inputs give unspecified
+ *    (but memory-safe) results.
+ *
+ * Sources.  The operations follow these pages (title, then section):
+ *  [MX] "nemo_automodel.components.quantization.mxfp4": module docstring
+ *       (packed layout), quantize_mxfp4, dequantize_mxfp4, MXFP4GroupedMM,
+ *       _FP4_E2M1_TABLE, _FP4_E2M1_MIDPOINTS, MXFP4_BLOCK_SIZE.
+ *  [CQ] "nemo_automodel.components.models.deepseek_v41.quantization":
+ *       quantize_cache, _power_of_two_ceiling.
+ *  [MO] "NVIDIA Model Optimizer: from mtq.quantize to a 4.95-bit
+ *       DeepSeek-R1", section "NVFP4 in the code: two scales and a nibble"
+ *       (E2M1 tie rule and nibble packing, E4M3 maximum 448).
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MXQ_OK = 0,
+  MXQ_ERR_INVALID_ARG = -1, /* null pointer, bad enum, aliasing in/out    */
+  MXQ_ERR_SHAPE = -2,       /* negative size, K % 32 != 0, ...            */
+  MXQ_ERR_ALIGNMENT = -3,   /* a pointer the call needs aligned is not    */
+  MXQ_ERR_UNSUPPORTED = -4, /* valid request this build does not handle   */
+  MXQ_ERR_CUDA = -5,        /* launch failed                              */
+  MXQ_ERR_BAD_OFFS = -6,    /* device-side: offs not a valid partition    */
+  MXQ_ERR_TIMEOUT = -7      /* device-side: a pipeline wait gave up       */
+} mxq_status;
+
+typedef enum { MXQ_BF16 = 0, MXQ_F16 = 1, MXQ_F32 = 2 } mxq_dtype;
+
+typedef enum { MXQ_FMT_FP8 = 0, MXQ_FMT_MXFP4 = 1, MXQ_FMT_NVFP4 = 2 } mxq_format;
+
+/* MXFP4 quantize + pack along the last dimension  ([MX] quantize_mxfp4).
+ *
+ *  x       device, [rows, K] elements of x_dtype (bf16, f16 or f32), 16-byte
+ *          aligned.
+ *  packed  device, [rows, K/2] bytes, 16-byte aligned (output).  Byte j of a
+ *          row holds the E2M1 code of column 2j in its low nibble and of
+ *          column 2j+1 in its high nibble ([MX] module docstring).
+ *  scales  device, [rows, K/32] bytes (output): one E8M0 scale (float8_e8m0fnu
+ *          bits, value 2^(byte-127)) per 32 contiguous columns.
+ *
+ *  Per 32-column block: amax = max |x|; scale exponent e = floor(log2(amax))
+ *  - 2, clamped to [-127, 127] (an all-zero block takes -127, byte 0x00);
+ *  code = E2M1 cast of x / 2^e: the nearest of {0,0.5,1,1.5,2,3,4,6}, ties
+ *  to the even code (ties at 0.75, 1.75, 3.5 go up, [MO] _cast_fp4), values
+ *  beyond 6 saturate to 6, sign bit set iff x < 0.
+ *  Errors: K % 32 != 0 -> MXQ_ERR_SHAPE; null or misaligned x/packed ->
+ *  MXQ_ERR_INVALID_ARG / MXQ_ERR_ALIGNMENT.  rows == 0 or K == 0: no-op. */
+int mx_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                void* scales, void* stream);
+
+/* MXFP4 unpack + scale ([MX] dequantize_mxfp4).
+ *
+ *  packed  device, [rows, K/2] bytes, 16-byte aligned (layout as above).
+ *  scales  device, [rows, K/32] E8M0 bytes.
+ *  out     device, [rows, K] elements of out_dtype, 16-byte aligned (output).
+ *
+ *  out[r][k] = E2M1_TABLE[nibble] * 2^(scale_byte - 127), rounded to
+ *  out_dtype (exact in bf16/f32 except overflow; f16 overflows above 65504
+ *  to +-inf).  Nibble 8 decodes to +0.0.  Scale byte 0xFF (E8M0 NaN) gives
+ *  NaN (bf16 0x7FC0, f16 0x7E00, f32 0x7FC00000) for its 32 values.
+ *  Errors as for mx_quantize. */
+int mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t K, void* out,
+                  int out_dtype, void* stream);
+
+/* Fake quantization of cache values ([CQ] quantize_cache).
+ *
+ *  in, out  device, [rows, channels] elements of dtype; out must not overlap
+ *           in (the result is independently stored).
+ *  format   MXQ_FMT_FP8 (E4M3 elements), MXQ_FMT_MXFP4 (E2M1 elements,
+ *           E8M0-range scales) or MXQ_FMT_NVFP4 (E2M1 elements, E4M3-range
+ *           scales).
+ *  block_size  channels per scale (>= 1).  A final partial group of a row
+ *           uses its own channels only (the page's zero padding).
+ *
+ *  Per group: amax = max |x|; qmax = 448 (fp8) or 6 (fp4); scale s = the
+ *  least power of two with s*qmax >= amax (_power_of_two_ceiling of
+ *  amax/qmax, decided exactly), clamped to [2^-126, 2^127] (fp8, mxfp4) or
+ *  [2^-9, 2^8] (nvfp4); an all-zero group takes the lower clamp.
+ *  out = round_dtype(q(x/s) * s) with q the E4M3 cast (nearest-even,
+ *  saturating at 448, sign of zero kept) or the E2M1 cast above (a zero
+ *  magnitude gives +0.0).
+ *  Fast path: block_size in {8,16,32,64,128,256}, channels % block_size == 0,
+ *  16-byte aligned in/out.  Anything else runs a slower general kernel.
+ *  Errors: block_size < 1 -> MXQ_ERR_SHAPE; bad format/dtype or overlapping
+ *  in/out -> MXQ_ERR_INVALID_ARG. */
+int quantize_cache(const void* in, void* out, int dtype, int64_t rows, int64_t channels,
+                   int format, int32_t block_size, void* stream);
+
+/* Grouped GEMM over MXFP4-packed expert weights, dequantized on the fly
+ * ([MX] MXFP4GroupedMM forward and backward).
+ *
+ *  a        device, bf16 [T, Kin], rows grouped contiguously by expert,
+ *           16-byte aligned.
+ *  packed   device, [E, N, K/2] bytes; scales device, [E, N, K/32] E8M0
+ *           bytes: W_e[n][k] = dequantized value, exactly representable in
+ *           bf16 for scale bytes <= 252.
+ *  offs     device, int32 [E]: inclusive prefix sums of the expert row counts;
+ *           expert e owns rows [offs[e-1], offs[e]) with offs[-1] = 0.
+ *  transpose_w = 0 (forward):        Kin = K, y bf16 [T, N], y = a . W_e^T
+ *  transpose_w = 1 (input gradient): Kin = N, y bf16 [T, K], y = a . W_e
+ *  Products accumulate in fp32; y is rounded to bf16 (nearest-even).
+ *  dev_status  device int32 (nullable).  If offs is not non-decreasing
+ *           with offs[E-1] == T the kernel writes MXQ_ERR_BAD_OFFS there and
+ *           leaves y unwritten; if a pipeline wait gives up it writes
+ *           MXQ_ERR_TIMEOUT.  The kernel never writes MXQ_OK: clear the word
+ *           before the call to read it afterwards.
+ *  Errors (host): K % 32 != 0, E < 1, N < 1, T < 0 -> MXQ_ERR_SHAPE; null
+ *  pointers -> MXQ_ERR_INVALID_ARG.  The tensor-core path needs N and K
+ *  multiples of 128 and 64 and 16-byte aligned a / y; other shapes run a
+ *  slower general kernel. */
+int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
+                     int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
+                     int32_t* dev_status, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* mxq_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int mxq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

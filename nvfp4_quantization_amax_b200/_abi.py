@@ -1,0 +1,183 @@
+"""ctypes binding of libmxq.so: argument marshalling only."""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmxq.so")
+
+_DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+_FORMATS = {"fp8": 0, "mxfp4": 1, "nvfp4": 2}
+
+_lib = None
+
+
+class MxqError(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__("%s failed: %s (%d)" % (what, status_string(status), status))
+        self.status = status
+
+
+def lib_path():
+    return _LIB_PATH
+
+
+def lib():
+    """Load libmxq.so (built in-tree by nvfp4_quantization_amax_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libmxq.so not found at %s; build it with "
+                               "`python -m nvfp4_quantization_amax_b200.build`" % _LIB_PATH)
+        L = ctypes.CDLL(_LIB_PATH)
+        i, i32, i64, p = ctypes.c_int, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
+        L.mx_quantize.restype = i
+        L.mx_quantize.argtypes = [p, i, i64, i64, p, p, p]
+        L.mx_dequantize.restype = i
+        L.mx_dequantize.argtypes = [p, p, i64, i64, p, i, p]
+        L.quantize_cache.restype = i
+        L.quantize_cache.argtypes = [p, p, i, i64, i64, i, i32, p]
+        L.mxfp4_grouped_mm.restype = i
+        L.mxfp4_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, p, p]
+        L.mxq_status_string.restype = ctypes.c_char_p
+        L.mxq_status_string.argtypes = [i]
+        L.mxq_version.restype = i
+        L.mxq_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().mxq_status_string(int(status)).decode()
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise MxqError(rc, what)
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _to_device(t):
+    """(device tensor, was_on_host).  Host tensors are moved to the current
+    CUDA device; pinned ones without blocking the host."""
+    if t.is_cuda:
+        return t, False
+    if not torch.cuda.is_available():
+        raise RuntimeError("no CUDA device: libmxq runs only on the GPU")
+    return t.to(torch.device("cuda", torch.cuda.current_device()),
+                non_blocking=t.is_pinned()), True
+
+
+def _to_host(t):
+    out = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    out.copy_(t, non_blocking=True)
+    torch.cuda.current_stream(t.device).synchronize()
+    return out
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mx_quantize(x, packed=None, scales=None):
+    """MXFP4 quantize + pack along the last dim.
+
+    x: bf16/f16/f32 [..., K], K % 32 == 0.  Returns (packed uint8 [..., K/2],
+    scales uint8 [..., K/32]): two E2M1 codes per byte (low nibble = even
+    column) and one E8M0 scale byte (float8_e8m0fnu bits) per 32 columns.
+    """
+    if x.dtype not in _DTYPES:
+        raise TypeError("mx_quantize: unsupported dtype %s" % x.dtype)
+    x, host = _to_device(x)
+    x = x.contiguous()
+    K = x.shape[-1]
+    rows = x.numel() // K if K else 0
+    if packed is None:
+        packed = torch.empty(x.shape[:-1] + (K // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (K // 32,), dtype=torch.uint8, device=x.device)
+    rc = lib().mx_quantize(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed), _ptr(scales),
+                           _stream(x.device))
+    _check(rc, "mx_quantize")
+    if host:
+        return _to_host(packed), _to_host(scales)
+    return packed, scales
+
+
+def mx_dequantize(packed, scales, dtype=torch.bfloat16, out=None):
+    """Unpack [..., K/2] E2M1 bytes with [..., K/32] E8M0 scales to dtype [..., K]."""
+    if dtype not in _DTYPES:
+        raise TypeError("mx_dequantize: unsupported dtype %s" % dtype)
+    packed, host = _to_device(packed)
+    scales, _ = _to_device(scales)
+    packed = packed.contiguous()
+    scales = scales.contiguous()
+    Kh = packed.shape[-1]
+    K = 2 * Kh
+    rows = packed.numel() // Kh if Kh else 0
+    if scales.numel() != rows * (K // 32):
+        raise ValueError("mx_dequantize: scales must have shape [..., K/32]")
+    if out is None:
+        out = torch.empty(packed.shape[:-1] + (K,), dtype=dtype, device=packed.device)
+    rc = lib().mx_dequantize(_ptr(packed), _ptr(scales), rows, K, _ptr(out), _DTYPES[dtype],
+                             _stream(packed.device))
+    _check(rc, "mx_dequantize")
+    return _to_host(out) if host else out
+
+
+def quantize_cache(values, format, block_size, out=None):
+    """Fake quantization of [..., channels] values in fp8 / mxfp4 / nvfp4;
+    returns a new tensor of the input dtype."""
+    if values.dtype not in _DTYPES:
+        raise TypeError("quantize_cache: unsupported dtype %s" % values.dtype)
+    if format not in _FORMATS:
+        raise ValueError("quantize_cache: format must be one of %s" % sorted(_FORMATS))
+    values, host = _to_device(values)
+    values = values.contiguous()
+    C = values.shape[-1] if values.dim() else 1
+    rows = values.numel() // C if C else 0
+    if out is None:
+        out = torch.empty_like(values)
+    rc = lib().quantize_cache(_ptr(values), _ptr(out), _DTYPES[values.dtype], rows, C,
+                              _FORMATS[format], int(block_size), _stream(values.device))
+    _check(rc, "quantize_cache")
+    return _to_host(out) if host else out
+
+
+def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, status=None):
+    """Grouped GEMM over MXFP4-packed expert weights.
+
+    a: bf16 [T, Kin] grouped by expert; packed uint8 [E, N, K/2]; scales
+    uint8 [E, N, K/32]; offs int32 [E] (cumulative row counts).
+    transpose_w False: Kin = K, returns a . W_e^T [T, N];
+    transpose_w True:  Kin = N, returns a . W_e   [T, K].
+    status: optional device int32 [1]; a bad offs or a timed-out pipeline
+    wait is reported there (the call itself is asynchronous).
+    """
+    if a.dtype != torch.bfloat16:
+        raise TypeError("mxfp4_grouped_mm: activations must be bf16")
+    a, host = _to_device(a)
+    packed, _ = _to_device(packed)
+    scales, _ = _to_device(scales)
+    offs, _ = _to_device(offs)
+    a, packed, scales = a.contiguous(), packed.contiguous(), scales.contiguous()
+    offs = offs.to(torch.int32).contiguous()
+    E, N, Kh = packed.shape
+    K = 2 * Kh
+    T = a.shape[0]
+    kin, nout = (N, K) if transpose_w else (K, N)
+    if a.shape[1] != kin:
+        raise ValueError("mxfp4_grouped_mm: a must be [T, %d]" % kin)
+    if tuple(scales.shape) != (E, N, K // 32) or offs.numel() != E:
+        raise ValueError("mxfp4_grouped_mm: scales [E, N, K/32] and offs [E] expected")
+    if out is None:
+        out = torch.empty((T, nout), dtype=torch.bfloat16, device=a.device)
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    rc = lib().mxfp4_grouped_mm(_ptr(a), _ptr(packed), _ptr(scales), _ptr(offs), T, E, N, K,
+                                1 if transpose_w else 0, _ptr(out), st, _stream(a.device))
+    _check(rc, "mxfp4_grouped_mm")
+    return _to_host(out) if host else out

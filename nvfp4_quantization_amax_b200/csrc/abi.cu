@@ -1,0 +1,110 @@
+// extern "C" entry points of libmxq.so: argument validation on the host,
+// then a launch on the caller's stream.  Declarations and the contract of
+// each call are in include/mxq.h.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "mxq.h"
+#include "mxq_launch.h"
+
+namespace mxq {
+
+int num_sms() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static bool valid_dtype(int d) { return d == MXQ_BF16 || d == MXQ_F16 || d == MXQ_F32; }
+static int elem_bytes(int d) { return d == MXQ_F32 ? 4 : 2; }
+
+static bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+  auto x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
+}
+
+}  // namespace mxq
+
+using namespace mxq;
+
+extern "C" {
+
+int mx_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed, void* scales,
+                void* stream) {
+  if (!valid_dtype(x_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 32 != 0) return MXQ_ERR_SHAPE;
+  if (rows == 0 || K == 0) return MXQ_OK;
+  if (!x || !packed || !scales) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed)) return MXQ_ERR_ALIGNMENT;
+  return launch_mx_quantize(x, x_dtype, rows, K, packed, scales, (cudaStream_t)stream);
+}
+
+int mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t K, void* out,
+                  int out_dtype, void* stream) {
+  if (!valid_dtype(out_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 32 != 0) return MXQ_ERR_SHAPE;
+  if (rows == 0 || K == 0) return MXQ_OK;
+  if (!packed || !scales || !out) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  return launch_mx_dequantize(packed, scales, rows, K, out, out_dtype, (cudaStream_t)stream);
+}
+
+int quantize_cache(const void* in, void* out, int dtype, int64_t rows, int64_t channels,
+                   int format, int32_t block_size, void* stream) {
+  if (!valid_dtype(dtype)) return MXQ_ERR_INVALID_ARG;
+  if (format != MXQ_FMT_FP8 && format != MXQ_FMT_MXFP4 && format != MXQ_FMT_NVFP4)
+    return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || channels < 0 || block_size < 1) return MXQ_ERR_SHAPE;
+  if (rows == 0 || channels == 0) return MXQ_OK;
+  if (!in || !out) return MXQ_ERR_INVALID_ARG;
+  int64_t bytes = rows * channels * elem_bytes(dtype);
+  if (overlap(in, bytes, out, bytes)) return MXQ_ERR_INVALID_ARG;
+  int B = block_size;
+  bool pow2_b = B >= 8 && B <= 256 && (B & (B - 1)) == 0;
+  bool fast = pow2_b && channels % B == 0 && aligned16(in) && aligned16(out);
+  return launch_quantize_cache(in, out, dtype, rows, channels, format, B, fast,
+                               (cudaStream_t)stream);
+}
+
+int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
+                     int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
+                     int32_t* dev_status, void* stream) {
+  if (T < 0 || E < 1 || N < 1 || K < 32 || K % 32 != 0) return MXQ_ERR_SHAPE;
+  if (transpose_w != 0 && transpose_w != 1) return MXQ_ERR_INVALID_ARG;
+  if (!packed || !scales || !offs) return MXQ_ERR_INVALID_ARG;
+  if (T == 0) return MXQ_OK;
+  if (!a || !y) return MXQ_ERR_INVALID_ARG;
+  if (E > 65536) return MXQ_ERR_UNSUPPORTED;
+  return launch_grouped_mm(a, packed, scales, offs, T, E, N, K, transpose_w, y, dev_status,
+                           (cudaStream_t)stream);
+}
+
+const char* mxq_status_string(int status) {
+  switch (status) {
+    case MXQ_OK: return "MXQ_OK";
+    case MXQ_ERR_INVALID_ARG: return "MXQ_ERR_INVALID_ARG";
+    case MXQ_ERR_SHAPE: return "MXQ_ERR_SHAPE";
+    case MXQ_ERR_ALIGNMENT: return "MXQ_ERR_ALIGNMENT";
+    case MXQ_ERR_UNSUPPORTED: return "MXQ_ERR_UNSUPPORTED";
+    case MXQ_ERR_CUDA: return "MXQ_ERR_CUDA";
+    case MXQ_ERR_BAD_OFFS: return "MXQ_ERR_BAD_OFFS";
+    case MXQ_ERR_TIMEOUT: return "MXQ_ERR_TIMEOUT";
+    default: return "MXQ_ERR_UNKNOWN";
+  }
+}
+
+int mxq_version(void) { return 100; }
+
+}  // extern "C"

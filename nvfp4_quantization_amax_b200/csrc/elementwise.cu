@@ -1,0 +1,343 @@
+// HBM-bound kernels: MXFP4 pack (mx_quantize), MXFP4 unpack (mx_dequantize)
+// and cache fake quantization (quantize_cache) for sm_100a.
+//
+// All three are streaming passes.  The work unit ("item") is 8 consecutive
+// elements of one row: one 16-byte load of bf16/f16 input.  A block of B
+// channels is B/8 consecutive items, handled by B/8 consecutive lanes of one
+// warp, which combine their block maximum with xor-shuffles.  Each thread
+// keeps kUnroll independent items in flight (coalesced 16-byte loads with
+// L1 no-allocate), and the grid is a whole number of waves over the SMs.
+//
+// Page references (title, then section):
+//  "nemo_automodel.components.quantization.mxfp4": quantize_mxfp4 (scale
+//   2^(floor(log2 amax) - 2), K % 32), dequantize_mxfp4, module docstring
+//   (low nibble = even column, one E8M0 scale per 32 columns).
+//  "nemo_automodel.components.models.deepseek_v41.quantization":
+//   quantize_cache (formats, block sizes, zero-padded tail group),
+//   _power_of_two_ceiling.
+#include "mxq_device.cuh"
+#include "mxq_launch.h"
+
+namespace mxq {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+// ---------------------------------------------------------- mx_quantize
+
+// Scale exponent of quantize_mxfp4 from the f32 bit pattern of a block's
+// amax: floor(log2 amax) - 2 clamped to [-127, 127]; zero -> -127.
+__device__ __forceinline__ int mx_scale_exp(uint32_t amax_f32bits) {
+  if (amax_f32bits == 0) return -127;
+  int e = floor_log2_f32bits(amax_f32bits) - 2;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads)
+mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
+                   uint8_t* __restrict__ scales, int64_t n_items) {
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
+       base += stride * kUnroll) {
+    uint32_t bits[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      if (item < n_items) load8<DT>(x, item, bits[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      bool valid = item < n_items;
+      // Block amax on magnitude bit patterns (monotone in |x| for finite x).
+      uint32_t m = 0;
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(bits[u][j]));
+      }
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (!valid) continue;
+      int e = mx_scale_exp(m);
+      float inv = exp2i(-e);  // exact power of two
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t b = bits[u][j];
+        // -0.0 carries no sign into the code; any other negative does.
+        uint32_t negzero = (DT == kF32) ? 0x80000000u : 0x8000u;
+        if (b == negzero) b = 0;
+        v[j] = elem_to_f32<DT>(b) * inv;  // exact: power-of-two scaling
+      }
+      packed[item] = e2m1x8(v);
+      if ((lane & 3) == 0) scales[item >> 2] = (uint8_t)(e + 127);
+    }
+  }
+}
+
+// -------------------------------------------------------- mx_dequantize
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads)
+mx_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+                     void* __restrict__ out, int64_t n_items) {
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
+       base += stride * kUnroll) {
+    uint32_t p[kUnroll], s[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      if (item < n_items) {
+        p[u] = ld_stream_u32(packed + item);
+        s[u] = ld_stream_u8(scales + (item >> 2));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      if (item >= n_items) continue;
+      if (s[u] == 0xFFu) {  // E8M0 NaN
+        store8_bits<DT>(out, item, ElemTraits<DT>::kNaN);
+        continue;
+      }
+      float scale = exp2i((int)s[u] - 127);  // 2^-127 .. 2^127, exact
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
+        // value * scale is exact; adding +0 turns the -0 of nibble 8 into +0
+        v[2 * j] = fmaf(f16lo(h2), scale, 0.0f);
+        v[2 * j + 1] = fmaf(f16hi(h2), scale, 0.0f);
+      }
+      store8<DT>(out, item, v);
+    }
+  }
+}
+
+// ------------------------------------------------------- quantize_cache
+
+template <int FMT>
+struct CacheFormat;
+template <>
+struct CacheFormat<MXQ_FMT_FP8> {
+  static constexpr int kLo = -126, kHi = 127;
+  // qmax = 448 = 1.75 * 2^8
+  static constexpr int kQExp = 8;
+  static constexpr uint32_t kQFrac = 0x600000u;
+};
+template <>
+struct CacheFormat<MXQ_FMT_MXFP4> {
+  static constexpr int kLo = -126, kHi = 127;
+  // qmax = 6 = 1.5 * 2^2
+  static constexpr int kQExp = 2;
+  static constexpr uint32_t kQFrac = 0x400000u;
+};
+template <>
+struct CacheFormat<MXQ_FMT_NVFP4> {
+  static constexpr int kLo = -9, kHi = 8;
+  static constexpr int kQExp = 2;
+  static constexpr uint32_t kQFrac = 0x400000u;
+};
+
+// Exponent k of the least power of two with 2^k * qmax >= amax, clamped:
+// with amax = 2^E * (1 + f) and qmax = 2^Q * (1 + g), k = E - Q when
+// f <= g and E - Q + 1 otherwise.
+template <int FMT>
+__device__ __forceinline__ int cache_scale_exp(uint32_t amax_f32bits) {
+  using F = CacheFormat<FMT>;
+  if (amax_f32bits == 0) return F::kLo;
+  int k = floor_log2_f32bits(amax_f32bits) - F::kQExp +
+          (frac23_f32bits(amax_f32bits) > F::kQFrac ? 1 : 0);
+  return k < F::kLo ? F::kLo : (k > F::kHi ? F::kHi : k);
+}
+
+// Fake-quantize 8 values already divided by the scale; multiply back by s.
+template <int FMT>
+__device__ __forceinline__ void fake_quant8(float* v, float s) {
+  if constexpr (FMT == MXQ_FMT_FP8) {
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      uint32_t h2 = e4m3x2_to_f16x2(e4m3x2(v[j], v[j + 1]));
+      v[j] = f16lo(h2) * s;  // exact; the sign of zero is kept
+      v[j + 1] = f16hi(h2) * s;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      uint32_t h2 = e2m1x2_to_f16x2(e2m1x2(v[j], v[j + 1]));
+      v[j] = fmaf(f16lo(h2), s, 0.0f);  // exact; zero magnitudes become +0
+      v[j + 1] = fmaf(f16hi(h2), s, 0.0f);
+    }
+  }
+}
+
+template <int DT, int FMT, int LPB>
+__global__ void __launch_bounds__(kThreads)
+quantize_cache_kernel(const void* __restrict__ in, void* __restrict__ out, int64_t n_items) {
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
+       base += stride * kUnroll) {
+    uint32_t bits[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      if (item < n_items) load8<DT>(in, item, bits[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      int64_t item = base + u * stride + lane;
+      bool valid = item < n_items;
+      uint32_t m = 0;
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(bits[u][j]));
+      }
+#pragma unroll
+      for (int o = 1; o < LPB; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (!valid) continue;
+      int k = cache_scale_exp<FMT>(m);
+      float inv = exp2i(-k), s = exp2i(k);
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = elem_to_f32<DT>(bits[u][j]) * inv;  // exact
+      fake_quant8<FMT>(v, s);
+      store8<DT>(out, item, v);
+    }
+  }
+}
+
+// General kernel: any block size, any channel count, any alignment.  One
+// thread per (row, group); the last group of a row may be partial.
+template <int DT>
+__device__ __forceinline__ uint32_t load_elem_bits(const void* p, int64_t i) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) return ((const uint16_t*)p)[i];
+  else return ((const uint32_t*)p)[i];
+}
+template <int DT>
+__device__ __forceinline__ void store_elem(void* p, int64_t i, float v) {
+  if constexpr (DT == kBF16) {
+    ((uint16_t*)p)[i] = pack2<DT>(v, 0.0f) & 0xFFFFu;
+  } else if constexpr (DT == kF16) {
+    ((uint16_t*)p)[i] = pack2<DT>(v, 0.0f) & 0xFFFFu;
+  } else {
+    ((float*)p)[i] = v;
+  }
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kThreads)
+quantize_cache_general_kernel(const void* __restrict__ in, void* __restrict__ out, int64_t rows,
+                              int64_t C, int B) {
+  const int64_t groups_per_row = (C + B - 1) / B;
+  const int64_t n_groups = rows * groups_per_row;
+  for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < n_groups;
+       g += (int64_t)gridDim.x * kThreads) {
+    int64_t r = g / groups_per_row;
+    int64_t c0 = (g % groups_per_row) * B;
+    int64_t c1 = c0 + B < C ? c0 + B : C;
+    uint32_t m = 0;
+    for (int64_t c = c0; c < c1; ++c) m = max(m, mag_as_f32_bits<DT>(load_elem_bits<DT>(in, r * C + c)));
+    int k = cache_scale_exp<FMT>(m);
+    float inv = exp2i(-k), s = exp2i(k);
+    for (int64_t c = c0; c < c1; c += 8) {
+      float v[8];
+      int n = (int)(c1 - c < 8 ? c1 - c : 8);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = j < n ? elem_to_f32<DT>(load_elem_bits<DT>(in, r * C + c + j)) * inv : 0.0f;
+      fake_quant8<FMT>(v, s);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < n) store_elem<DT>(out, r * C + c + j, v[j]);
+    }
+  }
+}
+
+// ------------------------------------------------------------ launchers
+
+static int grid_for(int64_t n_units, int per_block) {
+  int64_t need = (n_units + per_block - 1) / per_block;
+  int64_t cap = (int64_t)num_sms() * (2048 / kThreads);
+  if (need > cap) need = cap;
+  return (int)(need < 1 ? 1 : need);
+}
+
+int launch_mx_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed, void* scales,
+                       cudaStream_t st) {
+  int64_t n_items = rows * (K / 8);
+  int grid = grid_for(n_items, kThreads * kUnroll);
+  auto* p = (uint32_t*)packed;
+  auto* s = (uint8_t*)scales;
+  switch (dt) {
+    case kBF16: mx_quantize_kernel<kBF16><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
+    case kF16: mx_quantize_kernel<kF16><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
+    default: mx_quantize_kernel<kF32><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t K, void* out,
+                         int dt, cudaStream_t st) {
+  int64_t n_items = rows * (K / 8);
+  int grid = grid_for(n_items, kThreads * kUnroll);
+  auto* p = (const uint32_t*)packed;
+  auto* s = (const uint8_t*)scales;
+  switch (dt) {
+    case kBF16: mx_dequantize_kernel<kBF16><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
+    case kF16: mx_dequantize_kernel<kF16><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
+    default: mx_dequantize_kernel<kF32><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+template <int DT, int FMT>
+static void launch_cache_fast(const void* in, void* out, int64_t n_items, int lpb, cudaStream_t st) {
+  int grid = grid_for(n_items, kThreads * kUnroll);
+  switch (lpb) {
+    case 1: quantize_cache_kernel<DT, FMT, 1><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    case 2: quantize_cache_kernel<DT, FMT, 2><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    case 4: quantize_cache_kernel<DT, FMT, 4><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    case 8: quantize_cache_kernel<DT, FMT, 8><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    case 16: quantize_cache_kernel<DT, FMT, 16><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    default: quantize_cache_kernel<DT, FMT, 32><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+  }
+}
+
+template <int DT, int FMT>
+static void launch_cache(const void* in, void* out, int64_t rows, int64_t C, int B, bool fast,
+                         cudaStream_t st) {
+  if (fast) {
+    launch_cache_fast<DT, FMT>(in, out, rows * (C / 8), B / 8, st);
+  } else {
+    int64_t n_groups = rows * ((C + B - 1) / B);
+    quantize_cache_general_kernel<DT, FMT><<<grid_for(n_groups, kThreads), kThreads, 0, st>>>(
+        in, out, rows, C, B);
+  }
+}
+
+template <int DT>
+static void launch_cache_dt(const void* in, void* out, int64_t rows, int64_t C, int fmt, int B,
+                            bool fast, cudaStream_t st) {
+  switch (fmt) {
+    case MXQ_FMT_FP8: launch_cache<DT, MXQ_FMT_FP8>(in, out, rows, C, B, fast, st); break;
+    case MXQ_FMT_MXFP4: launch_cache<DT, MXQ_FMT_MXFP4>(in, out, rows, C, B, fast, st); break;
+    default: launch_cache<DT, MXQ_FMT_NVFP4>(in, out, rows, C, B, fast, st); break;
+  }
+}
+
+int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64_t C, int fmt,
+                          int B, bool fast, cudaStream_t st) {
+  switch (dt) {
+    case kBF16: launch_cache_dt<kBF16>(in, out, rows, C, fmt, B, fast, st); break;
+    case kF16: launch_cache_dt<kF16>(in, out, rows, C, fmt, B, fast, st); break;
+    default: launch_cache_dt<kF32>(in, out, rows, C, fmt, B, fast, st); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+}  // namespace mxq

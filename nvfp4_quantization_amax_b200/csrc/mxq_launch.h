@@ -1,0 +1,23 @@
+// Host-side launcher declarations shared by the ABI layer and the kernel
+// translation units.  Arguments reaching these functions are validated.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+int launch_mx_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed, void* scales,
+                       cudaStream_t st);
+int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t K, void* out,
+                         int dt, cudaStream_t st);
+int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64_t C, int fmt,
+                          int B, bool fast, cudaStream_t st);
+int launch_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
+                      int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
+                      int32_t* dev_status, cudaStream_t st);
+
+}  // namespace mxq

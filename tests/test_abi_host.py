@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/mxq.h declares, and rejects bad arguments before launching anything
+(every call here fails validation or is a no-op, so no GPU is touched)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import nvfp4_quantization_amax_b200 as mxq
+from nvfp4_quantization_amax_b200 import build as mxq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxq.h")
+
+OK, EARG, ESHAPE, EALIGN, EUNSUP = 0, -1, -2, -3, -4
+NULL = None
+BAD = ctypes.c_void_p(0x1001)  # misaligned, never dereferenced
+A1, A2 = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)  # never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    mxq_build.build()
+    return mxq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^(?:int|const char\*)\s+(\w+)\(", text, re.M)
+
+
+def test_header_declares_the_boundary():
+    assert set(declared_functions()) >= {"mx_quantize", "mx_dequantize", "quantize_cache",
+                                         "mxfp4_grouped_mm", "mxq_status_string", "mxq_version"}
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", mxq.lib_path()]).decode()
+    exported = set(re.findall(r"\sT\s(\w+)$", out, re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_library_is_built_for_sm100a_only():
+    assert mxq_build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert "--use_fast_math" not in mxq_build.FLAGS and "-lineinfo" in mxq_build.FLAGS
+
+
+def test_status_strings(L):
+    assert mxq.status_string(0) == "MXQ_OK"
+    assert mxq.status_string(-6) == "MXQ_ERR_BAD_OFFS"
+    assert mxq.status_string(-7) == "MXQ_ERR_TIMEOUT"
+    assert mxq.status_string(-99) == "MXQ_ERR_UNKNOWN"
+    assert L.mxq_version() >= 100
+
+
+def test_mx_quantize_validation(L):
+    assert L.mx_quantize(NULL, 0, 4, 64, NULL, NULL, NULL) == EARG
+    assert L.mx_quantize(A1, 0, 4, 48, A2, A2, NULL) == ESHAPE
+    assert L.mx_quantize(A1, 0, -1, 64, A2, A2, NULL) == ESHAPE
+    assert L.mx_quantize(A1, 7, 4, 64, A2, A2, NULL) == EARG
+    assert L.mx_quantize(BAD, 0, 4, 64, A2, A2, NULL) == EALIGN
+    assert L.mx_quantize(A1, 0, 4, 64, BAD, A2, NULL) == EALIGN
+    assert L.mx_quantize(NULL, 0, 0, 64, NULL, NULL, NULL) == OK  # empty: no-op
+
+
+def test_mx_dequantize_validation(L):
+    assert L.mx_dequantize(NULL, NULL, 4, 64, NULL, 0, NULL) == EARG
+    assert L.mx_dequantize(A1, A2, 4, 40, A1, 0, NULL) == ESHAPE
+    assert L.mx_dequantize(A1, A2, 4, 64, A1, 3, NULL) == EARG
+    assert L.mx_dequantize(BAD, A2, 4, 64, A1, 0, NULL) == EALIGN
+    assert L.mx_dequantize(A1, A2, 4, 64, BAD, 0, NULL) == EALIGN
+    assert L.mx_dequantize(NULL, NULL, 4, 0, NULL, 0, NULL) == OK
+
+
+def test_quantize_cache_validation(L):
+    assert L.quantize_cache(NULL, NULL, 0, 4, 64, 0, 32, NULL) == EARG
+    assert L.quantize_cache(A1, A2, 0, 4, 64, 5, 32, NULL) == EARG
+    assert L.quantize_cache(A1, A2, 9, 4, 64, 0, 32, NULL) == EARG
+    assert L.quantize_cache(A1, A2, 0, 4, 64, 0, 0, NULL) == ESHAPE
+    assert L.quantize_cache(A1, A2, 0, -4, 64, 0, 16, NULL) == ESHAPE
+    # the output must be independent storage: overlapping in/out is rejected
+    assert L.quantize_cache(A1, A1, 0, 4, 64, 0, 16, NULL) == EARG
+    assert L.quantize_cache(A1, ctypes.c_void_p(0x10000 + 64), 0, 4, 64, 1, 32, NULL) == EARG
+    assert L.quantize_cache(NULL, NULL, 0, 0, 64, 0, 16, NULL) == OK
+
+
+def test_grouped_mm_validation(L):
+    f = L.mxfp4_grouped_mm
+    assert f(A1, A2, A2, A2, 8, 0, 16, 64, 0, A1, NULL, NULL) == ESHAPE  # E < 1
+    assert f(A1, A2, A2, A2, 8, 2, 16, 48, 0, A1, NULL, NULL) == ESHAPE  # K % 32
+    assert f(A1, A2, A2, A2, 8, 2, 0, 64, 0, A1, NULL, NULL) == ESHAPE  # N < 1
+    assert f(A1, A2, A2, A2, -1, 2, 16, 64, 0, A1, NULL, NULL) == ESHAPE
+    assert f(A1, A2, A2, A2, 8, 2, 16, 64, 2, A1, NULL, NULL) == EARG  # transpose flag
+    assert f(A1, A2, A2, NULL, 8, 2, 16, 64, 0, A1, NULL, NULL) == EARG  # offs
+    assert f(NULL, A2, A2, A2, 8, 2, 16, 64, 0, A1, NULL, NULL) == EARG  # a
+    assert f(A1, A2, A2, A2, 0, 2, 16, 64, 0, A1, NULL, NULL) == OK  # T == 0: no-op
+
+
+def test_binding_fails_loudly_without_gpu():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-only check")
+    with pytest.raises(RuntimeError):
+        mxq.quantize_cache(torch.zeros(4, 32, dtype=torch.bfloat16), "fp8", 32)
