@@ -99,7 +99,7 @@ def special_blocks():
     t8 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
     mids = [(a + b) / 2 for a, b in zip(t8[:-1], t8[1:])]
     rows = []
-    for e in (-133, -127, -126, -20, 0, 3, 100, 125):
+    for e in (-133, -127, -126, -20, 0, 3, 100, 124):  # 8 * 2^124 stays finite
         for sgn in (1.0, -1.0):
             blk = [6.0] + [m * sgn for m in mids] + [(m + 1e-3) * sgn for m in mids] + \
                   [(m - 1e-3) * sgn for m in mids] + [7.0 * sgn, -0.0, 0.0, 5.9 * sgn, 1e-3 * sgn,
