@@ -112,7 +112,7 @@ class ClockSampler:
     def __enter__(self):
         cmd = ["nvidia-smi", "-i", str(self.index),
                "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-               "--format=csv,noheader,nounits", "-lms", "100"]
+               "--format=csv,noheader,nounits", "-lms", "20"]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
@@ -429,7 +429,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
     ap.add_argument("--no-cpu-baseline", action="store_true")

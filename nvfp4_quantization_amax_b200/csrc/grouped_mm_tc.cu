@@ -7,28 +7,32 @@
 // with W_e[n, k] = E2M1(nibble) * 2^(scale - 127) decoded on the fly from
 // the packed [E, N, K/2] bytes and [E, N, K/32] E8M0 scales.
 //
-// Mapping onto tcgen05 (one CTA per SM, persistent over tiles):
+// Mapping onto tcgen05 (persistent kernel, one CTA per SM):
 //   D[m, j] (f32, TMEM)  +=  A[m, r] (bf16, TMEM)  *  B[j, r] (bf16, smem)
-// with m = an output feature (a weight row n in the forward, a column k in
-// the backward; 128 per tile), j = a token of the expert (256 per tile) and
-// r = the reduction index (64 per pipeline stage).
+// with m an output feature (a weight row n in the forward, a column k in
+// the backward), j a token of the expert and r the reduction index (64 per
+// pipeline stage).  A tile is 128 output features per CTA by up to 256
+// tokens; in the CTA-pair form two SMs of a cluster share one tile of 256
+// output features (tcgen05.mma.cta_group::2), each holding its 128 features
+// in TMEM and half of the tokens in shared memory, so each SM streams half
+// as many activation bytes per MMA.
 //   * B (activations) arrives by TMA, 128-byte swizzled, K-major.
 //   * A (weights) never exists in bf16 outside the SM: dequantization warps
 //     read the packed bytes from global memory, decode them exactly to bf16
 //     in registers and write them straight into TMEM with tcgen05.st.  In
 //     the backward the 8x8 blocks are transposed in registers with
 //     movmatrix first, since TMEM lanes must be the output features k.
-//   * One thread issues tcgen05.mma (M=128, N=256, K=16) and signals stage
-//     release with tcgen05.commit.
+//   * One thread issues tcgen05.mma (K=16 steps; N = the tile's token count
+//     rounded up, so ragged expert tails cost no idle columns) and releases
+//     stages with tcgen05.commit.
 //   * Four epilogue warps drain D (tcgen05.ld), round to bf16, stage the
-//     tile in shared memory and store rows that belong to the expert.
+//     tile in shared memory and store the rows that belong to the expert.
 // Every mbarrier wait is bounded: on a time-out the CTA stops all roles,
 // drains what it issued, frees TMEM and reports MXQ_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <cstdio>
 #include <mutex>
 
 #include "mxq.h"
@@ -47,40 +51,56 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;        // output features per tile (MMA M, TMEM lanes)
+constexpr int kBM = 128;        // output features per CTA (TMEM lanes)
 constexpr int kBN = 256;        // tokens per tile (MMA N)
 constexpr int kBK = 64;         // reduction elements per stage (128 bytes of bf16)
-constexpr int kStages = 4;
 constexpr int kTmemCols = 512;
 constexpr int kDCol = 0;        // accumulator: columns [0, 256)
 constexpr int kACol = 256;      // A stages: 32 columns (64 bf16) each
+constexpr int kMaxStages = 8;   // TMEM holds up to eight A stages
 constexpr int kEpiWarps = 4;    // warps 0..3
 constexpr int kDqWarps = 8;     // warps 4..11
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kThreads = 14 * 32;
-constexpr uint32_t kStageBytesB = kBN * kBK * 2;    // 32 KB
 constexpr uint32_t kStagingBytes = kBN * kBM * 2;   // 64 KB
-constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytesB + kStagingBytes + 256;
-constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
+constexpr int kMaxSmemExperts = 4096;               // offs cached in smem up to this E
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
+template <bool kPair>
+struct Geo {
+  static constexpr int kCG = kPair ? 2 : 1;
+  static constexpr int kTileM = kBM * kCG;            // output features per tile
+  static constexpr int kRowsB = kBN / kCG;            // token rows per CTA per stage
+  static constexpr uint32_t kStageBytes = kRowsB * kBK * 2;
+  // One B stage per A stage: 8 x 16 KB per CTA in pairs, 4 x 32 KB alone.
+  static constexpr int kStages = kPair ? 8 : 4;
+  static constexpr uint32_t kSmem =
+      1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
+  // Token count of a tile rounded to what the MMA accepts.
+  __host__ __device__ static int64_t mma_n(int64_t rows) {
+    return kPair ? (rows + 31) & ~31 : (rows + 15) & ~15;
+  }
+};
+
 struct Shared {
-  uint64_t full_a[kStages];
-  uint64_t full_b[kStages];
-  uint64_t empty[kStages];
+  uint64_t full_a[kMaxStages];
+  uint64_t full_b[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t d_full, d_empty, drain;
   uint32_t tmem_base;
   int abort;
 };
 
-// Two E2M1 codes (one byte) -> two exact bf16 values times 2^(s-127).
+// Two E2M1 codes (one byte) -> two bf16 values times the block scale
+// 2^(s-127): exact E2M1 -> f16 (cvt), exact f32 products, one rounding to
+// bf16 that is exact whenever the weight is a normal bf16 value.
+__device__ __forceinline__ float scale_f32(uint32_t s) { return exp2i((int)s - 127); }
+
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t byte, float scale) {
-  uint32_t h2 = e2m1x2_to_f16x2(byte);
+  const uint32_t h2 = e2m1x2_to_f16x2(byte);
   return pack2<kBF16>(f16lo(h2) * scale, f16hi(h2) * scale);
 }
-
-__device__ __forceinline__ float e8m0_scale(uint32_t s) { return exp2i((int)s - 127); }
 
 __device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
@@ -103,50 +123,80 @@ __device__ __forceinline__ bool epi_any(bool pred) {
   return r != 0;
 }
 
-// Bounded wait whose outcome is the same on every lane of the warp (the
-// tcgen05 ld/st that follow are warp-collective).
+// Bounded wait (the same form whether or not the peer CTA arrives too).
+template <bool kPair>
+__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                      uint64_t limit_ns) {
+  return mbar_wait(bar, parity, abort, limit_ns);
+}
+
+// Same outcome on every lane of the warp (the tcgen05 ld/st that follow
+// are warp-collective).
+template <bool kPair>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
-  bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  const bool ok = bwait<kPair>(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
-template <bool kDgrad>
+// Arrive on the even CTA's copy of a barrier (a local arrive when unpaired).
+template <bool kPair>
+__device__ __forceinline__ void arrive_leader(uint64_t* bar) {
+  if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_addr(bar), 0));
+  else mbar_arrive(bar);
+}
+
+template <bool kDgrad, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t* __restrict__ packed,
                      const uint8_t* __restrict__ scales, const int32_t* __restrict__ offs, int64_t T,
                      int64_t E, int64_t N, int64_t K, __nv_bfloat16* __restrict__ y,
                      int32_t* dev_status, uint64_t wait_limit_ns) {
+  using G = Geo<kPair>;
+  constexpr int S = G::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = smem;
-  uint16_t* sY = (uint16_t*)(smem + kStages * kStageBytesB);
-  Shared* sh = (Shared*)(smem + kStages * kStageBytesB + kStagingBytes);
+  uint16_t* sY = (uint16_t*)(smem + S * G::kStageBytes);
+  Shared* sh = (Shared*)((uint8_t*)sY + kStagingBytes);
+  int32_t* s_offs = (int32_t*)((uint8_t*)sh + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;  // 0 leads the pair
+  const int64_t unit = kPair ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
+  const int64_t units = kPair ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+
+  // Both CTAs of a pair read the same offs, so both leave here together.
   if (!offs_valid(offs, E, T)) {
     if (blockIdx.x == 0 && threadIdx.x == 0 && dev_status) *dev_status = MXQ_ERR_BAD_OFFS;
     return;
   }
+  // Tile walks read the expert partition from shared memory when it fits.
+  const int32_t* t_offs = offs;
+  if (E <= kMaxSmemExperts) {
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) s_offs[e] = offs[e];
+    t_offs = s_offs;
+  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh->full_a[s], kDqWarps);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&sh->full_a[s], kDqWarps * G::kCG);
       mbar_init(&sh->full_b[s], 1);
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->d_full, 1);
-    mbar_init(&sh->d_empty, kEpiWarps);
+    mbar_init(&sh->d_empty, kEpiWarps * G::kCG);
     mbar_init(&sh->drain, 1);
     sh->abort = 0;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&sh->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_cg<G::kCG>(&sh->tmem_base, kTmemCols);
+    tmem_relinquish_cg<G::kCG>();
   }
   if (warp == kTmaWarp && lane == 0) prefetch_tmap(&tmap_act);
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
 
   const uint32_t tmem = sh->tmem_base;
@@ -154,67 +204,92 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
   const int64_t kin = kDgrad ? N : K;
   const int64_t nout = kDgrad ? K : N;
   const int nk = (int)(kin / kBK);
-  const int64_t col_tiles = nout / kBM;
+  const int64_t col_tiles = nout / G::kTileM;
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------ TMA producer (B)
     if (lane == 0) {
-      TileWalker walk(offs, E, kBN, col_tiles);
+      TileWalker walk(t_offs, E, kBN, col_tiles);
       uint32_t it = 0;
-      for (int64_t tile = blockIdx.x; !*abort && walk.seek(tile); tile += gridDim.x) {
+      for (int64_t tile = unit; !*abort && walk.seek(tile); tile += units) {
+        const int64_t rows = walk.row_end - walk.row0 < kBN ? walk.row_end - walk.row0 : kBN;
+        // this CTA's share of the tile's tokens
+        const int32_t yrow = (int32_t)(walk.row0 + rank * (G::mma_n(rows) / 2));
         for (int ks = 0; ks < nk; ++ks, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)) break;
-          mbar_arrive_expect_tx(&sh->full_b[s], kStageBytesB);
-          tma_load_2d(smem_addr(sB + s * kStageBytesB), &tmap_act, ks * kBK, (int32_t)walk.row0,
-                      &sh->full_b[s]);
+          const int s = it % S;
+          if (!bwait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)) break;
+          if constexpr (kPair) {
+            if (rank == 0) mbar_arrive_expect_tx(&sh->full_b[s], 2 * G::kStageBytes);
+            tma_load_2d_pair(smem_addr(sB + s * G::kStageBytes), &tmap_act, ks * kBK, yrow,
+                             mapa_shared(smem_addr(&sh->full_b[s]), 0));
+          } else {
+            mbar_arrive_expect_tx(&sh->full_b[s], G::kStageBytes);
+            tma_load_2d(smem_addr(sB + s * G::kStageBytes), &tmap_act, ks * kBK, yrow,
+                        &sh->full_b[s]);
+          }
         }
       }
-      // Loads still in flight land before the CTA may exit.
-      int abort_local = 0;
-      for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
-        mbar_wait(&sh->full_b[j % kStages], (j / kStages) & 1, &abort_local, kDrainLimitNs);
+      // Loads still in flight land before the CTA may exit (the even CTA's
+      // barrier counts both CTAs' bytes).
+      if (rank == 0) {
+        int abort_local = 0;
+        for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
+          bwait<kPair>(&sh->full_b[j % S], (j / S) & 1, &abort_local, kDrainLimitNs);
+      }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      TileWalker walk(offs, E, kBN, col_tiles);
+    if (lane == 0 && rank == 0) {
+      TileWalker walk(t_offs, E, kBN, col_tiles);
       uint32_t it = 0, lt = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x, ++lt) {
-        if (!(ok = mbar_wait(&sh->d_empty, (lt & 1) ^ 1, abort, wait_limit_ns))) break;
+      for (int64_t tile = unit; ok && walk.seek(tile); tile += units, ++lt) {
+        if (!(ok = bwait<kPair>(&sh->d_empty, (lt & 1) ^ 1, abort, wait_limit_ns))) break;
         tc_fence_after();
+        const int64_t rows = walk.row_end - walk.row0 < kBN ? walk.row_end - walk.row0 : kBN;
+        const uint32_t idesc = idesc_bf16_f32(G::kTileM, (int)G::mma_n(rows));
         for (int ks = 0; ks < nk; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!(ok = mbar_wait(&sh->full_a[s], ph, abort, wait_limit_ns))) break;
-          if (!(ok = mbar_wait(&sh->full_b[s], ph, abort, wait_limit_ns))) break;
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!(ok = bwait<kPair>(&sh->full_a[s], ph, abort, wait_limit_ns))) break;
+          if (!(ok = bwait<kPair>(&sh->full_b[s], ph, abort, wait_limit_ns))) break;
           tc_fence_after();
-          const uint64_t bdesc = smem_desc_sw128(smem_addr(sB + s * kStageBytesB));
+          const uint64_t bdesc = smem_desc_sw128(smem_addr(sB + s * G::kStageBytes));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16_ts(tmem + kDCol, tmem + kACol + 32 * s + 8 * kk, bdesc + 2 * kk, kIdesc,
-                        (ks | kk) != 0);
-          mma_commit(&sh->empty[s]);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            if constexpr (kPair)
+              mma_bf16_ts_pair(tmem + kDCol, tmem + kACol + 32 * s + 8 * kk, bdesc + 2 * kk, idesc,
+                               (ks | kk) != 0);
+            else
+              mma_bf16_ts(tmem + kDCol, tmem + kACol + 32 * s + 8 * kk, bdesc + 2 * kk, idesc,
+                          (ks | kk) != 0);
+          }
+          if constexpr (kPair) mma_commit_pair(&sh->empty[s]);
+          else mma_commit(&sh->empty[s]);
         }
-        if (ok) mma_commit(&sh->d_full);
+        if (ok) {
+          if constexpr (kPair) mma_commit_pair(&sh->d_full);
+          else mma_commit(&sh->d_full);
+        }
       }
       // Every MMA issued has completed before TMEM is released.
-      mma_commit(&sh->drain);
+      if constexpr (kPair) mma_commit_pair(&sh->drain);
+      else mma_commit(&sh->drain);
       int abort_local = 0;
       mbar_wait(&sh->drain, 0, &abort_local, kDrainLimitNs);
     }
     __syncwarp();
   } else if (warp >= kEpiWarps) {
     // -------------------------------------------- dequantization (A)
-    const int q = warp & 3;          // TMEM lane quarter
-    const int h = (warp - kEpiWarps) >> 2;  // which half of the 64-wide stage
-    TileWalker walk(offs, E, kBN, col_tiles);
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int h = (warp - kEpiWarps) >> 2;   // which half of the 64-wide stage
+    TileWalker walk(t_offs, E, kBN, col_tiles);
     uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; !*abort && walk.seek(tile); tile += gridDim.x) {
+    bool ok = true;
+    for (int64_t tile = unit; ok && walk.seek(tile); tile += units) {
       const int64_t e = walk.expert;
-      const int64_t m0 = walk.col_tile * kBM;
+      const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;  // this CTA's features
       if constexpr (!kDgrad) {
         // Thread = weight row n; 32 consecutive k per stage half.
         const int64_t n = m0 + 32 * q + lane;
@@ -228,14 +303,13 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
             pb[j] = ldg16(prow + 32 * j);
             sb[j] = srow[2 * j];
           }
-        bool ok = true;
         for (int ks0 = 0; ks0 < nk && ok; ks0 += 4) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int ks = ks0 + j;
             if (ks >= nk || !ok) break;
             const uint4 d = pb[j];
-            const float sc = e8m0_scale(sb[j]);
+            const float sc = scale_f32(sb[j]);
             if (ks + 4 < nk) {
               pb[j] = ldg16(prow + 32 * (ks + 4));
               sb[j] = srow[2 * (ks + 4)];
@@ -243,16 +317,17 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
             uint32_t v[16];
             const uint32_t w[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
-            const int s = it % kStages;
-            if (!(ok = warp_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
+            for (int i = 0; i < 16; ++i)
+              v[i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
+            const int s = it % S;
+            if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
               break;
             tc_fence_after();
             tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + kACol + 32 * s + 16 * h, v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh->full_a[s]);
+            if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
             ++it;
           }
         }
@@ -267,17 +342,16 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
         const uint8_t* scol = scales + e * N * (K / 32) + kq / 32;
         uint4 pb[2][4];
         uint32_t sb[2][4];
-        auto load = [&](int ks, uint4* P, uint32_t* S) {
+        auto load = [&](int ks, uint4* P, uint32_t* Sc) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int64_t n = (int64_t)ks * kBK + 32 * h + 8 * j + rsub;
             P[j] = ldg16(pcol + n * (K / 2));
-            S[j] = scol[n * (K / 32)];
+            Sc[j] = scol[n * (K / 32)];
           }
         };
         load(0, pb[0], sb[0]);
         if (nk > 1) load(1, pb[1], sb[1]);
-        bool ok = true;
         for (int ks0 = 0; ks0 < nk && ok; ks0 += 2) {
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
@@ -286,7 +360,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
             uint32_t v[2][8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float sc = e8m0_scale(sb[u][j]);
+              const float sc = scale_f32(sb[u][j]);
               const uint32_t w[4] = {pb[u][j].x, pb[u][j].y, pb[u][j].z, pb[u][j].w};
 #pragma unroll
               for (int r = 0; r < 2; ++r)
@@ -297,8 +371,8 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
                 }
             }
             if (ks + 2 < nk) load(ks + 2, pb[u], sb[u]);
-            const int s = it % kStages;
-            if (!(ok = warp_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
+            const int s = it % S;
+            if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
               break;
             tc_fence_after();
 #pragma unroll
@@ -308,7 +382,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh->full_a[s]);
+            if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
             ++it;
           }
         }
@@ -316,45 +390,48 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    TileWalker walk(offs, E, kBN, col_tiles);
+    TileWalker walk(t_offs, E, kBN, col_tiles);
     uint32_t lt = 0;
-    for (int64_t tile = blockIdx.x; walk.seek(tile); tile += gridDim.x, ++lt) {
-      // (also: the previous tile's staged rows have been stored)
+    for (int64_t tile = unit; walk.seek(tile); tile += units, ++lt) {
+      // (also orders the previous tile's staging reads before new writes)
       if (epi_any(*abort != 0)) break;
-      const bool ok = mbar_wait(&sh->d_full, lt & 1, abort, wait_limit_ns);
+      const bool ok = bwait<kPair>(&sh->d_full, lt & 1, abort, wait_limit_ns);
       if (epi_any(!ok)) break;
       tc_fence_after();
-      const int col = 32 * warp + lane;  // output feature within the tile
+      const int64_t row0 = walk.row0;
+      const int64_t rows = walk.row_end - row0 < kBN ? walk.row_end - row0 : kBN;
+      const int col = 32 * warp + lane;  // output feature within this CTA's 128
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < (int)((rows + 31) / 32); ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          sY[(32 * c + j) * kBM + col] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+        for (int j = 0; j < 32; j += 2) {
+          const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+          sY[(32 * c + j) * kBM + col] = (uint16_t)(pr & 0xFFFFu);
+          sY[(32 * c + j + 1) * kBM + col] = (uint16_t)(pr >> 16);
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->d_empty);
+      if (lane == 0) arrive_leader<kPair>(&sh->d_empty);
       epi_bar();  // the whole tile is staged
-      const int64_t row0 = walk.row0;
-      const int64_t rows = walk.row_end - row0 < kBN ? walk.row_end - row0 : kBN;
-      const int64_t o0 = walk.col_tile * kBM;
+      __nv_bfloat16* yt = y + row0 * nout + walk.col_tile * G::kTileM + rank * kBM;
       // two rows of 128 outputs (256 bytes each) per warp instruction
       for (int r = 2 * warp + (lane >> 4); r < rows; r += 2 * kEpiWarps) {
         const uint4 val = *reinterpret_cast<const uint4*>(sY + r * kBM + 8 * (lane & 15));
-        *reinterpret_cast<uint4*>(y + (row0 + r) * nout + o0 + 8 * (lane & 15)) = val;
+        *reinterpret_cast<uint4*>(yt + (int64_t)r * nout + 8 * (lane & 15)) = val;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // no peer still uses this CTA's TMEM or barriers
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_cg<G::kCG>(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort && dev_status) atomicExch(dev_status, MXQ_ERR_TIMEOUT);
 }
@@ -380,14 +457,14 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Row-major bf16 [rows, cols] activations, boxes of 64 columns x 256 rows,
-// 128-byte swizzle; rows past the end read as zero.
-bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols) {
+// Row-major bf16 [rows, cols] activations, boxes of 64 columns x box_rows
+// rows, 128-byte swizzle; rows past the end read as zero.
+bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {kBK, kBN};
+  cuuint32_t box[2] = {kBK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -396,26 +473,41 @@ bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
 
 uint64_t g_wait_limit_ns = 2000000000ull;
 
-template <bool kDgrad>
+template <bool kDgrad, bool kPair>
 int launch_tc(const void* a, const void* packed, const void* scales, const int32_t* offs,
               int64_t T, int64_t E, int64_t N, int64_t K, void* y, int32_t* dev_status,
               cudaStream_t st) {
+  using G = Geo<kPair>;
   const int64_t kin = kDgrad ? N : K, nout = kDgrad ? K : N;
   CUtensorMap map;
-  if (!make_act_map(&map, a, T, kin)) return MXQ_ERR_CUDA;
+  if (!make_act_map(&map, a, T, kin, G::kRowsB)) return MXQ_ERR_CUDA;
+  auto kernel = grouped_mm_tc_kernel<kDgrad, kPair>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_mm_tc_kernel<kDgrad>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
   });
   if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
-  int64_t tiles = ((T + kBN - 1) / kBN + E) * (nout / kBM);
-  int64_t grid = tiles < num_sms() ? tiles : num_sms();
-  grouped_mm_tc_kernel<kDgrad><<<(int)grid, kThreads, kSmemBytes, st>>>(
-      map, (const uint8_t*)packed, (const uint8_t*)scales, offs, T, E, N, K, (__nv_bfloat16*)y,
-      dev_status, g_wait_limit_ns);
-  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+  // Upper bound on the tile count: every expert may add one ragged tile.
+  const int64_t tiles = ((T + kBN - 1) / kBN + E) * (nout / G::kTileM);
+  const int64_t slots = num_sms() / G::kCG;
+  const int64_t units = tiles < slots ? tiles : slots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units * G::kCG), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = G::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G::kCG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, map, (const uint8_t*)packed,
+                                       (const uint8_t*)scales, offs, T, E, N, K,
+                                       (__nv_bfloat16*)y, dev_status, g_wait_limit_ns);
+  return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 }  // namespace
@@ -428,12 +520,15 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
   const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
   const bool tc = kin % kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
                   ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31;
-  if (tc) {
-    return transpose_w ? launch_tc<true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
-                       : launch_tc<false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
-  }
-  return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
-                                   dev_status, st);
+  if (!tc)
+    return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
+                                     dev_status, st);
+  const bool pair = nout % (2 * kBM) == 0 && num_sms() >= 2;
+  if (transpose_w)
+    return pair ? launch_tc<true, true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
+                : launch_tc<true, false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
+  return pair ? launch_tc<false, true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
+              : launch_tc<false, false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
 }
 
 }  // namespace mxq

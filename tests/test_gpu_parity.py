@@ -223,18 +223,18 @@ def test_cache_idempotent_on_gpu():
 
 # ------------------------------------------------------- grouped GEMM
 
-def moe_case(counts, N, K, seed=21):
+def moe_case(counts, N, K, seed=21, scale_lo=116, scale_hi=124):
     E = len(counts)
     offs = torch.tensor(np.cumsum(counts), dtype=torch.int32)
     T = int(offs[-1])
-    packed, scales = gen.random_packed(E, N, K, 116, 124, workload=seed)
+    packed, scales = gen.random_packed(E, N, K, scale_lo, scale_hi, workload=seed)
     x = gen.normal_bf16(gen.seed_for(seed, 3), (T, K))
     g = gen.normal_bf16(gen.seed_for(seed, 4), (T, N))
     return x, g, packed, scales, offs
 
 
-def check_gemm(counts, N, K, transpose_w, rows=None, seed=21):
-    x, g, packed, scales, offs = moe_case(counts, N, K, seed)
+def check_gemm(counts, N, K, transpose_w, rows=None, seed=21, scale_lo=116, scale_hi=124):
+    x, g, packed, scales, offs = moe_case(counts, N, K, seed, scale_lo, scale_hi)
     a = g if transpose_w else x
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     y = mxq.mxfp4_grouped_mm(a.to(DEV), packed.to(DEV), scales.to(DEV), offs.to(DEV),
@@ -255,6 +255,20 @@ def check_gemm(counts, N, K, transpose_w, rows=None, seed=21):
 def test_grouped_mm_ragged_experts(transpose_w):
     # several tiles, ragged tails, an empty expert and a one-row expert
     check_gemm([300, 0, 1, 257, 130, 512], N=256, K=512, transpose_w=transpose_w)
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_scales_across_decoder_paths(transpose_w):
+    # scale bytes 136..150 straddle the two weight-decoding paths (<= 142 and above)
+    check_gemm([129, 64, 300], N=256, K=256, transpose_w=transpose_w, scale_lo=136,
+               scale_hi=150)
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_many_small_experts(transpose_w):
+    # 40 experts of 0..40 rows: every tail width, many tiles per CTA
+    counts = [(7 * i) % 41 for i in range(40)]
+    check_gemm(counts, N=128, K=128, transpose_w=transpose_w)
 
 
 @pytest.mark.parametrize("transpose_w", [False, True])
