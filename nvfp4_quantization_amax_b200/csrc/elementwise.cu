@@ -23,6 +23,55 @@ namespace mxq {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 
+// Eight consecutive elements as raw bits: one 16-byte vector for bf16/f16,
+// two for f32.
+template <int DT>
+struct Raw8 {
+  uint4 a, b;
+};
+
+template <int DT>
+__device__ __forceinline__ Raw8<DT> load_raw8(const void* base, int64_t item) {
+  Raw8<DT> r;
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    r.a = ld_stream_v4((const char*)base + item * 16);
+  } else {
+    r.a = ld_stream_v4((const char*)base + item * 32);
+    r.b = ld_stream_v4((const char*)base + item * 32 + 16);
+  }
+  return r;
+}
+
+// Bits of element j (0..7).
+template <int DT>
+__device__ __forceinline__ uint32_t raw_elem(const Raw8<DT>& r, int j) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    const uint32_t w = j < 2 ? r.a.x : j < 4 ? r.a.y : j < 6 ? r.a.z : r.a.w;
+    return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+  } else {
+    const uint4& q = j < 4 ? r.a : r.b;
+    const int k = j & 3;
+    return k == 0 ? q.x : k == 1 ? q.y : k == 2 ? q.z : q.w;
+  }
+}
+
+// f32 bit pattern of max |x| over the eight elements.  For 16-bit formats
+// the magnitudes are compared pairwise as unsigned halves (monotone in |x|
+// for finite values).
+template <int DT>
+__device__ __forceinline__ uint32_t raw_amax(const Raw8<DT>& r) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    const uint32_t M = 0x7FFF7FFFu;
+    const uint32_t m2 = __vmaxu2(__vmaxu2(r.a.x & M, r.a.y & M), __vmaxu2(r.a.z & M, r.a.w & M));
+    return mag_as_f32_bits<DT>(max(m2 & 0xFFFFu, m2 >> 16));
+  } else {
+    const uint32_t M = 0x7FFFFFFFu;
+    const uint32_t m = max(max(max(r.a.x & M, r.a.y & M), max(r.a.z & M, r.a.w & M)),
+                           max(max(r.b.x & M, r.b.y & M), max(r.b.z & M, r.b.w & M)));
+    return m;
+  }
+}
+
 // ---------------------------------------------------------- mx_quantize
 
 // Scale exponent of quantize_mxfp4 from the f32 bit pattern of a block's
@@ -41,36 +90,29 @@ mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kUnroll) {
-    uint32_t bits[kUnroll][8];
+    Raw8<DT> raw[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      if (item < n_items) load8<DT>(x, item, bits[u]);
+      const int64_t item = base + u * stride + lane;
+      if (item < n_items) raw[u] = load_raw8<DT>(x, item);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      bool valid = item < n_items;
-      // Block amax on magnitude bit patterns (monotone in |x| for finite x).
-      uint32_t m = 0;
-      if (valid) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(bits[u][j]));
-      }
+      const int64_t item = base + u * stride + lane;
+      const bool valid = item < n_items;
+      // Block amax over the four lanes that hold one 32-element block.
+      uint32_t m = valid ? raw_amax<DT>(raw[u]) : 0u;
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (!valid) continue;
-      int e = mx_scale_exp(m);
-      float inv = exp2i(-e);  // exact power of two
+      const int e = mx_scale_exp(m);
+      const float inv = exp2i(-e);  // exact power of two
       float v[8];
+      // x * 2^-e is exact; adding +0 in the same rounding turns -0.0 into
+      // +0.0 (no sign bit for it) while a negative value that underflows
+      // keeps its sign, so the code's sign bit is set iff x < 0.
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t b = bits[u][j];
-        // -0.0 carries no sign into the code; any other negative does.
-        uint32_t negzero = (DT == kF32) ? 0x80000000u : 0x8000u;
-        if (b == negzero) b = 0;
-        v[j] = elem_to_f32<DT>(b) * inv;  // exact: power-of-two scaling
-      }
+      for (int j = 0; j < 8; ++j) v[j] = fmaf(elem_to_f32<DT>(raw_elem<DT>(raw[u], j)), inv, 0.0f);
       packed[item] = e2m1x8(v);
       if ((lane & 3) == 0) scales[item >> 2] = (uint8_t)(e + 127);
     }
@@ -182,29 +224,25 @@ quantize_cache_kernel(const void* __restrict__ in, void* __restrict__ out, int64
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kUnroll) {
-    uint32_t bits[kUnroll][8];
+    Raw8<DT> raw[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      if (item < n_items) load8<DT>(in, item, bits[u]);
+      const int64_t item = base + u * stride + lane;
+      if (item < n_items) raw[u] = load_raw8<DT>(in, item);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      bool valid = item < n_items;
-      uint32_t m = 0;
-      if (valid) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(bits[u][j]));
-      }
+      const int64_t item = base + u * stride + lane;
+      const bool valid = item < n_items;
+      uint32_t m = valid ? raw_amax<DT>(raw[u]) : 0u;
 #pragma unroll
       for (int o = 1; o < LPB; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (!valid) continue;
-      int k = cache_scale_exp<FMT>(m);
-      float inv = exp2i(-k), s = exp2i(k);
+      const int k = cache_scale_exp<FMT>(m);
+      const float inv = exp2i(-k), s = exp2i(k);
       float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = elem_to_f32<DT>(bits[u][j]) * inv;  // exact
+      for (int j = 0; j < 8; ++j) v[j] = elem_to_f32<DT>(raw_elem<DT>(raw[u], j)) * inv;  // exact
       fake_quant8<FMT>(v, s);
       store8<DT>(out, item, v);
     }

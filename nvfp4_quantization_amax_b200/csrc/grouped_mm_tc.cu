@@ -53,11 +53,11 @@ using namespace sm100;
 
 constexpr int kBM = 128;        // output features per CTA (TMEM lanes)
 constexpr int kBN = 256;        // tokens per tile (MMA N)
-constexpr int kBK = 64;         // reduction elements per stage (128 bytes of bf16)
+constexpr int kBox = 64;        // reduction elements per TMA box (128 bytes of bf16)
 constexpr int kTmemCols = 512;
 constexpr int kDCol = 0;        // accumulator: columns [0, 256)
-constexpr int kACol = 256;      // A stages: 32 columns (64 bf16) each
-constexpr int kMaxStages = 8;   // TMEM holds up to eight A stages
+constexpr int kACol = 256;      // A stages follow the accumulator
+constexpr int kMaxStages = 4;
 constexpr int kEpiWarps = 4;    // warps 0..3
 constexpr int kDqWarps = 8;     // warps 4..11
 constexpr int kTmaWarp = 12;
@@ -72,9 +72,16 @@ struct Geo {
   static constexpr int kCG = kPair ? 2 : 1;
   static constexpr int kTileM = kBM * kCG;            // output features per tile
   static constexpr int kRowsB = kBN / kCG;            // token rows per CTA per stage
-  static constexpr uint32_t kStageBytes = kRowsB * kBK * 2;
-  // One B stage per A stage: 8 x 16 KB per CTA in pairs, 4 x 32 KB alone.
-  static constexpr int kStages = kPair ? 8 : 4;
+  // Reduction depth of a stage: 128 in pairs (fewer, larger hand-offs
+  // between the dequantization warps and the MMA), 64 alone.
+  static constexpr int kBK = kPair ? 128 : 64;
+  static constexpr int kBoxes = kBK / kBox;           // TMA boxes per stage
+  static constexpr uint32_t kBoxBytes = kRowsB * kBox * 2;
+  static constexpr uint32_t kStageBytes = kBoxes * kBoxBytes;
+  static constexpr int kACols = kBK / 2;              // TMEM columns per A stage
+  // One B stage per A stage; 4 x 32 KB of activations per CTA either way,
+  // and 4 A stages of at most 64 columns beside the 256 accumulator columns.
+  static constexpr int kStages = 4;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
   // Token count of a tile rounded to what the MMA accepts.
@@ -203,6 +210,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
   volatile int* abort = &sh->abort;
   const int64_t kin = kDgrad ? N : K;
   const int64_t nout = kDgrad ? K : N;
+  constexpr int kBK = G::kBK;
   const int nk = (int)(kin / kBK);
   const int64_t col_tiles = nout / G::kTileM;
 
@@ -220,12 +228,17 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
           if (!bwait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)) break;
           if constexpr (kPair) {
             if (rank == 0) mbar_arrive_expect_tx(&sh->full_b[s], 2 * G::kStageBytes);
-            tma_load_2d_pair(smem_addr(sB + s * G::kStageBytes), &tmap_act, ks * kBK, yrow,
-                             mapa_shared(smem_addr(&sh->full_b[s]), 0));
+            const uint32_t bar = mapa_shared(smem_addr(&sh->full_b[s]), 0);
+#pragma unroll
+            for (int b = 0; b < G::kBoxes; ++b)
+              tma_load_2d_pair(smem_addr(sB + s * G::kStageBytes + b * G::kBoxBytes), &tmap_act,
+                               ks * kBK + b * kBox, yrow, bar);
           } else {
             mbar_arrive_expect_tx(&sh->full_b[s], G::kStageBytes);
-            tma_load_2d(smem_addr(sB + s * G::kStageBytes), &tmap_act, ks * kBK, yrow,
-                        &sh->full_b[s]);
+#pragma unroll
+            for (int b = 0; b < G::kBoxes; ++b)
+              tma_load_2d(smem_addr(sB + s * G::kStageBytes + b * G::kBoxBytes), &tmap_act,
+                          ks * kBK + b * kBox, yrow, &sh->full_b[s]);
           }
         }
       }
@@ -258,12 +271,13 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
           const uint64_t bdesc = smem_desc_sw128(smem_addr(sB + s * G::kStageBytes));
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
+            // K16 step kk: box kk/4, 32-byte column offset kk%4 inside it
+            const uint64_t bd = bdesc + (uint64_t)(((kk >> 2) * G::kBoxBytes) >> 4) + 2 * (kk & 3);
+            const uint32_t a = tmem + kACol + G::kACols * s + 8 * kk;
             if constexpr (kPair)
-              mma_bf16_ts_pair(tmem + kDCol, tmem + kACol + 32 * s + 8 * kk, bdesc + 2 * kk, idesc,
-                               (ks | kk) != 0);
+              mma_bf16_ts_pair(tmem + kDCol, a, bd, idesc, (ks | kk) != 0);
             else
-              mma_bf16_ts(tmem + kDCol, tmem + kACol + 32 * s + 8 * kk, bdesc + 2 * kk, idesc,
-                          (ks | kk) != 0);
+              mma_bf16_ts(tmem + kDCol, a, bd, idesc, (ks | kk) != 0);
           }
           if constexpr (kPair) mma_commit_pair(&sh->empty[s]);
           else mma_commit(&sh->empty[s]);
@@ -291,39 +305,58 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
       const int64_t e = walk.expert;
       const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;  // this CTA's features
       if constexpr (!kDgrad) {
-        // Thread = weight row n; 32 consecutive k per stage half.
+        // Thread = weight row n; kBK/2 consecutive k (kBK/4 bytes, one or
+        // two 16-byte loads, one scale per 32 k) per stage half.
+        constexpr int kV = kBK / 64;  // 16-byte loads per thread per stage
         const int64_t n = m0 + 32 * q + lane;
-        const uint8_t* prow = packed + (e * N + n) * (K / 2) + 16 * h;
-        const uint8_t* srow = scales + (e * N + n) * (K / 32) + h;
-        uint4 pb[4];
-        uint32_t sb[4];
+        const uint8_t* prow = packed + (e * N + n) * (K / 2) + (kBK / 4) * h;
+        const uint8_t* srow = scales + (e * N + n) * (K / 32) + kV * h;
+        uint4 pb[4][kV];
+        uint32_t sb[4][kV];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (j < nk) {
-            pb[j] = ldg16(prow + 32 * j);
-            sb[j] = srow[2 * j];
+#pragma unroll
+            for (int c = 0; c < kV; ++c) {
+              pb[j][c] = ldg16(prow + (kBK / 2) * j + 16 * c);
+              sb[j][c] = srow[(kBK / 32) * j + c];
+            }
           }
         for (int ks0 = 0; ks0 < nk && ok; ks0 += 4) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int ks = ks0 + j;
             if (ks >= nk || !ok) break;
-            const uint4 d = pb[j];
-            const float sc = scale_f32(sb[j]);
-            if (ks + 4 < nk) {
-              pb[j] = ldg16(prow + 32 * (ks + 4));
-              sb[j] = srow[2 * (ks + 4)];
-            }
-            uint32_t v[16];
-            const uint32_t w[4] = {d.x, d.y, d.z, d.w};
+            uint4 d[kV];
+            float sc[kV];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              v[i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
+            for (int c = 0; c < kV; ++c) {
+              d[c] = pb[j][c];
+              sc[c] = scale_f32(sb[j][c]);
+            }
+            if (ks + 4 < nk) {
+#pragma unroll
+              for (int c = 0; c < kV; ++c) {
+                pb[j][c] = ldg16(prow + (kBK / 2) * (ks + 4) + 16 * c);
+                sb[j][c] = srow[(kBK / 32) * (ks + 4) + c];
+              }
+            }
+            uint32_t v[16 * kV];
+#pragma unroll
+            for (int c = 0; c < kV; ++c) {
+              const uint32_t w[4] = {d[c].x, d[c].y, d[c].z, d[c].w};
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc[c]);
+            }
             const int s = it % S;
             if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
               break;
             tc_fence_after();
-            tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + kACol + 32 * s + 16 * h, v);
+            const uint32_t col = kACol + G::kACols * s + 16 * kV * h;
+#pragma unroll
+            for (int c = 0; c < kV; ++c)
+              tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + col + 16 * c, v + 16 * c);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -333,30 +366,35 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
         }
       } else {
         // Output features k = m0 + 32q + (0..31) are the TMEM lanes of this
-        // warp; each stage half covers 32 reduction indices n.  Thread t
-        // decodes byte (n0 + t/4, k/2 = kq/2 + 8r + 4b + t%4) for its four
-        // rows n0 = base + 8j, then movmatrix transposes each 8x8 block.
+        // warp; a stage half covers kBK/2 reduction indices n, done in
+        // sub-steps of 32.  Thread t decodes byte (n0 + t/4, k/2 = kq/2 + 8r
+        // + 4b + t%4) for its four rows n0 = base + 8j of a sub-step, then
+        // movmatrix transposes each 8x8 block.
+        constexpr int kSub = kBK / 64;  // sub-steps per stage half
         const int64_t kq = m0 + 32 * q;
         const int rsub = lane >> 2, csub = lane & 3;
         const uint8_t* pcol = packed + e * N * (K / 2) + kq / 2;
         const uint8_t* scol = scales + e * N * (K / 32) + kq / 32;
+        const int ng = nk * kSub;  // sub-steps in this tile
         uint4 pb[2][4];
         uint32_t sb[2][4];
-        auto load = [&](int ks, uint4* P, uint32_t* Sc) {
+        auto load = [&](int g, uint4* P, uint32_t* Sc) {
+          const int64_t nbase = (int64_t)(g / kSub) * kBK + (kBK / 2) * h + 32 * (g % kSub);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int64_t n = (int64_t)ks * kBK + 32 * h + 8 * j + rsub;
+            const int64_t n = nbase + 8 * j + rsub;
             P[j] = ldg16(pcol + n * (K / 2));
             Sc[j] = scol[n * (K / 32)];
           }
         };
         load(0, pb[0], sb[0]);
-        if (nk > 1) load(1, pb[1], sb[1]);
-        for (int ks0 = 0; ks0 < nk && ok; ks0 += 2) {
+        if (ng > 1) load(1, pb[1], sb[1]);
+        for (int g0 = 0; g0 < ng && ok; g0 += 2) {
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int ks = ks0 + u;
-            if (ks >= nk || !ok) break;
+            const int g = g0 + u;
+            if (g >= ng || !ok) break;
+            const int sub_i = g % kSub;
             uint32_t v[2][8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -370,20 +408,24 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
                   v[r][2 * j + b] = movmatrix_trans(dequant_pair(byte, sc));
                 }
             }
-            if (ks + 2 < nk) load(ks + 2, pb[u], sb[u]);
+            if (g + 2 < ng) load(g + 2, pb[u], sb[u]);
             const int s = it % S;
-            if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
-              break;
-            tc_fence_after();
+            if (sub_i == 0) {
+              if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
+                break;
+              tc_fence_after();
+            }
+            const uint32_t col = kACol + G::kACols * s + (kBK / 4) * h + 16 * sub_i;
 #pragma unroll
             for (int r = 0; r < 2; ++r)
-              tmem_st_16x128b_x4(tmem + ((uint32_t)(32 * q + 16 * r) << 16) + kACol + 32 * s + 16 * h,
-                                 v[r]);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
-            ++it;
+              tmem_st_16x128b_x4(tmem + ((uint32_t)(32 * q + 16 * r) << 16) + col, v[r]);
+            if (sub_i == kSub - 1) {
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
+              ++it;
+            }
           }
         }
       }
@@ -464,7 +506,7 @@ bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {kBK, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {kBox, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -518,12 +560,12 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                       int32_t* dev_status, cudaStream_t st) {
   const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
-  const bool tc = kin % kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
+  const bool pair = nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2;
+  const bool tc = kin % Geo<false>::kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
                   ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31;
   if (!tc)
     return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
                                      dev_status, st);
-  const bool pair = nout % (2 * kBM) == 0 && num_sms() >= 2;
   if (transpose_w)
     return pair ? launch_tc<true, true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
                 : launch_tc<true, false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
