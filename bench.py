@@ -223,6 +223,17 @@ def time_e2e(torch, mxq, step, steps):
     return dt, h2d, d2h
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def run_gpu(args, rank, world):
     import torch
     import torch.distributed as dist
@@ -261,17 +272,12 @@ def run_gpu(args, rank, world):
         dist.barrier()
     total_ms = start.elapsed_time(stop)
     kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
-    if world > 1:
-        t = torch.tensor([total_ms] + [kern_ms[n] for n in step.names], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        kern_ms = {n: float(v) for n, v in zip(step.names, t[1:])}
+    red = max_over_ranks([total_ms] + [kern_ms[n] for n in step.names], dev)
+    total_ms = red[0]
+    kern_ms = dict(zip(step.names, red[1:]))
 
     e2e_dt, h2d, d2h = time_e2e(torch, mxq, step, max(1, min(args.steps, 3)))
-    if world > 1:
-        t = torch.tensor([e2e_dt], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_dt = float(t[0])
+    e2e_dt = max_over_ranks([e2e_dt], dev)[0]
 
     if rank == 0:
         report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary())

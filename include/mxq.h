@@ -138,6 +138,13 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
                      int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                      int32_t* dev_status, void* stream);
 
+/* Limit, in nanoseconds, after which a pipeline wait inside the grouped GEMM
+ * gives up (the kernel then drains what it issued, frees its tensor memory
+ * and reports MXQ_ERR_TIMEOUT through dev_status).  Default 2e9 (2 s); it
+ * only ever matters if the GPU stops making progress.  Process-wide; applies
+ * to launches made after the call.  Returns the previous limit. */
+uint64_t mxq_set_wait_limit_ns(uint64_t ns);
+
 /* Human-readable name of a status code (static storage). */
 const char* mxq_status_string(int status);
 

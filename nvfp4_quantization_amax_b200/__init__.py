@@ -19,5 +19,6 @@ from ._abi import (  # noqa: F401
     mx_quantize,
     mxfp4_grouped_mm,
     quantize_cache,
+    set_wait_limit_ns,
     status_string,
 )

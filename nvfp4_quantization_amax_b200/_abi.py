@@ -44,12 +44,19 @@ def lib():
         L.mxq_status_string.argtypes = [i]
         L.mxq_version.restype = i
         L.mxq_version.argtypes = []
+        L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64
+        L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
     return _lib
 
 
 def status_string(status):
     return lib().mxq_status_string(int(status)).decode()
+
+
+def set_wait_limit_ns(ns):
+    """Set the grouped GEMM's pipeline-wait limit (ns); returns the previous one."""
+    return int(lib().mxq_set_wait_limit_ns(int(ns)))
 
 
 def _check(rc, what):

@@ -105,6 +105,8 @@ const char* mxq_status_string(int status) {
   }
 }
 
+uint64_t mxq_set_wait_limit_ns(uint64_t ns) { return set_wait_limit_ns(ns); }
+
 int mxq_version(void) { return 100; }
 
 }  // extern "C"

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "mxq.h"
@@ -66,6 +67,7 @@ constexpr int kThreads = 14 * 32;
 constexpr uint32_t kStagingBytes = kBN * kBM * 2;   // 64 KB
 constexpr int kMaxSmemExperts = 4096;               // offs cached in smem up to this E
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
+constexpr uint64_t kAbortSettleNs = 50000ull;
 
 template <bool kPair>
 struct Geo {
@@ -470,7 +472,16 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
 
   tc_fence_before();
   __syncthreads();
-  if constexpr (kPair) cluster_sync();  // no peer still uses this CTA's TMEM or barriers
+  if constexpr (kPair) {
+    // After an abort the odd CTA may still have a TMA load in flight that
+    // counts on the even CTA's barrier; give it time to land (bounded).
+    if (*abort) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < kAbortSettleNs) {
+      }
+    }
+    cluster_sync();  // no peer still uses this CTA's TMEM or barriers
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc_cg<G::kCG>(tmem, kTmemCols);
@@ -513,7 +524,7 @@ bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-uint64_t g_wait_limit_ns = 2000000000ull;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 template <bool kDgrad, bool kPair>
 int launch_tc(const void* a, const void* packed, const void* scales, const int32_t* offs,
@@ -548,13 +559,17 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, map, (const uint8_t*)packed,
                                        (const uint8_t*)scales, offs, T, E, N, K,
-                                       (__nv_bfloat16*)y, dev_status, g_wait_limit_ns);
+                                       (__nv_bfloat16*)y, dev_status, g_wait_limit_ns.load());
   return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 }  // namespace
 
-void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+uint64_t set_wait_limit_ns(uint64_t ns) {
+  const uint64_t prev = g_wait_limit_ns;
+  g_wait_limit_ns = ns;
+  return prev;
+}
 
 int launch_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,

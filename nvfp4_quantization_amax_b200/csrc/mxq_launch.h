@@ -16,6 +16,7 @@ int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, i
                          int dt, cudaStream_t st);
 int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64_t C, int fmt,
                           int B, bool fast, cudaStream_t st);
+uint64_t set_wait_limit_ns(uint64_t ns);
 int launch_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                       int32_t* dev_status, cudaStream_t st);

@@ -28,12 +28,13 @@ def L():
 
 def declared_functions():
     text = open(HEADER).read()
-    return re.findall(r"^(?:int|const char\*)\s+(\w+)\(", text, re.M)
+    return re.findall(r"^(?:int|uint64_t|const char\*)\s+(\w+)\(", text, re.M)
 
 
 def test_header_declares_the_boundary():
     assert set(declared_functions()) >= {"mx_quantize", "mx_dequantize", "quantize_cache",
-                                         "mxfp4_grouped_mm", "mxq_status_string", "mxq_version"}
+                                         "mxfp4_grouped_mm", "mxq_status_string", "mxq_version",
+                                         "mxq_set_wait_limit_ns"}
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -106,3 +107,8 @@ def test_binding_fails_loudly_without_gpu():
         pytest.skip("host-only check")
     with pytest.raises(RuntimeError):
         mxq.quantize_cache(torch.zeros(4, 32, dtype=torch.bfloat16), "fp8", 32)
+
+
+def test_wait_limit_setter_round_trips(L):
+    prev = mxq.set_wait_limit_ns(123)
+    assert mxq.set_wait_limit_ns(prev) == 123

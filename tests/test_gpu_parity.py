@@ -315,3 +315,20 @@ def test_grouped_mm_full_size_sampled(transpose_w):
                             transpose_w=transpose_w, rows=rows)
     yv = oracle.decode(bits(y[torch.tensor(rows, device=DEV)]), "bf16")
     assert gemm_error(yv, ref) <= GEMM_TOL
+
+
+def test_grouped_mm_wait_timeout_reports_status():
+    # A zero wait limit makes the first pipeline wait that is not already
+    # satisfied give up: the kernel must drain, free TMEM and report
+    # MXQ_ERR_TIMEOUT, and the context must stay usable.
+    x, g, packed, scales, offs = moe_case([700, 300, 50], N=128, K=512)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    prev = mxq.set_wait_limit_ns(0)
+    try:
+        mxq.mxfp4_grouped_mm(x.to(DEV), packed.to(DEV), scales.to(DEV), offs.to(DEV),
+                             status=status)
+        torch.cuda.synchronize()
+    finally:
+        mxq.set_wait_limit_ns(prev)
+    assert int(status.item()) == -7
+    check_gemm([700, 300, 50], N=128, K=512, transpose_w=False)
