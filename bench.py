@@ -203,6 +203,34 @@ class Step:
                 ev[i][1].record()
 
 
+def time_next_rows(torch, mxq, step, dev, reps=5):
+    """Device time (ms, mean over reps, max over ranks) of the next-row
+    kernels on the expert weights: NVFP4 two-level quantize and dequantize.
+    Timed after, and outside, the main step."""
+    packed, bscales, g = mxq.nvfp4_quantize(step.W)
+    ws = torch.empty(16, dtype=torch.uint8, device=dev)
+    calls = {
+        "nvfp4_quantize": lambda: mxq.nvfp4_quantize(step.W, packed, bscales, g, ws),
+        "nvfp4_dequantize": lambda: mxq.nvfp4_dequantize(packed, bscales, g, torch.bfloat16,
+                                                         step.Wout),
+    }
+    out = {}
+    for name, fn in calls.items():
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        out[name] = a.elapsed_time(b) / reps
+    names = list(out)
+    vals = max_over_ranks([out[n] for n in names], dev)
+    return dict(zip(names, vals))
+
+
 def time_e2e(torch, mxq, step, steps):
     """Same metric through the public API with host (pinned) buffers: every
     call copies its inputs host->device and its result device->host."""
@@ -278,14 +306,15 @@ def run_gpu(args, rank, world):
 
     e2e_dt, h2d, d2h = time_e2e(torch, mxq, step, max(1, min(args.steps, 3)))
     e2e_dt = max_over_ranks([e2e_dt], dev)[0]
+    next_ms = time_next_rows(torch, mxq, step, dev)
 
     if rank == 0:
-        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary())
+        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary(), next_ms)
     if world > 1:
         dist.destroy_process_group()
 
 
-def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks):
+def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=None):
     peaks, peak_src = load_peaks()
     ab = algorithmic_bytes()
     qd_bytes = ab["mx_quantize"] + ab["mx_dequantize"] + 3 * ab["quantize_cache"]
@@ -355,6 +384,17 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks):
         "gpu_launches": 7 * args.steps,
         "clocks": clocks,
     }
+    if next_ms:
+        w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
+        # quantize: the per-tensor scale needs the whole tensor's maximum
+        # first, so x is read twice; packed codes + E4M3 scales written once
+        nb = {"nvfp4_quantize": 2 * 2 * w + w // 2 + w // 16,
+              "nvfp4_dequantize": w // 2 + w // 16 + 2 * w}
+        line["next_rows"] = {
+            n: {"ms": round(ms, 4), "gbs": round(nb[n] / (ms * 1e-3) / 1e9, 1),
+                "frac": round(nb[n] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "workload": "bf16 [64,2048,7168] expert weights"}
+            for n, ms in next_ms.items()}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     print(json.dumps(line), flush=True)

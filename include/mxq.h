@@ -138,6 +138,41 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
                      int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                      int32_t* dev_status, void* stream);
 
+/* Device workspace nvfp4_quantize needs (bytes, 16-byte aligned). */
+#define MXQ_NVFP4_WORKSPACE_BYTES 16
+
+/* NVFP4 two-level quantize + pack along the last dimension ([MO] "NVFP4 in
+ * the code: two scales and a nibble"; block 16 with E4M3 scales from the
+ * numerics YAML in "mtq.quantize is three moves").
+ *
+ *  x             device, [rows, K] elements of x_dtype, K % 16 == 0, 16-byte
+ *                aligned.
+ *  packed        device, [rows, K/2] bytes (output), 16-byte aligned: E2M1
+ *                codes, low nibble = even column.
+ *  block_scales  device, [rows, K/16] E4M3 bytes (output), one per 16 values.
+ *  global_scale  device, one float (output): g = max|x| / (6 * 448).
+ *  workspace     device, MXQ_NVFP4_WORKSPACE_BYTES bytes of scratch, owned by
+ *                the caller, clobbered; calls that overlap on the GPU must not
+ *                share it.
+ *
+ *  In binary32 arithmetic: g = amax / 2688; per block s_b = E4M3(amax_b /
+ *  (6 g)) after replacing a zero quotient by 1.0 and clamping to [2^-9, 448];
+ *  code = E2M1(x / (s_b * g)) (nearest-even on the grid, saturating at 6,
+ *  sign bit iff x < 0).  An all-zero tensor gives g = 0, codes 0 and block
+ *  scales 1.0.  Precondition: max|x| is 0 or at least 2^-126.
+ *  Errors: K % 16 != 0 -> MXQ_ERR_SHAPE; null -> MXQ_ERR_INVALID_ARG;
+ *  misaligned x/packed/workspace -> MXQ_ERR_ALIGNMENT. */
+int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                   void* block_scales, float* global_scale, void* workspace, void* stream);
+
+/* NVFP4 unpack: out[r][k] = round_dtype(fl32(E2M1(nibble) * s_b * g)) (the
+ * binary32 product, rounded once more to out_dtype).  Nibble 8 gives +0.0.
+ *  packed [rows, K/2] (16-byte aligned), block_scales [rows, K/16] E4M3,
+ *  global_scale device float, out [rows, K] (16-byte aligned).
+ *  Errors as for nvfp4_quantize. */
+int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
+                     int64_t rows, int64_t K, void* out, int out_dtype, void* stream);
+
 /* Limit, in nanoseconds, after which a pipeline wait inside the grouped GEMM
  * gives up (the kernel then drains what it issued, frees its tensor memory
  * and reports MXQ_ERR_TIMEOUT through dev_status).  Default 2e9 (2 s); it

@@ -18,6 +18,8 @@ from ._abi import (  # noqa: F401
     mx_dequantize,
     mx_quantize,
     mxfp4_grouped_mm,
+    nvfp4_dequantize,
+    nvfp4_quantize,
     quantize_cache,
     set_wait_limit_ns,
     status_string,

@@ -44,6 +44,10 @@ def lib():
         L.mxq_status_string.argtypes = [i]
         L.mxq_version.restype = i
         L.mxq_version.argtypes = []
+        L.nvfp4_quantize.restype = i
+        L.nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p, p, p]
+        L.nvfp4_dequantize.restype = i
+        L.nvfp4_dequantize.argtypes = [p, p, p, i64, i64, p, i, p]
         L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64
         L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
@@ -187,4 +191,60 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
     rc = lib().mxfp4_grouped_mm(_ptr(a), _ptr(packed), _ptr(scales), _ptr(offs), T, E, N, K,
                                 1 if transpose_w else 0, _ptr(out), st, _stream(a.device))
     _check(rc, "mxfp4_grouped_mm")
+    return _to_host(out) if host else out
+
+
+NVFP4_WORKSPACE_BYTES = 16
+
+
+def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspace=None):
+    """NVFP4 two-level quantize + pack along the last dim (K % 16 == 0).
+
+    Returns (packed uint8 [..., K/2], E4M3 block scales uint8 [..., K/16],
+    global scale float32 [1]); the per-tensor scale is g = max|x| / 2688.
+    `workspace` (device uint8, at least NVFP4_WORKSPACE_BYTES) is scratch.
+    """
+    if x.dtype not in _DTYPES:
+        raise TypeError("nvfp4_quantize: unsupported dtype %s" % x.dtype)
+    x, host = _to_device(x)
+    x = x.contiguous()
+    K = x.shape[-1]
+    rows = x.numel() // K if K else 0
+    dev = x.device
+    if packed is None:
+        packed = torch.empty(x.shape[:-1] + (K // 2,), dtype=torch.uint8, device=dev)
+    if block_scales is None:
+        block_scales = torch.empty(x.shape[:-1] + (K // 16,), dtype=torch.uint8, device=dev)
+    if global_scale is None:
+        global_scale = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(NVFP4_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    rc = lib().nvfp4_quantize(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed),
+                              _ptr(block_scales), _ptr(global_scale), _ptr(workspace),
+                              _stream(dev))
+    _check(rc, "nvfp4_quantize")
+    if host:
+        return _to_host(packed), _to_host(block_scales), _to_host(global_scale)
+    return packed, block_scales, global_scale
+
+
+def nvfp4_dequantize(packed, block_scales, global_scale, dtype=torch.bfloat16, out=None):
+    """Unpack NVFP4 storage: E2M1 code * E4M3 block scale * global scale."""
+    if dtype not in _DTYPES:
+        raise TypeError("nvfp4_dequantize: unsupported dtype %s" % dtype)
+    packed, host = _to_device(packed)
+    block_scales, _ = _to_device(block_scales)
+    global_scale, _ = _to_device(global_scale)
+    packed, block_scales = packed.contiguous(), block_scales.contiguous()
+    global_scale = global_scale.to(torch.float32).contiguous()
+    Kh = packed.shape[-1]
+    K = 2 * Kh
+    rows = packed.numel() // Kh if Kh else 0
+    if block_scales.numel() != rows * (K // 16):
+        raise ValueError("nvfp4_dequantize: block_scales must have shape [..., K/16]")
+    if out is None:
+        out = torch.empty(packed.shape[:-1] + (K,), dtype=dtype, device=packed.device)
+    rc = lib().nvfp4_dequantize(_ptr(packed), _ptr(block_scales), _ptr(global_scale), rows, K,
+                                _ptr(out), _DTYPES[dtype], _stream(packed.device))
+    _check(rc, "nvfp4_dequantize")
     return _to_host(out) if host else out

@@ -91,6 +91,29 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
                            (cudaStream_t)stream);
 }
 
+int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                   void* block_scales, float* global_scale, void* workspace, void* stream) {
+  if (!valid_dtype(x_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
+  if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
+    return MXQ_ERR_ALIGNMENT;
+  return launch_nvfp4_quantize(x, x_dtype, rows, K, packed, block_scales, global_scale,
+                               (uint32_t*)workspace, (cudaStream_t)stream);
+}
+
+int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
+                     int64_t rows, int64_t K, void* out, int out_dtype, void* stream) {
+  if (!valid_dtype(out_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
+  if (rows == 0 || K == 0) return MXQ_OK;
+  if (!packed || !block_scales || !global_scale || !out) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  return launch_nvfp4_dequantize(packed, block_scales, global_scale, rows, K, out, out_dtype,
+                                 (cudaStream_t)stream);
+}
+
 const char* mxq_status_string(int status) {
   switch (status) {
     case MXQ_OK: return "MXQ_OK";

@@ -16,6 +16,11 @@ int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, i
                          int dt, cudaStream_t st);
 int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64_t C, int fmt,
                           int B, bool fast, cudaStream_t st);
+int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed,
+                          void* block_scales, float* global_scale, uint32_t* amax_word,
+                          cudaStream_t st);
+int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
+                            int64_t rows, int64_t K, void* out, int dt, cudaStream_t st);
 uint64_t set_wait_limit_ns(uint64_t ns);
 int launch_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,

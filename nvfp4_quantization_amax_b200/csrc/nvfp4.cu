@@ -1,0 +1,217 @@
+// NVFP4 two-level quantization ("NVIDIA Model Optimizer: from mtq.quantize to
+// a 4.95-bit DeepSeek-R1", section "NVFP4 in the code: two scales and a
+// nibble"): a per-tensor binary32 scale g = max|W| / (6 * 448), one E4M3
+// scale per 16 values s_b = E4M3(amax_b / (6 g)) (zero -> 1.0, clamped to
+// [2^-9, 448]) and E2M1 codes of W / (s_b g), packed two per byte.
+//
+// Three launches on the caller's stream: clear the amax word of the
+// workspace, a grid-wide amax (warp and CTA reductions, one atomicMax per
+// CTA on the magnitude bits, which order like the values), then the
+// streaming quantize pass (same item/lane layout as the MXFP4 pack, with a
+// block of 16 held by two lanes).  Every binary32 operation the recipe names
+// (the divisions and products) is the IEEE-rounded one (div.rn / mul.rn), so
+// the codes match a plain float32 implementation bit for bit.
+#include "mxq_device.cuh"
+#include "mxq_launch.h"
+
+namespace mxq {
+
+namespace {
+
+constexpr int kNvThreads = 256;
+constexpr int kNvUnroll = 4;
+
+template <int DT>
+__device__ __forceinline__ uint32_t elem_bits(const uint4& a, const uint4& b, int j) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    const uint32_t w = j < 2 ? a.x : j < 4 ? a.y : j < 6 ? a.z : a.w;
+    return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+  } else {
+    const uint4& q = j < 4 ? a : b;
+    const int k = j & 3;
+    return k == 0 ? q.x : k == 1 ? q.y : k == 2 ? q.z : q.w;
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t amax8(const uint4& a, const uint4& b) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(elem_bits<DT>(a, b, j)));
+  return m;
+}
+
+template <int DT>
+__device__ __forceinline__ void load_vec8(const void* x, int64_t item, uint4& a, uint4& b) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    a = ld_stream_v4((const char*)x + item * 16);
+  } else {
+    a = ld_stream_v4((const char*)x + item * 32);
+    b = ld_stream_v4((const char*)x + item * 32 + 16);
+  }
+}
+
+__global__ void clear_word_kernel(uint32_t* w) { *w = 0u; }
+
+// max |x| over the tensor as binary32 bits, accumulated with atomicMax.
+template <int DT>
+__global__ void __launch_bounds__(kNvThreads)
+nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restrict__ amax_word) {
+  __shared__ uint32_t s_max[kNvThreads / 32];
+  uint32_t m = 0;
+  const int64_t stride = (int64_t)gridDim.x * kNvThreads;
+  for (int64_t it = (int64_t)blockIdx.x * kNvThreads + threadIdx.x; it < n_items; it += stride) {
+    uint4 a, b;
+    load_vec8<DT>(x, it, a, b);
+    m = max(m, amax8<DT>(a, b));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < kNvThreads / 32 ? s_max[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (threadIdx.x == 0 && m != 0u) atomicMax(amax_word, m);
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kNvThreads)
+nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
+                      uint8_t* __restrict__ block_scales, float* __restrict__ global_scale,
+                      const uint32_t* __restrict__ amax_word, int64_t n_items) {
+  const float amax = __uint_as_float(*amax_word);
+  const bool zero = amax == 0.0f;
+  const float g = zero ? 0.0f : __fdiv_rn(amax, 2688.0f);  // 6 * 448
+  const float t = __fmul_rn(6.0f, g);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *global_scale = g;
+  const int lane = threadIdx.x & 31;
+  const uint32_t negzero = (DT == kF32) ? 0x80000000u : 0x8000u;
+  const int64_t stride = (int64_t)gridDim.x * kNvThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
+       base += stride * kNvUnroll) {
+    uint4 va[kNvUnroll], vb[kNvUnroll];
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      if (item < n_items) load_vec8<DT>(x, item, va[u], vb[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      const bool valid = item < n_items;
+      uint32_t m = valid ? amax8<DT>(va[u], vb[u]) : 0u;
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));  // the two lanes of a 16-block
+      if (!valid) continue;
+      uint32_t sbyte;
+      uint32_t codes = 0;
+      if (zero) {
+        sbyte = 0x38u;  // E4M3 1.0
+      } else {
+        float q = __fdiv_rn(__uint_as_float(m), t);
+        if (q == 0.0f) q = 1.0f;
+        q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
+        sbyte = e4m3x2(q, 0.0f) & 0xFFu;
+        const float s = f16lo(e4m3x2_to_f16x2(sbyte));
+        const float d = __fmul_rn(s, g);
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t bits = elem_bits<DT>(va[u], vb[u], j);
+          if (bits == negzero) bits = 0u;  // -0.0 carries no sign into the code
+          v[j] = __fdiv_rn(elem_to_f32<DT>(bits), d);  // keeps the sign on underflow
+        }
+        codes = e2m1x8(v);
+      }
+      packed[item] = codes;
+      if ((lane & 1) == 0) block_scales[item >> 1] = (uint8_t)sbyte;
+    }
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kNvThreads)
+nvfp4_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __restrict__ block_scales,
+                        const float* __restrict__ global_scale, void* __restrict__ out,
+                        int64_t n_items) {
+  const float g = *global_scale;
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * kNvThreads;
+  for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
+       base += stride * kNvUnroll) {
+    uint32_t p[kNvUnroll], sb[kNvUnroll];
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      if (item < n_items) {
+        p[u] = ld_stream_u32(packed + item);
+        sb[u] = ld_stream_u8(block_scales + (item >> 1));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      if (item >= n_items) continue;
+      const float s = f16lo(e4m3x2_to_f16x2(sb[u]));
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
+        // code * s_b is exact in binary32; times g rounds once; adding +0
+        // in the same fma turns the -0 of nibble 8 into +0
+        v[2 * j] = fmaf(f16lo(h2) * s, g, 0.0f);
+        v[2 * j + 1] = fmaf(f16hi(h2) * s, g, 0.0f);
+      }
+      store8<DT>(out, item, v);
+    }
+  }
+}
+
+int grid_for(int64_t n_units, int per_block, int resident) {
+  int64_t need = (n_units + per_block - 1) / per_block;
+  int64_t cap = (int64_t)num_sms() * resident;
+  if (need > cap) need = cap;
+  return (int)(need < 1 ? 1 : need);
+}
+
+template <int DT>
+int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* block_scales,
+                 float* global_scale, uint32_t* amax_word, cudaStream_t st) {
+  const int64_t n_items = rows * (K / 8);
+  clear_word_kernel<<<1, 1, 0, st>>>(amax_word);
+  if (n_items > 0) {
+    nvfp4_amax_kernel<DT><<<grid_for(n_items, kNvThreads * 4, 8), kNvThreads, 0, st>>>(
+        x, n_items, amax_word);
+  }
+  nvfp4_quantize_kernel<DT><<<grid_for(n_items, kNvThreads * kNvUnroll, 4), kNvThreads, 0, st>>>(
+      x, (uint32_t*)packed, (uint8_t*)block_scales, global_scale, amax_word, n_items);
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed,
+                          void* block_scales, float* global_scale, uint32_t* amax_word,
+                          cudaStream_t st) {
+  switch (dt) {
+    case kBF16: return run_quantize<kBF16>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
+    case kF16: return run_quantize<kF16>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
+    default: return run_quantize<kF32>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
+  }
+}
+
+int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
+                            int64_t rows, int64_t K, void* out, int dt, cudaStream_t st) {
+  const int64_t n_items = rows * (K / 8);
+  const int grid = grid_for(n_items, kNvThreads * kNvUnroll, 8);
+  auto* p = (const uint32_t*)packed;
+  auto* s = (const uint8_t*)block_scales;
+  switch (dt) {
+    case kBF16: nvfp4_dequantize_kernel<kBF16><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
+    case kF16: nvfp4_dequantize_kernel<kF16><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
+    default: nvfp4_dequantize_kernel<kF32><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+}  // namespace mxq

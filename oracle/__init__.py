@@ -54,6 +54,14 @@ def lib():
         L.orc_quantize_cache.argtypes = [p, p, i, i64, i64, i, i]
         L.orc_check_offs.restype = i
         L.orc_check_offs.argtypes = [p, i64, i64]
+        L.orc_nvfp4_global_scale.restype = d
+        L.orc_nvfp4_global_scale.argtypes = [d]
+        L.orc_nvfp4_block_scale.restype = d
+        L.orc_nvfp4_block_scale.argtypes = [d, d]
+        L.orc_nvfp4_quantize.restype = i
+        L.orc_nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p]
+        L.orc_nvfp4_dequantize.restype = i
+        L.orc_nvfp4_dequantize.argtypes = [p, p, ctypes.c_float, i64, i64, p, i]
         L.orc_grouped_mm.restype = i
         L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
         _lib = L
@@ -201,3 +209,40 @@ def grouped_mm(a_bits, packed, scales, offs, transpose_w=False, rows=None):
         raise ValueError("oracle grouped_mm: rc=%d" % rc)
     return out
 
+
+
+def nvfp4_global_scale(amax):
+    return lib().orc_nvfp4_global_scale(float(amax))
+
+
+def nvfp4_block_scale(amax_b, g):
+    return lib().orc_nvfp4_block_scale(float(amax_b), float(g))
+
+
+def nvfp4_quantize(x_bits, dtype="bf16"):
+    """x [..., K] (K % 16 == 0) -> (packed uint8 [..., K/2], E4M3 block scales
+    uint8 [..., K/16], global scale g as a Python float)."""
+    x = _c(x_bits, _BITS[dtype])
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    packed = np.empty(x.shape[:-1] + (K // 2,), np.uint8)
+    bs = np.empty(x.shape[:-1] + (K // 16,), np.uint8)
+    g = ctypes.c_float(0.0)
+    rc = lib().orc_nvfp4_quantize(_ptr(x), DTYPES[dtype], rows, K, _ptr(packed), _ptr(bs),
+                                  ctypes.byref(g))
+    if rc != 0:
+        raise ValueError("oracle nvfp4_quantize: bad arguments rc=%d" % rc)
+    return packed, bs, g.value
+
+
+def nvfp4_dequantize(packed, block_scales, global_scale, dtype="bf16"):
+    p = _c(packed, np.uint8)
+    s = _c(block_scales, np.uint8)
+    K = p.shape[-1] * 2
+    rows = p.size // p.shape[-1] if p.shape[-1] else 0
+    out = np.empty(p.shape[:-1] + (K,), _BITS[dtype])
+    rc = lib().orc_nvfp4_dequantize(_ptr(p), _ptr(s), float(global_scale), rows, K, _ptr(out),
+                                    DTYPES[dtype])
+    if rc != 0:
+        raise ValueError("oracle nvfp4_dequantize: bad arguments rc=%d" % rc)
+    return out

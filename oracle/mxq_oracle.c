@@ -407,3 +407,88 @@ int orc_grouped_mm(const uint16_t* a, const uint8_t* packed, const uint8_t* scal
   free(w);
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 two-level quantization ([MO] "NVFP4 in the code: two scales and a  */
+/* nibble"; block 16 and e4m3 scales from the numerics YAML of "mtq.quantize */
+/* is three moves").                                                         */
+/* ------------------------------------------------------------------------ */
+
+/* binary32 arithmetic, emulated: the exact real result rounded once to
+   binary32.  For inputs that are binary32 values, computing in double and
+   rounding to binary32 gives exactly the correctly rounded binary32 result
+   for + - * / (double rounding is innocuous when 53 >= 2*24 + 2; Figueroa,
+   "When is double rounding innocuous?", SIGNUM 1995). */
+static double f32_mul(double a, double b) { return orc_round_f32(a * b); }
+static double f32_div(double a, double b) { return orc_round_f32(a / b); }
+
+/* Per-tensor scale g = max|W| / (6 * 448) as a binary32 value. */
+double orc_nvfp4_global_scale(double amax) { return f32_div(amax, 6.0 * 448.0); }
+
+/* Block scale s_b = E4M3(amax_b / (6 g)) with a zero quotient replaced by
+   1.0 and the quotient clamped to [2^-9, 448] before the cast. */
+double orc_nvfp4_block_scale(double amax_b, double g) {
+  double q = f32_div(amax_b, f32_mul(6.0, g));
+  if (q == 0.0) q = 1.0;
+  if (q < ldexp(1.0, -9)) q = ldexp(1.0, -9);
+  if (q > 448.0) q = 448.0;
+  return orc_round_e4m3(q);
+}
+
+/* x: [rows, K] (K % 16 == 0).  packed [rows, K/2] (E2M1 codes, low nibble =
+   even column); block_scales [rows, K/16] (E4M3 bytes); *global_scale = g.
+   The element cast is E2M1(W / (s_b g)) with s_b * g and the quotient in
+   binary32.  An all-zero tensor gives g = 0, codes 0 and block scales 1.0. */
+int orc_nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t K, uint8_t* packed,
+                       uint8_t* block_scales, float* global_scale) {
+  if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  double amax = 0.0;
+  for (int64_t i = 0; i < rows * K; ++i) {
+    double a = fabs(load_elem(x, dtype, i));
+    if (a > amax) amax = a;
+  }
+  double g = amax == 0.0 ? 0.0 : orc_nvfp4_global_scale(amax);
+  *global_scale = (float)g;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < K / 16; ++b) {
+      int64_t base = r * K + b * 16;
+      double amax_b = 0.0;
+      for (int i = 0; i < 16; ++i) {
+        double a = fabs(load_elem(x, dtype, base + i));
+        if (a > amax_b) amax_b = a;
+      }
+      double s = amax == 0.0 ? 1.0 : orc_nvfp4_block_scale(amax_b, g);
+      block_scales[r * (K / 16) + b] = orc_encode_e4m3(s);
+      double d = f32_mul(s, g);
+      for (int j = 0; j < 8; ++j) {
+        int lo = 0, hi = 0;
+        if (amax != 0.0) {
+          /* the sign bit follows x itself: a binary32 quotient of a tiny
+             negative value may underflow to -0.0 */
+          double x0 = load_elem(x, dtype, base + 2 * j), x1 = load_elem(x, dtype, base + 2 * j + 1);
+          lo = (orc_e2m1_code(fabs(f32_div(x0, d))) & 7) | (x0 < 0.0 ? 8 : 0);
+          hi = (orc_e2m1_code(fabs(f32_div(x1, d))) & 7) | (x1 < 0.0 ? 8 : 0);
+        }
+        packed[r * (K / 2) + b * 8 + j] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* out[r][k] = E2M1(nibble) * s_b * g, evaluated in binary32 (the product of
+   the code and the E4M3 scale is exact there; times g rounds once), then
+   rounded to out_dtype. */
+int orc_nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scales, float global_scale,
+                         int64_t rows, int64_t K, void* out, int out_dtype) {
+  if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k) {
+      uint8_t byte = packed[r * (K / 2) + k / 2];
+      int nib = (k % 2 == 0) ? (byte & 15) : (byte >> 4);
+      double s = orc_decode_e4m3(block_scales[r * (K / 16) + k / 16]);
+      double v = f32_mul(E2M1_TABLE[nib] * s, (double)global_scale);
+      store_rounded(out, out_dtype, r * K + k, v);
+    }
+  return ORC_OK;
+}

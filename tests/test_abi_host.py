@@ -112,3 +112,16 @@ def test_binding_fails_loudly_without_gpu():
 def test_wait_limit_setter_round_trips(L):
     prev = mxq.set_wait_limit_ns(123)
     assert mxq.set_wait_limit_ns(prev) == 123
+
+
+def test_nvfp4_validation(L):
+    assert L.nvfp4_quantize(A1, 0, 4, 40, A2, A2, A2, A1, NULL) == ESHAPE
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, A2, NULL, NULL) == EARG  # workspace
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, NULL, A1, NULL) == EARG  # global scale
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, A2, BAD, NULL) == EALIGN
+    assert L.nvfp4_quantize(BAD, 0, 4, 64, A2, A2, A2, A1, NULL) == EALIGN
+    assert L.nvfp4_quantize(A1, 9, 4, 64, A2, A2, A2, A1, NULL) == EARG
+    assert L.nvfp4_dequantize(A1, A2, A2, 4, 24, A1, 0, NULL) == ESHAPE
+    assert L.nvfp4_dequantize(A1, A2, NULL, 4, 32, A1, 0, NULL) == EARG
+    assert L.nvfp4_dequantize(BAD, A2, A2, 4, 32, A1, 0, NULL) == EALIGN
+    assert L.nvfp4_dequantize(NULL, NULL, NULL, 0, 32, NULL, 0, NULL) == OK

@@ -332,3 +332,53 @@ def test_grouped_mm_wait_timeout_reports_status():
         mxq.set_wait_limit_ns(prev)
     assert int(status.item()) == -7
     check_gemm([700, 300, 50], N=128, K=512, transpose_w=False)
+
+
+# ------------------------------------------------------- NVFP4 two-level
+
+def nv_inputs(dtype):
+    x = torch.cat([gen.kv_cache((1, 64, 512)).view(64, 512), gen.mixed_blocks(64, 512),
+                   gen.normal_bf16(41, (64, 512))]).to(dtype)
+    if dtype == torch.float32:
+        x.view(-1)[:4096] = f32_edge_values(4096, 9) * 1e-25
+    return x
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_nvfp4_quantize_exact(dtype):
+    x = nv_inputs(dtype).to(DEV)
+    p, s, g = mxq.nvfp4_quantize(x)
+    wp, ws, wg = oracle.nvfp4_quantize(bits(x), _NAME[dtype])
+    assert float(g.item()) == wg
+    assert_bits_equal(u8(s), ws, "block scales")
+    assert_bits_equal(u8(p), wp, "packed")
+
+
+def test_nvfp4_expert_weights_exact():
+    x = gen.expert_weights(4, 2048, 7168, device=DEV)
+    p, s, g = mxq.nvfp4_quantize(x)
+    wp, ws, wg = oracle.nvfp4_quantize(bits(x))
+    assert float(g.item()) == wg
+    assert_bits_equal(u8(s), ws, "block scales")
+    assert_bits_equal(u8(p), wp, "packed")
+    assert int(s.max()) == 0x7E  # the top block is scaled by exactly 448
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_nvfp4_dequantize_exact(dtype):
+    wp, ws, wg = oracle.nvfp4_quantize(bits(nv_inputs(torch.bfloat16)))
+    y = mxq.nvfp4_dequantize(torch.from_numpy(wp).to(DEV), torch.from_numpy(ws).to(DEV),
+                             torch.tensor([wg], dtype=torch.float32, device=DEV), dtype)
+    assert_bits_equal(bits(y), oracle.nvfp4_dequantize(wp, ws, wg, _NAME[dtype]), "dequant")
+
+
+def test_nvfp4_zero_and_ragged():
+    z = torch.zeros(3, 48, dtype=torch.bfloat16, device=DEV)
+    p, s, g = mxq.nvfp4_quantize(z)
+    assert float(g.item()) == 0.0 and int(p.max()) == 0 and bool((s == 0x38).all())
+    x = gen.normal_bf16(77, (5, 48), device=DEV)  # 30 items: a partial warp
+    p, s, g = mxq.nvfp4_quantize(x)
+    wp, ws, wg = oracle.nvfp4_quantize(bits(x))
+    assert float(g.item()) == wg
+    assert_bits_equal(u8(p), wp, "packed")
+    assert_bits_equal(u8(s), ws, "scales")

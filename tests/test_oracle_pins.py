@@ -487,3 +487,110 @@ def test_grouped_mm_rejects_bad_offs():
     with pytest.raises(ValueError):
         oracle.grouped_mm(a, packed, scales, np.array([3, 3, 6], np.int32))
     assert oracle.check_offs(np.array([0, 0, 7], np.int32), 7)
+
+
+# ----------------------------------------------------- NVFP4 two-level
+
+def e2m1_bruteforce_code(v):
+    """Nearest E2M1 code of a finite value (ties to the even magnitude),
+    sign bit iff v < 0 (a -0.0 quotient of a negative input keeps it below)."""
+    mag = int(bruteforce_e2m1_mag(np.array([abs(v)]))[0]) if abs(v) < 2.0**40 else 7
+    return mag
+
+
+def nvfp4_reference(xv):
+    """NVFP4 two-level quantization computed with numpy binary32 arithmetic
+    and torch's E4M3 cast (independent of the oracle's own routines)."""
+    f32 = np.float32
+    amax = f32(np.abs(xv).max())
+    rows, K = xv.shape
+    packed = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, K // 16), np.uint8)
+    if amax == 0:
+        scales[:] = torch.tensor([1.0]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+        return packed, scales, 0.0
+    g = f32(amax) / f32(2688.0)
+    t = f32(6.0) * g
+    for r in range(rows):
+        for b in range(K // 16):
+            blk = xv[r, 16 * b:16 * b + 16].astype(np.float32)
+            q = f32(np.abs(blk).max()) / t
+            q = f32(1.0) if q == 0 else q
+            q = min(max(q, f32(2.0**-9)), f32(448.0))
+            e4 = torch.tensor([float(q)], dtype=torch.float32).to(torch.float8_e4m3fn)
+            scales[r, b] = e4.view(torch.uint8).item()
+            s = f32(e4.to(torch.float32).item())
+            d = s * g
+            codes = []
+            for v in blk:
+                qv = f32(v) / d
+                codes.append(e2m1_bruteforce_code(float(qv)) | (8 if v < 0 else 0))
+            for j in range(8):
+                packed[r, 8 * b + j] = codes[2 * j] | (codes[2 * j + 1] << 4)
+    return packed, scales, float(g)
+
+
+def test_nvfp4_matches_float32_reference():
+    x = torch.cat([gen.kv_cache((1, 3, 64)).view(3, 64), gen.mixed_blocks(3, 64),
+                   gen.normal_bf16(31, (2, 64))])
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    wp, ws, wg = nvfp4_reference(oracle.decode(bits, "bf16"))
+    assert g == wg
+    assert np.array_equal(s, ws)
+    assert np.array_equal(p, wp)
+
+
+def test_nvfp4_page_facts(facts):
+    x = gen.expert_weights(1, 32, 256).view(32, 256).clone()
+    x[5, 16:32] = 0.0  # one all-zero block
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    xv = oracle.decode(bits, "bf16")
+    amax = np.abs(xv).max()
+    assert g == np.float32(np.float32(amax) / np.float32(facts["nvfp4_global_denominator"]))
+    decoded = np.array([oracle.decode_e4m3(b) for b in s.reshape(-1)]).reshape(s.shape)
+    # the block holding the tensor's largest value gets exactly 448
+    r, c = np.unravel_index(np.argmax(np.abs(xv)), xv.shape)
+    assert decoded[r, c // 16] == facts["nvfp4_top_block_scale"]
+    assert decoded.max() == 448.0 and decoded.min() >= 2.0**-9
+    # a zero block takes scale 1.0 and codes 0
+    assert decoded[5, 1] == facts["nvfp4_zero_block_scale"]
+    assert (p[5, 8:16] == 0).all()
+    # 4.5 bits per value: scale bytes are one eighth of packed bytes
+    assert s.nbytes * 8 == p.nbytes
+
+
+def test_nvfp4_dequant_matches_float32_reference():
+    x = gen.kv_cache((1, 4, 128)).view(4, 128)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    out = oracle.nvfp4_dequantize(p, s, g, "f32")
+    tab = full_table()
+    codes = np.stack([p & 15, p >> 4], axis=-1).reshape(4, 128)
+    sc = torch.from_numpy(s.copy()).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    sc = np.repeat(sc, 16, axis=1)
+    want = (tab[codes].astype(np.float32) * sc) * np.float32(g)
+    assert np.array_equal(out.view(np.float32), want.astype(np.float32))
+    # bf16 output: the binary32 value rounded once more
+    outb = oracle.nvfp4_dequantize(p, s, g, "bf16")
+    wantb = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(outb, wantb.view(np.uint16))
+
+
+def test_nvfp4_error_bound():
+    # every value lands within half a grid step of its block's scaled grid
+    x = gen.expert_weights(1, 16, 512).view(16, 512)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    y = oracle.decode(oracle.nvfp4_dequantize(p, s, g, "f32"), "f32")
+    xv = oracle.decode(bits, "bf16")
+    sc = np.repeat(np.array([oracle.decode_e4m3(b) for b in s.reshape(-1)]).reshape(s.shape), 16, 1)
+    step = sc * g  # one unit of the E2M1 grid in the block; gaps are at most 2 units
+    assert (np.abs(y - xv) <= step * 1.0 + 1e-30).all()
+
+
+def test_nvfp4_zero_tensor():
+    bits = np.zeros((2, 32), np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    assert g == 0.0 and (p == 0).all() and (s == 0x38).all()  # 0x38 is E4M3 1.0
