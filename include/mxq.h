@@ -173,6 +173,33 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
 int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                      int64_t rows, int64_t K, void* out, int out_dtype, void* stream);
 
+/* Size of the library's own static device scratch used by
+ * nvfp4_quantize_noalloc (bytes per GPU, held from library load to exit). */
+#define MXQ_NOALLOC_SCRATCH_BYTES 256
+
+/* nvfp4_quantize without a workspace argument and without allocating.
+ *
+ * No counterpart on the source pages: this entry point exists for callers
+ * that own all device memory up front and may not allocate while they run,
+ * for example an inference engine or a plugin whose memory pool is fixed at
+ * start-up, where cudaMalloc would synchronize the device or fail once the
+ * pool holds everything.  Such callers still pass inputs and outputs; the
+ * 16 bytes of scratch the quantization needs (the tensor-wide maximum) come
+ * from a static device array inside libmxq.so instead of a workspace.
+ *
+ * Arguments, results and errors are those of nvfp4_quantize without the
+ * workspace.  The scratch need does not grow with the input (16 bytes for
+ * any shape); a build whose need exceeded MXQ_NOALLOC_SCRATCH_BYTES would
+ * return MXQ_ERR_UNSUPPORTED.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before capturing the stream into a graph.  All calls
+ * share the one array: the call clears it before use, and calls that overlap
+ * on the GPU (for instance on two streams) race on it and must be
+ * serialized by the caller.  Never allocates: no cudaMalloc, cudaFree or
+ * allocating library routine is called. */
+int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                           void* block_scales, float* global_scale, void* stream);
+
 /* Limit, in nanoseconds, after which a pipeline wait inside the grouped GEMM
  * gives up (the kernel then drains what it issued, frees its tensor memory
  * and reports MXQ_ERR_TIMEOUT through dev_status).  Default 2e9 (2 s); it

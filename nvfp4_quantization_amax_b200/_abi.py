@@ -46,6 +46,8 @@ def lib():
         L.mxq_version.argtypes = []
         L.nvfp4_quantize.restype = i
         L.nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p, p, p]
+        L.nvfp4_quantize_noalloc.restype = i
+        L.nvfp4_quantize_noalloc.argtypes = [p, i, i64, i64, p, p, p, p]
         L.nvfp4_dequantize.restype = i
         L.nvfp4_dequantize.argtypes = [p, p, p, i64, i64, p, i, p]
         L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64

@@ -103,6 +103,20 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
                                (uint32_t*)workspace, (cudaStream_t)stream);
 }
 
+int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                           void* block_scales, float* global_scale, void* stream) {
+  if (!valid_dtype(x_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
+  if (!global_scale) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))) return MXQ_ERR_ALIGNMENT;
+  int status = MXQ_OK;
+  uint32_t* scratch = noalloc_scratch(MXQ_NVFP4_WORKSPACE_BYTES, &status);
+  if (!scratch) return status;
+  return launch_nvfp4_quantize(x, x_dtype, rows, K, packed, block_scales, global_scale, scratch,
+                               (cudaStream_t)stream);
+}
+
 int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                      int64_t rows, int64_t K, void* out, int out_dtype, void* stream) {
   if (!valid_dtype(out_dtype)) return MXQ_ERR_INVALID_ARG;

@@ -19,6 +19,9 @@ int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64
 int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed,
                           void* block_scales, float* global_scale, uint32_t* amax_word,
                           cudaStream_t st);
+// Device address of the static scratch of the allocation-free entry point on
+// the current device (looked up once per device), or nullptr on failure.
+uint32_t* noalloc_scratch(size_t need_bytes, int* status);
 int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                             int64_t rows, int64_t K, void* out, int dt, cudaStream_t st);
 uint64_t set_wait_limit_ns(uint64_t ns);

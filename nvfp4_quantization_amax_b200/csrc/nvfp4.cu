@@ -11,6 +11,8 @@
 // block of 16 held by two lanes).  Every binary32 operation the recipe names
 // (the divisions and products) is the IEEE-rounded one (div.rn / mul.rn), so
 // the codes match a plain float32 implementation bit for bit.
+#include <mutex>
+
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
 
@@ -188,7 +190,38 @@ int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* blo
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+// Scratch of the allocation-free entry point: one copy per GPU that loads
+// the library, alive until the process exits.  Host code must not pass the
+// symbol itself to a kernel (on the host it names a stand-in, not device
+// memory); it passes the address cudaGetSymbolAddress returns.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[MXQ_NOALLOC_SCRATCH_BYTES / 4];
+
 }  // namespace
+
+uint32_t* noalloc_scratch(size_t need_bytes, int* status) {
+  if (need_bytes > sizeof(g_noalloc_scratch)) {
+    *status = MXQ_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  static std::mutex mu;
+  static uint32_t* by_device[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *status = MXQ_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (by_device[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *status = MXQ_ERR_CUDA;
+      return nullptr;
+    }
+    by_device[dev] = (uint32_t*)p;
+  }
+  *status = MXQ_OK;
+  return by_device[dev];
+}
 
 int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed,
                           void* block_scales, float* global_scale, uint32_t* amax_word,

@@ -125,3 +125,11 @@ def test_nvfp4_validation(L):
     assert L.nvfp4_dequantize(A1, A2, NULL, 4, 32, A1, 0, NULL) == EARG
     assert L.nvfp4_dequantize(BAD, A2, A2, 4, 32, A1, 0, NULL) == EALIGN
     assert L.nvfp4_dequantize(NULL, NULL, NULL, 0, 32, NULL, 0, NULL) == OK
+
+
+def test_nvfp4_noalloc_validation_needs_no_gpu(L):
+    # argument errors are reported before the scratch is looked up
+    assert L.nvfp4_quantize_noalloc(A1, 0, 4, 40, A2, A2, A2, NULL) == ESHAPE
+    assert L.nvfp4_quantize_noalloc(A1, 0, 4, 64, A2, A2, NULL, NULL) == EARG
+    assert L.nvfp4_quantize_noalloc(BAD, 0, 4, 64, A2, A2, A2, NULL) == EALIGN
+    assert L.nvfp4_quantize_noalloc(A1, 5, 4, 64, A2, A2, A2, NULL) == EARG
