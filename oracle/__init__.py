@@ -60,8 +60,22 @@ def lib():
         L.orc_nvfp4_block_scale.argtypes = [d, d]
         L.orc_nvfp4_quantize.restype = i
         L.orc_nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p]
+        L.orc_nvfp4_block_sq_error.restype = d
+        L.orc_nvfp4_block_sq_error.argtypes = [p, d, i]
+        L.orc_nvfp4_mse_code.restype = i
+        L.orc_nvfp4_mse_code.argtypes = [p, d]
+        L.orc_nvfp4_quantize_mse_rows.restype = i
+        L.orc_nvfp4_quantize_mse_rows.argtypes = [p, i, i64, i64, d, p, p]
+        L.orc_nvfp4_quantize_mse.restype = i
+        L.orc_nvfp4_quantize_mse.argtypes = [p, i, i64, i64, p, p, p]
         L.orc_nvfp4_dequantize.restype = i
         L.orc_nvfp4_dequantize.argtypes = [p, p, ctypes.c_float, i64, i64, p, i]
+        L.orc_cache_scale_byte.restype = ctypes.c_uint8
+        L.orc_cache_scale_byte.argtypes = [i, i]
+        L.orc_quantize_cache_packed.restype = i
+        L.orc_quantize_cache_packed.argtypes = [p, i, i64, i64, i, i, p, p]
+        L.orc_dequantize_cache_packed.restype = i
+        L.orc_dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i, p, i]
         L.orc_grouped_mm.restype = i
         L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
         _lib = L
@@ -246,3 +260,71 @@ def nvfp4_dequantize(packed, block_scales, global_scale, dtype="bf16"):
     if rc != 0:
         raise ValueError("oracle nvfp4_dequantize: bad arguments rc=%d" % rc)
     return out
+
+
+def quantize_cache_packed(x_bits, fmt, block_size, dtype="bf16"):
+    """Stored form of quantize_cache: (codes, scale bytes)."""
+    x = _c(x_bits, _BITS[dtype])
+    C = x.shape[-1]
+    rows = x.size // C if C else 0
+    ncode = C if fmt == "fp8" else C // 2
+    codes = np.zeros(x.shape[:-1] + (ncode,), np.uint8)
+    scales = np.empty(x.shape[:-1] + (C // int(block_size),), np.uint8)
+    rc = lib().orc_quantize_cache_packed(_ptr(x), DTYPES[dtype], rows, C, FORMATS[fmt],
+                                         int(block_size), _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError("oracle quantize_cache_packed: bad arguments rc=%d" % rc)
+    return codes, scales
+
+
+def dequantize_cache_packed(codes, scales, fmt, block_size, channels, dtype="bf16"):
+    c = _c(codes, np.uint8)
+    s = _c(scales, np.uint8)
+    C = int(channels)
+    rows = s.size // (C // int(block_size))
+    out = np.empty(s.shape[:-1] + (C,), _BITS[dtype])
+    rc = lib().orc_dequantize_cache_packed(_ptr(c), _ptr(s), rows, C, FORMATS[fmt],
+                                           int(block_size), _ptr(out), DTYPES[dtype])
+    if rc != 0:
+        raise ValueError("oracle dequantize_cache_packed: bad arguments rc=%d" % rc)
+    return out
+
+
+def cache_scale_byte(k, fmt):
+    return lib().orc_cache_scale_byte(int(k), FORMATS[fmt])
+
+
+def nvfp4_block_sq_error(w16, g, code):
+    """Squared weight error of one 16-block (float64 values) under an E4M3
+    block-scale code."""
+    w = np.ascontiguousarray(w16, np.float64)
+    assert w.size == 16
+    return lib().orc_nvfp4_block_sq_error(_ptr(w), float(g), int(code))
+
+
+def nvfp4_mse_code(w16, g):
+    w = np.ascontiguousarray(w16, np.float64)
+    assert w.size == 16
+    return lib().orc_nvfp4_mse_code(_ptr(w), float(g))
+
+
+def nvfp4_quantize_mse(x_bits, dtype="bf16", g=None):
+    """NVFP4 with mse block scales -> (packed, block scales, g).  With g
+    given, rows are quantized with that per-tensor scale (for samples of a
+    larger tensor)."""
+    x = _c(x_bits, _BITS[dtype])
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    packed = np.empty(x.shape[:-1] + (K // 2,), np.uint8)
+    bs = np.empty(x.shape[:-1] + (K // 16,), np.uint8)
+    if g is None:
+        gf = ctypes.c_float(0.0)
+        rc = lib().orc_nvfp4_quantize_mse(_ptr(x), DTYPES[dtype], rows, K, _ptr(packed),
+                                          _ptr(bs), ctypes.byref(gf))
+        g = gf.value
+    else:
+        rc = lib().orc_nvfp4_quantize_mse_rows(_ptr(x), DTYPES[dtype], rows, K, float(g),
+                                               _ptr(packed), _ptr(bs))
+    if rc != 0:
+        raise ValueError("oracle nvfp4_quantize_mse: bad arguments rc=%d" % rc)
+    return packed, bs, g

@@ -492,3 +492,152 @@ int orc_nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scales, flo
     }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Packed cache storage: the stored form of quantize_cache ([CQ]).           */
+/* ------------------------------------------------------------------------ */
+
+/* Scale byte of a cache block with scale 2^k: E8M0 (k + 127) for fp8 and
+   mxfp4, the E4M3 encoding of 2^k for nvfp4. */
+uint8_t orc_cache_scale_byte(int k, int fmt) {
+  if (fmt == ORC_NVFP4) return orc_encode_e4m3(ldexp(1.0, k));
+  return (uint8_t)(k + 127);
+}
+
+/* in [rows, C] (C % B == 0; B even for the fp4 formats).  codes: fp8 -> [rows, C] E4M3 bytes of
+   x / 2^k; mxfp4/nvfp4 -> [rows, C/2] E2M1 codes (low nibble = even column,
+   sign bit iff x < 0).  scales: [rows, C/B] scale bytes. */
+int orc_quantize_cache_packed(const void* in, int dtype, int64_t rows, int64_t C, int fmt, int B,
+                              uint8_t* codes, uint8_t* scales) {
+  if (B < 1 || C % B != 0 || rows < 0 || fmt < 0 || fmt > 2) return ORC_EARG;
+  if (fmt != ORC_FP8 && B % 2 != 0) return ORC_EARG; /* nibble pairs stay in a group */
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c0 = 0; c0 < C; c0 += B) {
+      double amax = 0.0;
+      for (int64_t c = c0; c < c0 + B; ++c) {
+        double a = fabs(load_elem(in, dtype, r * C + c));
+        if (a > amax) amax = a;
+      }
+      int k = orc_cache_scale_exp(amax, fmt);
+      scales[r * (C / B) + c0 / B] = orc_cache_scale_byte(k, fmt);
+      for (int64_t c = c0; c < c0 + B; ++c) {
+        double x = load_elem(in, dtype, r * C + c);
+        double v = ldexp(x, -k);
+        if (fmt == ORC_FP8) {
+          codes[r * C + c] = orc_encode_e4m3(orc_round_e4m3(v));
+        } else {
+          int code = orc_e2m1_code(v);
+          uint8_t* byte = &codes[r * (C / 2) + c / 2];
+          if (c % 2 == 0) *byte = (uint8_t)code;
+          else *byte = (uint8_t)(*byte | (code << 4));
+        }
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* out[r][c] = round_dtype(decode(code) * scale); fp4 zeros are +0 (as in
+   the fake quantization), fp8 keeps the sign of zero. */
+int orc_dequantize_cache_packed(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                                int64_t C, int fmt, int B, void* out, int out_dtype) {
+  if (B < 1 || C % B != 0 || rows < 0 || fmt < 0 || fmt > 2) return ORC_EARG;
+  if (fmt != ORC_FP8 && B % 2 != 0) return ORC_EARG; /* nibble pairs stay in a group */
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < C; ++c) {
+      uint8_t sb = scales[r * (C / B) + c / B];
+      double s = fmt == ORC_NVFP4 ? orc_decode_e4m3(sb)
+                 : sb == 0xFF       ? NAN /* the E8M0 NaN */
+                                    : ldexp(1.0, (int)sb - 127);
+      double v;
+      if (fmt == ORC_FP8) {
+        v = orc_decode_e4m3(codes[r * C + c]) * s;
+      } else {
+        uint8_t byte = codes[r * (C / 2) + c / 2];
+        v = E2M1_TABLE[(c % 2 == 0) ? (byte & 15) : (byte >> 4)] * s;
+        if (v == 0.0) v = 0.0; /* a zero fp4 element is +0 whatever the signs */
+      }
+      store_rounded(out, out_dtype, r * C + c, v);
+    }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 block scale chosen by least squared weight error ([MO] "NVFP4's    */
+/* own rules": mse).                                                         */
+/* ------------------------------------------------------------------------ */
+
+/* Squared weight error of one 16-block under block-scale code c (an E4M3
+   byte, 1..126):  d = s_c * g in binary32; each weight is cast to E2M1 as
+   the max rule casts it (binary32 quotient w / d, nearest-even, saturating);
+   the error of weight i is e_i = q_i * d - w_i, which double arithmetic
+   holds exactly; the sum of e_i^2 is accumulated over i = 0..15 in order,
+   one fused multiply-add in double per term.  A code whose d underflows to
+   zero can represent nothing and gets +infinity. */
+double orc_nvfp4_block_sq_error(const double* w, double g, int code) {
+  double d = f32_mul(orc_decode_e4m3((uint8_t)code), g);
+  if (d == 0.0) return INFINITY;
+  double err = 0.0;
+  for (int i = 0; i < 16; ++i) {
+    double q = orc_e2m1_value(orc_e2m1_code(fabs(f32_div(w[i], d)))) * (w[i] < 0.0 ? -1.0 : 1.0);
+    double e = fma(q, d, -w[i]);
+    err = fma(e, e, err);
+  }
+  return err;
+}
+
+/* The code with the least error over the 126 positive finite E4M3 codes,
+   the smallest code among equal least errors. */
+int orc_nvfp4_mse_code(const double* w, double g) {
+  int best = 1;
+  double best_err = INFINITY;
+  for (int c = 1; c <= 126; ++c) {
+    double err = orc_nvfp4_block_sq_error(w, g, c);
+    if (err < best_err) {
+      best_err = err;
+      best = c;
+    }
+  }
+  return best;
+}
+
+/* NVFP4 quantize with mse block scales, given the per-tensor scale g (the
+   max rule's amax / 2688).  g == 0 (an all-zero tensor) gives the max
+   rule's output: scale code 1.0 (0x38) and zero codes everywhere. */
+int orc_nvfp4_quantize_mse_rows(const void* x, int dtype, int64_t rows, int64_t K, double g,
+                                uint8_t* packed, uint8_t* block_scales) {
+  if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < K / 16; ++b) {
+      int64_t base = r * K + b * 16;
+      double w[16];
+      for (int i = 0; i < 16; ++i) w[i] = load_elem(x, dtype, base + i);
+      int code = g == 0.0 ? 0x38 : orc_nvfp4_mse_code(w, g);
+      block_scales[r * (K / 16) + b] = (uint8_t)code;
+      double d = f32_mul(orc_decode_e4m3((uint8_t)code), g);
+      for (int j = 0; j < 8; ++j) {
+        int nib[2] = {0, 0};
+        for (int h = 0; h < 2 && g != 0.0; ++h) {
+          double xi = w[2 * j + h];
+          if (xi == 0.0) continue; /* code 0, also where d underflowed to 0 */
+          nib[h] = (orc_e2m1_code(fabs(f32_div(xi, d))) & 7) | (xi < 0.0 ? 8 : 0);
+        }
+        packed[r * (K / 2) + b * 8 + j] = (uint8_t)(nib[0] | (nib[1] << 4));
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+int orc_nvfp4_quantize_mse(const void* x, int dtype, int64_t rows, int64_t K, uint8_t* packed,
+                           uint8_t* block_scales, float* global_scale) {
+  if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  double amax = 0.0;
+  for (int64_t i = 0; i < rows * K; ++i) {
+    double a = fabs(load_elem(x, dtype, i));
+    if (a > amax) amax = a;
+  }
+  double g = amax == 0.0 ? 0.0 : orc_nvfp4_global_scale(amax);
+  *global_scale = (float)g;
+  return orc_nvfp4_quantize_mse_rows(x, dtype, rows, K, g, packed, block_scales);
+}

@@ -594,3 +594,176 @@ def test_nvfp4_zero_tensor():
     bits = np.zeros((2, 32), np.uint16)
     p, s, g = oracle.nvfp4_quantize(bits)
     assert g == 0.0 and (p == 0).all() and (s == 0x38).all()  # 0x38 is E4M3 1.0
+
+
+# ----------------------------------------------------- packed cache storage
+
+@pytest.mark.parametrize("fmt,B", [("fp8", 128), ("fp8", 32), ("mxfp4", 32), ("nvfp4", 16)])
+def test_packed_cache_unpacks_to_the_fake_quantization(fmt, B):
+    x = torch.cat([gen.kv_cache((1, 8, 256)).view(8, 256), gen.mixed_blocks(8, 256)])
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    codes, scales = oracle.quantize_cache_packed(bits, fmt, B)
+    back = oracle.dequantize_cache_packed(codes, scales, fmt, B, 256)
+    assert np.array_equal(back, oracle.quantize_cache(bits, fmt, B))
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "mxfp4", "nvfp4"])
+def test_packed_cache_scale_bytes_decode_to_the_power_of_two(fmt):
+    lo, hi = CLAMP[fmt]
+    for k in range(lo, hi + 1):
+        b = oracle.cache_scale_byte(k, fmt)
+        if fmt == "nvfp4":
+            v = torch.tensor([b], dtype=torch.uint8).view(torch.float8_e4m3fn).float().item()
+        else:
+            v = 2.0 ** (b - 127)
+        assert v == 2.0 ** k, (fmt, k, b)
+
+
+def test_packed_cache_codes_follow_the_element_casts():
+    x = gen.kv_cache((1, 4, 128)).view(4, 128)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    xv = oracle.decode(bits, "bf16")
+    codes, scales = oracle.quantize_cache_packed(bits, "fp8", 32)
+    ks = scales.astype(int) - 127
+    s = np.repeat(2.0 ** ks, 32, axis=1)
+    want = torch.from_numpy((xv / s).astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(codes, want.view(torch.uint8).numpy())
+    c4, s4 = oracle.quantize_cache_packed(bits, "mxfp4", 32)
+    k4 = np.repeat(s4.astype(int) - 127, 32, axis=1)
+    v = xv / 2.0 ** k4
+    nib = np.stack([c4 & 15, c4 >> 4], axis=-1).reshape(4, 128)
+    mag = bruteforce_e2m1_mag(np.abs(v).reshape(-1)).reshape(4, 128)
+    assert np.array_equal(nib, mag | np.where(xv < 0, 8, 0))
+
+
+# ----------------------------------------------------- NVFP4 mse block scale
+
+from fractions import Fraction  # noqa: E402
+
+E4M3_VALUE = dict((int(c), float(v)) for v, c in zip(*e4m3_candidates()))
+
+
+def exact_block_errors(w, g):
+    """Exact (rational) squared error of a 16-block for each of the 126
+    codes, with the page's binary32 steps done by numpy float32 and the
+    E2M1 cast by brute force; None where d underflows to zero."""
+    f32 = np.float32
+    out = {}
+    for c in range(1, 127):
+        d = f32(E4M3_VALUE[c]) * f32(g)
+        if d == 0:
+            out[c] = None
+            continue
+        v = np.abs(w.astype(np.float32) / d).astype(np.float64)
+        q = T8[bruteforce_e2m1_mag(np.minimum(v, 1e30))] * np.where(w < 0, -1.0, 1.0)
+        out[c] = sum((Fraction(float(qi)) * Fraction(float(d)) - Fraction(float(wi))) ** 2
+                     for qi, wi in zip(q, w))
+    return out
+
+
+def mse_blocks(n_rows=6):
+    x = torch.cat([gen.expert_weights(1, n_rows, 64).view(n_rows, 64),
+                   gen.mixed_blocks(2, 64), gen.normal_bf16(41, (2, 64))])
+    return x.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_mse_block_error_is_the_exact_sum():
+    bits = mse_blocks(2)
+    xv = oracle.decode(bits, "bf16")
+    g = oracle.nvfp4_global_scale(np.abs(xv).max())
+    for w in xv.reshape(-1, 16)[:10]:
+        exact = exact_block_errors(w, g)
+        for c in (1, 17, 40, 56, 77, 100, 126):
+            got = oracle.nvfp4_block_sq_error(w, g, c)
+            if exact[c] is None:
+                assert got == math.inf
+            else:
+                # 16 double roundings of a sum of non-negative terms
+                assert abs(Fraction(got) - exact[c]) <= exact[c] * Fraction(16, 2**52)
+
+
+def test_mse_code_is_the_first_exact_minimum():
+    bits = mse_blocks()
+    xv = oracle.decode(bits, "bf16")
+    p, s, g = oracle.nvfp4_quantize_mse(bits)
+    assert g == oracle.nvfp4_global_scale(np.abs(xv).max())
+    blocks = xv.reshape(-1, 16)
+    for b, w in enumerate(blocks):
+        exact = {c: e for c, e in exact_block_errors(w, g).items() if e is not None}
+        best = min(exact.values())
+        c = int(s.reshape(-1)[b])
+        slack = best * Fraction(32, 2**52)
+        assert exact[c] <= best + slack, b
+        # no smaller code is clearly better, nor exactly as good (ties go
+        # to the first code)
+        assert all(exact[k] > exact[c] - slack for k in exact if k < c), b
+        assert not any(exact[k] == exact[c] for k in exact if k < c), b
+
+
+def test_mse_never_worse_than_the_max_rule():
+    bits = mse_blocks()
+    xv = oracle.decode(bits, "bf16")
+    _, s_mse, g = oracle.nvfp4_quantize_mse(bits)
+    _, s_max, g2 = oracle.nvfp4_quantize(bits)
+    assert g == g2
+    for b, w in enumerate(xv.reshape(-1, 16)):
+        e = exact_block_errors(w, g)
+        cm, cx = int(s_mse.reshape(-1)[b]), int(s_max.reshape(-1)[b])
+        assert e[cm] <= e[cx] * (1 + Fraction(32, 2**52)), b
+
+
+def test_mse_codes_follow_the_chosen_scale():
+    # the packed codes are the max rule's element cast under the chosen scale
+    bits = mse_blocks()
+    xv = oracle.decode(bits, "bf16")
+    p, s, g = oracle.nvfp4_quantize_mse(bits)
+    f32 = np.float32
+    rows, K = xv.shape
+    for r in range(rows):
+        for b in range(K // 16):
+            d = f32(E4M3_VALUE[int(s[r, b])]) * f32(g)
+            for j in range(16):
+                v = float(f32(xv[r, 16 * b + j]) / d)
+                want = 0 if xv[r, 16 * b + j] == 0 else (
+                    e2m1_bruteforce_code(abs(v)) | (8 if xv[r, 16 * b + j] < 0 else 0))
+                byte = p[r, 8 * b + j // 2]
+                assert (byte >> (4 * (j % 2))) & 15 == want, (r, b, j)
+
+
+def test_mse_block_on_the_grid_has_zero_error():
+    # g = 2^-10 exactly (amax 2.625 = 2688 * 2^-10); a block built as
+    # E2M1 values times d = s_c * g for c = 0x30 (1.0) is reconstructed
+    # exactly, so the chosen code has zero error
+    grid = np.array([6, 4, 3, -2, 1.5, 1, 0.5, 0, -6, -4, 3, 2, -1.5, 1, -0.5, 6])
+    d = E4M3_VALUE[0x30] * 2.0**-10
+    blk = grid * d
+    other = np.zeros(16)
+    other[3] = 2.625
+    xv = np.stack([np.concatenate([blk, other])])
+    bits = torch.from_numpy(xv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.decode(bits, "bf16"), xv)  # exact in bf16
+    p, s, g = oracle.nvfp4_quantize_mse(bits)
+    assert g == 2.0**-10
+    c = int(s[0, 0])
+    assert c <= 0x30 and exact_block_errors(xv[0, :16], g)[c] == 0
+    assert oracle.nvfp4_block_sq_error(xv[0, :16], g, c) == 0.0
+
+
+def test_mse_zero_block_and_zero_tensor():
+    bits = mse_blocks(1).copy()
+    bits[0, 16:32] = 0
+    p, s, g = oracle.nvfp4_quantize_mse(bits)
+    assert s[0, 1] == 0x01 and (p[0, 8:16] == 0).all()  # every code ties at 0: the first
+    p, s, g = oracle.nvfp4_quantize_mse(np.zeros((2, 32), np.uint16))
+    assert g == 0.0 and (p == 0).all() and (s == 0x38).all()
+
+
+def test_mse_moves_codes_both_ways():
+    # the page: under the sweep some blocks take a smaller code than the max
+    # rule (clipping their largest value) and others a larger one
+    x = gen.expert_weights(1, 16, 512).view(16, 512)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    _, s_mse, _ = oracle.nvfp4_quantize_mse(bits)
+    _, s_max, _ = oracle.nvfp4_quantize(bits)
+    diff = s_mse.astype(int) - s_max.astype(int)
+    assert (diff < 0).any() and (diff > 0).any()
