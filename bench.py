@@ -203,17 +203,28 @@ class Step:
                 ev[i][1].record()
 
 
-def time_next_rows(torch, mxq, step, dev, reps=5):
+def time_next_rows(torch, mxq, step, dev, reps=3):
     """Device time (ms, mean over reps, max over ranks) of the next-row
-    kernels on the expert weights: NVFP4 two-level quantize and dequantize.
-    Timed after, and outside, the main step."""
+    kernels: NVFP4 two-level quantize (max and mse block-scale rules) and
+    dequantize on the expert weights; packed cache quantize / unpack on the
+    three KV-cache tensors.  Timed after, and outside, the main step."""
     packed, bscales, g = mxq.nvfp4_quantize(step.W)
+    packed2, bscales2, g2 = mxq.nvfp4_quantize(step.W)
     ws = torch.empty(16, dtype=torch.uint8, device=dev)
     calls = {
         "nvfp4_quantize": lambda: mxq.nvfp4_quantize(step.W, packed, bscales, g, ws),
+        "nvfp4_quantize_mse": lambda: mxq.nvfp4_quantize(step.W, packed2, bscales2, g2, ws,
+                                                         rule="mse"),
         "nvfp4_dequantize": lambda: mxq.nvfp4_dequantize(packed, bscales, g, torch.bfloat16,
                                                          step.Wout),
     }
+    for i, (f, b) in enumerate(CACHE_RUNS):
+        codes, sc = mxq.quantize_cache_packed(step.kv[i], f, b)
+        calls["cache_pack_" + f] = (
+            lambda i=i, f=f, b=b, c=codes, s=sc: mxq.quantize_cache_packed(step.kv[i], f, b, c, s))
+        calls["cache_unpack_" + f] = (
+            lambda i=i, f=f, b=b, c=codes, s=sc: mxq.dequantize_cache_packed(
+                c, s, f, b, torch.bfloat16, step.kv_out[i]))
     out = {}
     for name, fn in calls.items():
         for _ in range(2):
@@ -229,6 +240,22 @@ def time_next_rows(torch, mxq, step, dev, reps=5):
     names = list(out)
     vals = max_over_ranks([out[n] for n in names], dev)
     return dict(zip(names, vals))
+
+
+def next_row_bytes():
+    """Algorithmic HBM bytes of each next-row call (bf16 inputs/outputs)."""
+    w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
+    n = KV_SHAPE[0] * KV_SHAPE[1] * KV_SHAPE[2]
+    # NVFP4 quantize: the per-tensor scale needs the whole tensor's maximum
+    # first, so x is read twice; packed codes + E4M3 scales written once
+    nb = {"nvfp4_quantize": 2 * 2 * w + w // 2 + w // 16,
+          "nvfp4_quantize_mse": 2 * 2 * w + w // 2 + w // 16,
+          "nvfp4_dequantize": w // 2 + w // 16 + 2 * w}
+    for f, b in CACHE_RUNS:
+        stored = (n if f == "fp8" else n // 2) + n // b
+        nb["cache_pack_" + f] = 2 * n + stored
+        nb["cache_unpack_" + f] = stored + 2 * n
+    return nb
 
 
 def time_e2e(torch, mxq, step, steps):
@@ -385,16 +412,20 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         "clocks": clocks,
     }
     if next_ms:
+        nb = next_row_bytes()
         w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
-        # quantize: the per-tensor scale needs the whole tensor's maximum
-        # first, so x is read twice; packed codes + E4M3 scales written once
-        nb = {"nvfp4_quantize": 2 * 2 * w + w // 2 + w // 16,
-              "nvfp4_dequantize": w // 2 + w // 16 + 2 * w}
-        line["next_rows"] = {
-            n: {"ms": round(ms, 4), "gbs": round(nb[n] / (ms * 1e-3) / 1e9, 1),
-                "frac": round(nb[n] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                "workload": "bf16 [64,2048,7168] expert weights"}
-            for n, ms in next_ms.items()}
+        rows = {}
+        for n, ms in next_ms.items():
+            gbs = nb[n] / (ms * 1e-3) / 1e9
+            rows[n] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                       "frac": round(gbs / peaks["hbm_gbs"], 4),
+                       "workload": ("bf16 [64,2048,7168] expert weights" if n.startswith("nvfp4")
+                                    else "bf16 [4,8192,512] KV cache")}
+        # the sweep is arithmetic: 126 candidate scales x 16 weights per block
+        rows["nvfp4_quantize_mse"]["bound"] = "alu"
+        rows["nvfp4_quantize_mse"]["g_candidates_per_s"] = round(
+            126 * w / (next_ms["nvfp4_quantize_mse"] * 1e-3) / 1e9, 1)
+        line["next_rows"] = rows
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     print(json.dumps(line), flush=True)

@@ -108,9 +108,45 @@ int mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t 
  *  Fast path: block_size in {8,16,32,64,128,256}, channels % block_size == 0,
  *  16-byte aligned in/out.  Anything else runs a slower general kernel.
  *  Errors: block_size < 1 -> MXQ_ERR_SHAPE; bad format/dtype or overlapping
- *  in/out -> MXQ_ERR_INVALID_ARG. */
+ *  in/out -> MXQ_ERR_INVALID_ARG; in/out not aligned to the element size ->
+ *  MXQ_ERR_ALIGNMENT. */
 int quantize_cache(const void* in, void* out, int dtype, int64_t rows, int64_t channels,
                    int format, int32_t block_size, void* stream);
+
+/* Packed (stored) cache quantization ([CQ] _CacheQuantization.forward:
+ * fp8; mxfp4 with an E8M0 scale; nvfp4 with an E4M3 scale).  Keeps the codes
+ * and scales that quantize_cache rounds to instead of multiplying back.
+ *
+ *  in       device, [rows, channels] elements of dtype (bf16, f16 or f32).
+ *  codes    device (output).  fp8: [rows, channels] E4M3 bytes (the cast of
+ *           x / 2^k, sign of zero kept).  mxfp4, nvfp4: [rows, channels/2]
+ *           bytes of two E2M1 codes, the even channel in the low nibble, sign
+ *           bit iff x < 0 (as mx_quantize).
+ *  scales   device, [rows, channels/block_size] bytes (output): the group's
+ *           scale 2^k (k chosen exactly as in quantize_cache) as an E8M0 byte
+ *           k + 127 for fp8 and mxfp4, as the E4M3 encoding of 2^k for nvfp4
+ *           (k in [-9, 8] is always an E4M3 value).
+ *  block_size  channels per scale; channels % block_size == 0 (no partial
+ *           group is stored) and, for mxfp4/nvfp4, block_size even.
+ *  dequantize_cache_packed(quantize_cache_packed(x)) equals
+ *  quantize_cache(x) bit for bit.
+ *  Fast path: block_size in {8,...,256} a power of two, 16-byte aligned in
+ *  and codes; anything else valid runs a slower general kernel.
+ *  Errors: bad dtype/format or null pointer -> MXQ_ERR_INVALID_ARG;
+ *  block_size < 1, channels % block_size != 0 or an odd fp4 block_size ->
+ *  MXQ_ERR_SHAPE; in not aligned to its element size -> MXQ_ERR_ALIGNMENT.
+ *  rows == 0 or channels == 0: no-op. */
+int quantize_cache_packed(const void* in, int dtype, int64_t rows, int64_t channels, int format,
+                          int32_t block_size, void* codes, void* scales, void* stream);
+
+/* Unpack the stored cache form: out = round_dtype(code value * scale), the
+ * product taken in f32 (exact for every code and scale the packer writes).
+ * fp4 zero codes (either sign) give +0.0; an E8M0 byte 0xFF gives NaN.
+ * Arguments, layout and errors as quantize_cache_packed, with out
+ * [rows, channels] of out_dtype. */
+int dequantize_cache_packed(const void* codes, const void* scales, int64_t rows, int64_t channels,
+                            int format, int32_t block_size, void* out, int out_dtype,
+                            void* stream);
 
 /* Grouped GEMM over MXFP4-packed expert weights, dequantized on the fly
  * ([MX] MXFP4GroupedMM forward and backward).
@@ -172,6 +208,24 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
  *  Errors as for nvfp4_quantize. */
 int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                      int64_t rows, int64_t K, void* out, int out_dtype, void* stream);
+
+/* NVFP4 quantize + pack with block scales chosen by least squared weight
+ * error ([MO] "NVFP4's own rules", the mse rule).
+ *
+ *  Arguments, layout, workspace, errors and the precondition as
+ *  nvfp4_quantize; g is the same max|x| / 2688.  Each 16-block tries the
+ *  126 positive finite E4M3 codes c (bytes 0x01..0x7E) as its scale: with
+ *  d = s_c * g (binary32), every x is cast to E2M1 as nvfp4_quantize casts
+ *  it (binary32 quotient x / d), the error (q * d - x) is formed exactly in
+ *  double and the squares are summed over the block in column order by
+ *  double fmas.  The block keeps the code with the least sum, the smallest
+ *  code among equal sums (so an all-zero block takes 0x01), and its codes
+ *  are E2M1(x / d) of that code (a zero x gives code 0).  A code whose d
+ *  underflows to 0 is not a candidate.  An all-zero tensor gives the
+ *  nvfp4_quantize output (g = 0, codes 0, block scales 1.0).
+ *  The result is read back with nvfp4_dequantize. */
+int nvfp4_quantize_mse(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                       void* block_scales, float* global_scale, void* workspace, void* stream);
 
 /* Size of the library's own static device scratch used by
  * nvfp4_quantize_noalloc (bytes per GPU, held from library load to exit). */

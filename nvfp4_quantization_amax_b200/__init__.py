@@ -12,6 +12,7 @@ current CUDA device (asynchronously when pinned), processed there, and the
 results are copied back to host memory before the call returns.
 """
 from ._abi import (  # noqa: F401
+    CacheQuantization,
     MxqError,
     lib,
     lib_path,
@@ -20,7 +21,9 @@ from ._abi import (  # noqa: F401
     mxfp4_grouped_mm,
     nvfp4_dequantize,
     nvfp4_quantize,
+    dequantize_cache_packed,
     quantize_cache,
+    quantize_cache_packed,
     set_wait_limit_ns,
     status_string,
 )

@@ -46,10 +46,16 @@ def lib():
         L.mxq_version.argtypes = []
         L.nvfp4_quantize.restype = i
         L.nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p, p, p]
+        L.nvfp4_quantize_mse.restype = i
+        L.nvfp4_quantize_mse.argtypes = [p, i, i64, i64, p, p, p, p, p]
         L.nvfp4_quantize_noalloc.restype = i
         L.nvfp4_quantize_noalloc.argtypes = [p, i, i64, i64, p, p, p, p]
         L.nvfp4_dequantize.restype = i
         L.nvfp4_dequantize.argtypes = [p, p, p, i64, i64, p, i, p]
+        L.quantize_cache_packed.restype = i
+        L.quantize_cache_packed.argtypes = [p, i, i64, i64, i, i32, p, p, p]
+        L.dequantize_cache_packed.restype = i
+        L.dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i32, p, i, p]
         L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64
         L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
@@ -161,6 +167,72 @@ def quantize_cache(values, format, block_size, out=None):
     return _to_host(out) if host else out
 
 
+def quantize_cache_packed(values, format, block_size, codes=None, scales=None):
+    """Stored form of quantize_cache: returns (codes, scales) uint8.
+
+    codes: fp8 -> [..., C] E4M3 bytes; mxfp4/nvfp4 -> [..., C/2] bytes of two
+    E2M1 codes (low nibble = even channel).  scales: [..., C/block_size],
+    E8M0 bytes for fp8 and mxfp4, E4M3 bytes for nvfp4.  C % block_size == 0.
+    """
+    if values.dtype not in _DTYPES:
+        raise TypeError("quantize_cache_packed: unsupported dtype %s" % values.dtype)
+    if format not in _FORMATS:
+        raise ValueError("quantize_cache_packed: format must be one of %s" % sorted(_FORMATS))
+    values, host = _to_device(values)
+    values = values.contiguous()
+    C = values.shape[-1] if values.dim() else 1
+    rows = values.numel() // C if C else 0
+    B = int(block_size)
+    lead = tuple(values.shape[:-1])
+    dev = values.device
+    if codes is None:
+        codes = torch.empty(lead + (C if format == "fp8" else C // 2,), dtype=torch.uint8,
+                            device=dev)
+    if scales is None:
+        scales = torch.empty(lead + (C // B if B > 0 else 0,), dtype=torch.uint8, device=dev)
+    rc = lib().quantize_cache_packed(_ptr(values), _DTYPES[values.dtype], rows, C,
+                                     _FORMATS[format], B, _ptr(codes), _ptr(scales), _stream(dev))
+    _check(rc, "quantize_cache_packed")
+    if host:
+        return _to_host(codes), _to_host(scales)
+    return codes, scales
+
+
+def dequantize_cache_packed(codes, scales, format, block_size, dtype=torch.bfloat16, out=None):
+    """Unpack the stored cache form to dtype [..., C] (C from the scales)."""
+    if dtype not in _DTYPES:
+        raise TypeError("dequantize_cache_packed: unsupported dtype %s" % dtype)
+    if format not in _FORMATS:
+        raise ValueError("dequantize_cache_packed: format must be one of %s" % sorted(_FORMATS))
+    codes, host = _to_device(codes)
+    scales, _ = _to_device(scales)
+    codes, scales = codes.contiguous(), scales.contiguous()
+    B = int(block_size)
+    C = scales.shape[-1] * B
+    rows = scales.numel() // scales.shape[-1] if scales.shape[-1] else 0
+    if codes.numel() != rows * (C if format == "fp8" else C // 2):
+        raise ValueError("dequantize_cache_packed: codes do not match the scales' shape")
+    if out is None:
+        out = torch.empty(tuple(scales.shape[:-1]) + (C,), dtype=dtype, device=codes.device)
+    rc = lib().dequantize_cache_packed(_ptr(codes), _ptr(scales), rows, C, _FORMATS[format], B,
+                                       _ptr(out), _DTYPES[dtype], _stream(codes.device))
+    _check(rc, "dequantize_cache_packed")
+    return _to_host(out) if host else out
+
+
+class CacheQuantization(torch.autograd.Function):
+    """quantize_cache in the forward pass, the gradient passed through
+    unchanged in the backward pass (straight-through estimator)."""
+
+    @staticmethod
+    def forward(ctx, values, block_size, format):
+        return quantize_cache(values, format, block_size)
+
+    @staticmethod
+    def backward(ctx, gradient):
+        return gradient, None, None
+
+
 def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, status=None):
     """Grouped GEMM over MXFP4-packed expert weights.
 
@@ -199,15 +271,20 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
 NVFP4_WORKSPACE_BYTES = 16
 
 
-def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspace=None):
+def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspace=None,
+                   rule="max"):
     """NVFP4 two-level quantize + pack along the last dim (K % 16 == 0).
 
     Returns (packed uint8 [..., K/2], E4M3 block scales uint8 [..., K/16],
     global scale float32 [1]); the per-tensor scale is g = max|x| / 2688.
+    rule "max": s_b = E4M3(amax_b / (6 g)); rule "mse": the E4M3 code with
+    the least squared weight error per block.
     `workspace` (device uint8, at least NVFP4_WORKSPACE_BYTES) is scratch.
     """
     if x.dtype not in _DTYPES:
         raise TypeError("nvfp4_quantize: unsupported dtype %s" % x.dtype)
+    if rule not in ("max", "mse"):
+        raise ValueError("nvfp4_quantize: rule must be 'max' or 'mse'")
     x, host = _to_device(x)
     x = x.contiguous()
     K = x.shape[-1]
@@ -221,10 +298,10 @@ def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspa
         global_scale = torch.empty(1, dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = torch.empty(NVFP4_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
-    rc = lib().nvfp4_quantize(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed),
-                              _ptr(block_scales), _ptr(global_scale), _ptr(workspace),
-                              _stream(dev))
-    _check(rc, "nvfp4_quantize")
+    fn = lib().nvfp4_quantize if rule == "max" else lib().nvfp4_quantize_mse
+    rc = fn(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed), _ptr(block_scales),
+            _ptr(global_scale), _ptr(workspace), _stream(dev))
+    _check(rc, "nvfp4_quantize" if rule == "max" else "nvfp4_quantize_mse")
     if host:
         return _to_host(packed), _to_host(block_scales), _to_host(global_scale)
     return packed, block_scales, global_scale

@@ -27,6 +27,10 @@ int num_sms() {
 }
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+// Elements must sit on their own size (2 or 4 bytes) for the general kernels.
+static bool elem_aligned(const void* p, int d) {
+  return ((uintptr_t)p & (uintptr_t)((d == MXQ_F32 ? 4 : 2) - 1)) == 0;
+}
 static bool valid_dtype(int d) { return d == MXQ_BF16 || d == MXQ_F16 || d == MXQ_F32; }
 static int elem_bytes(int d) { return d == MXQ_F32 ? 4 : 2; }
 
@@ -71,11 +75,49 @@ int quantize_cache(const void* in, void* out, int dtype, int64_t rows, int64_t c
   if (!in || !out) return MXQ_ERR_INVALID_ARG;
   int64_t bytes = rows * channels * elem_bytes(dtype);
   if (overlap(in, bytes, out, bytes)) return MXQ_ERR_INVALID_ARG;
+  if (!elem_aligned(in, dtype) || !elem_aligned(out, dtype)) return MXQ_ERR_ALIGNMENT;
   int B = block_size;
   bool pow2_b = B >= 8 && B <= 256 && (B & (B - 1)) == 0;
   bool fast = pow2_b && channels % B == 0 && aligned16(in) && aligned16(out);
   return launch_quantize_cache(in, out, dtype, rows, channels, format, B, fast,
                                (cudaStream_t)stream);
+}
+
+static int check_packed_cache(int dtype, int64_t rows, int64_t C, int format, int32_t B) {
+  if (!valid_dtype(dtype)) return MXQ_ERR_INVALID_ARG;
+  if (format != MXQ_FMT_FP8 && format != MXQ_FMT_MXFP4 && format != MXQ_FMT_NVFP4)
+    return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || C < 0 || B < 1 || C % B != 0) return MXQ_ERR_SHAPE;
+  if (format != MXQ_FMT_FP8 && B % 2 != 0) return MXQ_ERR_SHAPE;
+  return MXQ_OK;
+}
+
+static bool packed_fast(int32_t B, const void* elems, const void* codes) {
+  return B >= 8 && B <= 256 && (B & (B - 1)) == 0 && aligned16(elems) && aligned16(codes);
+}
+
+int quantize_cache_packed(const void* in, int dtype, int64_t rows, int64_t channels, int format,
+                          int32_t block_size, void* codes, void* scales, void* stream) {
+  int rc = check_packed_cache(dtype, rows, channels, format, block_size);
+  if (rc != MXQ_OK) return rc;
+  if (rows == 0 || channels == 0) return MXQ_OK;
+  if (!in || !codes || !scales) return MXQ_ERR_INVALID_ARG;
+  if (!elem_aligned(in, dtype)) return MXQ_ERR_ALIGNMENT;
+  return launch_quantize_cache_packed(in, dtype, rows, channels, format, block_size, codes, scales,
+                                      packed_fast(block_size, in, codes), (cudaStream_t)stream);
+}
+
+int dequantize_cache_packed(const void* codes, const void* scales, int64_t rows, int64_t channels,
+                            int format, int32_t block_size, void* out, int out_dtype,
+                            void* stream) {
+  int rc = check_packed_cache(out_dtype, rows, channels, format, block_size);
+  if (rc != MXQ_OK) return rc;
+  if (rows == 0 || channels == 0) return MXQ_OK;
+  if (!codes || !scales || !out) return MXQ_ERR_INVALID_ARG;
+  if (!elem_aligned(out, out_dtype)) return MXQ_ERR_ALIGNMENT;
+  return launch_dequantize_cache_packed(codes, scales, rows, channels, format, block_size, out,
+                                        out_dtype, packed_fast(block_size, out, codes),
+                                        (cudaStream_t)stream);
 }
 
 int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
@@ -101,6 +143,18 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
     return MXQ_ERR_ALIGNMENT;
   return launch_nvfp4_quantize(x, x_dtype, rows, K, packed, block_scales, global_scale,
                                (uint32_t*)workspace, (cudaStream_t)stream);
+}
+
+int nvfp4_quantize_mse(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
+                       void* block_scales, float* global_scale, void* workspace, void* stream) {
+  if (!valid_dtype(x_dtype)) return MXQ_ERR_INVALID_ARG;
+  if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
+  if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
+    return MXQ_ERR_ALIGNMENT;
+  return launch_nvfp4_quantize_mse(x, x_dtype, rows, K, packed, block_scales, global_scale,
+                                   (uint32_t*)workspace, (cudaStream_t)stream);
 }
 
 int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,

@@ -16,9 +16,20 @@ int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, i
                          int dt, cudaStream_t st);
 int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64_t C, int fmt,
                           int B, bool fast, cudaStream_t st);
+int launch_quantize_cache_packed(const void* in, int dt, int64_t rows, int64_t C, int fmt, int B,
+                                 void* codes, void* scales, bool fast, cudaStream_t st);
+int launch_dequantize_cache_packed(const void* codes, const void* scales, int64_t rows, int64_t C,
+                                   int fmt, int B, void* out, int dt, bool fast, cudaStream_t st);
 int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed,
                           void* block_scales, float* global_scale, uint32_t* amax_word,
                           cudaStream_t st);
+// Clear *amax_word, then atomicMax into it the binary32 bits of max |x| over
+// n_elems elements (n_elems % 8 == 0; 16-byte aligned x).
+void launch_nvfp4_amax(const void* x, int dt, int64_t n_elems, uint32_t* amax_word,
+                       cudaStream_t st);
+int launch_nvfp4_quantize_mse(const void* x, int dt, int64_t rows, int64_t K, void* packed,
+                              void* block_scales, float* global_scale, uint32_t* amax_word,
+                              cudaStream_t st);
 // Device address of the static scratch of the allocation-free entry point on
 // the current device (looked up once per device), or nullptr on failure.
 uint32_t* noalloc_scratch(size_t need_bytes, int* status);

@@ -177,14 +177,19 @@ int grid_for(int64_t n_units, int per_block, int resident) {
 }
 
 template <int DT>
-int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* block_scales,
-                 float* global_scale, uint32_t* amax_word, cudaStream_t st) {
-  const int64_t n_items = rows * (K / 8);
+void run_amax(const void* x, int64_t n_items, uint32_t* amax_word, cudaStream_t st) {
   clear_word_kernel<<<1, 1, 0, st>>>(amax_word);
   if (n_items > 0) {
     nvfp4_amax_kernel<DT><<<grid_for(n_items, kNvThreads * 4, 8), kNvThreads, 0, st>>>(
         x, n_items, amax_word);
   }
+}
+
+template <int DT>
+int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* block_scales,
+                 float* global_scale, uint32_t* amax_word, cudaStream_t st) {
+  const int64_t n_items = rows * (K / 8);
+  run_amax<DT>(x, n_items, amax_word, st);
   nvfp4_quantize_kernel<DT><<<grid_for(n_items, kNvThreads * kNvUnroll, 4), kNvThreads, 0, st>>>(
       x, (uint32_t*)packed, (uint8_t*)block_scales, global_scale, amax_word, n_items);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
@@ -230,6 +235,15 @@ int launch_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K, void* 
     case kBF16: return run_quantize<kBF16>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
     case kF16: return run_quantize<kF16>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
     default: return run_quantize<kF32>(x, rows, K, packed, block_scales, global_scale, amax_word, st);
+  }
+}
+
+void launch_nvfp4_amax(const void* x, int dt, int64_t n_elems, uint32_t* amax_word,
+                       cudaStream_t st) {
+  switch (dt) {
+    case kBF16: run_amax<kBF16>(x, n_elems / 8, amax_word, st); break;
+    case kF16: run_amax<kF16>(x, n_elems / 8, amax_word, st); break;
+    default: run_amax<kF32>(x, n_elems / 8, amax_word, st); break;
   }
 }
 

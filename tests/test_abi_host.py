@@ -133,3 +133,41 @@ def test_nvfp4_noalloc_validation_needs_no_gpu(L):
     assert L.nvfp4_quantize_noalloc(A1, 0, 4, 64, A2, A2, NULL, NULL) == EARG
     assert L.nvfp4_quantize_noalloc(BAD, 0, 4, 64, A2, A2, A2, NULL) == EALIGN
     assert L.nvfp4_quantize_noalloc(A1, 5, 4, 64, A2, A2, A2, NULL) == EARG
+
+
+def test_packed_cache_validation(L):
+    q, d = L.quantize_cache_packed, L.dequantize_cache_packed
+    assert q(A1, 0, 4, 64, 3, 32, A2, A2, NULL) == EARG  # format
+    assert q(A1, 7, 4, 64, 0, 32, A2, A2, NULL) == EARG  # dtype
+    assert q(A1, 0, 4, 64, 0, 0, A2, A2, NULL) == ESHAPE  # block_size < 1
+    assert q(A1, 0, 4, 60, 0, 32, A2, A2, NULL) == ESHAPE  # no partial group is stored
+    assert q(A1, 0, 4, 63, 1, 21, A2, A2, NULL) == ESHAPE  # odd fp4 block
+    assert q(A1, 0, -1, 64, 0, 32, A2, A2, NULL) == ESHAPE
+    assert q(A1, 0, 4, 64, 0, 32, NULL, A2, NULL) == EARG
+    assert q(BAD, 0, 4, 64, 0, 32, A2, A2, NULL) == EALIGN  # element alignment
+    assert q(NULL, 0, 0, 64, 0, 32, NULL, NULL, NULL) == OK  # rows == 0: no-op
+    assert d(A1, A2, 4, 64, 2, 16, BAD, 0, NULL) == EALIGN
+    assert d(A1, A2, 4, 64, 2, 15, A1, 0, NULL) == ESHAPE
+    assert d(A1, NULL, 4, 64, 2, 16, A1, 0, NULL) == EARG
+    assert d(NULL, NULL, 4, 0, 2, 16, NULL, 0, NULL) == OK
+
+
+def test_cache_quantization_function_passes_the_gradient_through():
+    # backward alone needs no GPU: the straight-through gradient is returned
+    # unchanged with no gradients for block_size and format
+    import torch
+    g = torch.randn(3, 64)
+    out = mxq.CacheQuantization.backward(None, g)
+    assert out[0] is g and out[1] is None and out[2] is None
+
+
+def test_nvfp4_mse_validation(L):
+    f = L.nvfp4_quantize_mse
+    assert f(A1, 0, 4, 40, A2, A2, A2, A1, NULL) == ESHAPE
+    assert f(A1, 0, 4, 64, A2, A2, A2, NULL, NULL) == EARG  # workspace
+    assert f(A1, 0, 4, 64, A2, A2, NULL, A1, NULL) == EARG  # global scale
+    assert f(BAD, 0, 4, 64, A2, A2, A2, A1, NULL) == EALIGN
+    assert f(A1, 3, 4, 64, A2, A2, A2, A1, NULL) == EARG
+    with pytest.raises(ValueError):
+        import torch
+        mxq.nvfp4_quantize(torch.zeros(2, 16, dtype=torch.bfloat16), rule="least")
