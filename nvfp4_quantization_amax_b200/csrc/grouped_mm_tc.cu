@@ -66,6 +66,8 @@ constexpr int kMmaWarp = 13;
 constexpr int kThreads = 14 * 32;
 constexpr uint32_t kStagingBytes = kBN * kBM * 2;   // 64 KB
 constexpr int kMaxSmemExperts = 4096;               // offs cached in smem up to this E
+constexpr int kMaxSmemExpertsDgrad = 256;           // (the input gradient's smem holds W stages)
+constexpr int kWStages = 3;                         // packed-weight stages of the input gradient
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 constexpr uint64_t kAbortSettleNs = 50000ull;
 
@@ -86,6 +88,14 @@ struct Geo {
   static constexpr int kStages = 4;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
+  // Input gradient: the packed weight tile of a stage (kBK rows n x 64
+  // bytes = 128 features k, 64-byte swizzled) and its scale bytes (a
+  // 16-byte box per row) arrive by TMA into kWStages slots.
+  static constexpr uint32_t kWBytes = kBK * 64;
+  static constexpr uint32_t kSBytes = kBK * 16;
+  static constexpr uint32_t kSmemDgrad = 1024 + kStages * kStageBytes +
+                                         kWStages * (kWBytes + kSBytes) + kStagingBytes + 256 +
+                                         4 * kMaxSmemExpertsDgrad;
   // Token count of a tile rounded to what the MMA accepts.
   __host__ __device__ static int64_t mma_n(int64_t rows) {
     return kPair ? (rows + 31) & ~31 : (rows + 15) & ~15;
@@ -96,6 +106,8 @@ struct Shared {
   uint64_t full_a[kMaxStages];
   uint64_t full_b[kMaxStages];
   uint64_t empty[kMaxStages];
+  uint64_t wfull[kWStages];   // packed weights (+ scales) of a stage landed
+  uint64_t wempty[kWStages];  // the dequantization warps are done with a slot
   uint64_t d_full, d_empty, drain;
   uint32_t tmem_base;
   int abort;
@@ -113,6 +125,13 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t byte, float scale) {
 
 __device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
+}
+
+// Input gradient: the feature held by TMEM lane L of a warp's 32.  Lane
+// L = 8c + r carries row r of the transposed 8x8 block c, whose rows are
+// the features k = 8(r >> 1) + 2c + (r & 1) (see the dequantization warps).
+__device__ __forceinline__ int kperm(int L) {
+  return ((L & 6) << 2) | ((L >> 3) << 1) | (L & 1);
 }
 
 // Named barrier 1 over the four epilogue warps (threads 0..127).
@@ -157,18 +176,24 @@ __device__ __forceinline__ void arrive_leader(uint64_t* bar) {
 
 template <bool kDgrad, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t* __restrict__ packed,
+grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
+                     const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_s, const uint8_t* __restrict__ packed,
                      const uint8_t* __restrict__ scales, const int32_t* __restrict__ offs, int64_t T,
                      int64_t E, int64_t N, int64_t K, __nv_bfloat16* __restrict__ y,
-                     int32_t* dev_status, uint64_t wait_limit_ns) {
+                     int32_t* dev_status, uint64_t wait_limit_ns, int scales_by_tma) {
   using G = Geo<kPair>;
   constexpr int S = G::kStages;
+  constexpr int kWS = kDgrad ? kWStages : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = smem;
-  uint16_t* sY = (uint16_t*)(smem + S * G::kStageBytes);
+  uint8_t* sW = smem + S * G::kStageBytes;        // input gradient only
+  uint8_t* sS = sW + kWS * G::kWBytes;
+  uint16_t* sY = (uint16_t*)(sS + kWS * G::kSBytes);
   Shared* sh = (Shared*)((uint8_t*)sY + kStagingBytes);
   int32_t* s_offs = (int32_t*)((uint8_t*)sh + 256);
+  constexpr int kOffsCache = kDgrad ? kMaxSmemExpertsDgrad : kMaxSmemExperts;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0;  // 0 leads the pair
@@ -182,7 +207,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
   }
   // Tile walks read the expert partition from shared memory when it fits.
   const int32_t* t_offs = offs;
-  if (E <= kMaxSmemExperts) {
+  if (E <= kOffsCache) {
     for (int64_t e = threadIdx.x; e < E; e += blockDim.x) s_offs[e] = offs[e];
     t_offs = s_offs;
   }
@@ -191,6 +216,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
       mbar_init(&sh->full_a[s], kDqWarps * G::kCG);
       mbar_init(&sh->full_b[s], 1);
       mbar_init(&sh->empty[s], 1);
+    }
+    for (int s = 0; s < kWS; ++s) {
+      mbar_init(&sh->wfull[s], 1);
+      mbar_init(&sh->wempty[s], kDqWarps);
     }
     mbar_init(&sh->d_full, 1);
     mbar_init(&sh->d_empty, kEpiWarps * G::kCG);
@@ -202,7 +231,13 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
     tmem_alloc_cg<G::kCG>(&sh->tmem_base, kTmemCols);
     tmem_relinquish_cg<G::kCG>();
   }
-  if (warp == kTmaWarp && lane == 0) prefetch_tmap(&tmap_act);
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tmap(&tmap_act);
+    if constexpr (kDgrad) {
+      prefetch_tmap(&tmap_w);
+      if (scales_by_tma) prefetch_tmap(&tmap_s);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) cluster_sync();  // the peer's barriers exist before any remote arrive
@@ -250,6 +285,38 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
         int abort_local = 0;
         for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
           bwait<kPair>(&sh->full_b[j % S], (j / S) & 1, &abort_local, kDrainLimitNs);
+      }
+    }
+    if constexpr (kDgrad) {
+      if (lane == 1) {
+        // ------------------------- weight producer (input gradient only)
+        // Stage ks of a tile: packed rows n = ks*kBK .. +kBK of expert e,
+        // bytes m0/2 .. +64 (this CTA's 128 features), and their scale
+        // bytes (a 16-byte box holding this CTA's 4).
+        const uint32_t tx = G::kWBytes + (scales_by_tma ? G::kSBytes : 0u);
+        TileWalker walk(t_offs, E, kBN, col_tiles);
+        uint32_t wit = 0;
+        for (int64_t tile = unit; !*abort && walk.seek(tile); tile += units) {
+          const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;
+          const int32_t wy = (int32_t)(walk.expert * N);
+          const int32_t sx = (int32_t)((m0 / 32) & ~(int64_t)15);
+          bool ok = true;
+          for (int ks = 0; ks < nk; ++ks, ++wit) {
+            const int ws = wit % kWS;
+            if (!(ok = bwait<kPair>(&sh->wempty[ws], ((wit / kWS) & 1) ^ 1, abort, wait_limit_ns)))
+              break;
+            mbar_arrive_expect_tx(&sh->wfull[ws], tx);
+            tma_load_2d(smem_addr(sW + ws * G::kWBytes), &tmap_w, (int32_t)(m0 / 2),
+                        wy + ks * kBK, &sh->wfull[ws]);
+            if (scales_by_tma)
+              tma_load_2d(smem_addr(sS + ws * G::kSBytes), &tmap_s, sx, wy + ks * kBK,
+                          &sh->wfull[ws]);
+          }
+          if (!ok) break;
+        }
+        int abort_local = 0;
+        for (uint32_t j = wit > (uint32_t)kWS ? wit - kWS : 0; j < wit; ++j)
+          bwait<kPair>(&sh->wfull[j % kWS], (j / kWS) & 1, &abort_local, kDrainLimitNs);
       }
     }
     __syncwarp();
@@ -302,6 +369,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
     const int h = (warp - kEpiWarps) >> 2;   // which half of the 64-wide stage
     TileWalker walk(t_offs, E, kBN, col_tiles);
     uint32_t it = 0;
+    uint32_t wit = 0;  // weight-slot ring position (input gradient)
     bool ok = true;
     for (int64_t tile = unit; ok && walk.seek(tile); tile += units) {
       const int64_t e = walk.expert;
@@ -367,51 +435,48 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
           }
         }
       } else {
-        // Output features k = m0 + 32q + (0..31) are the TMEM lanes of this
-        // warp; a stage half covers kBK/2 reduction indices n, done in
-        // sub-steps of 32.  Thread t decodes byte (n0 + t/4, k/2 = kq/2 + 8r
-        // + 4b + t%4) for its four rows n0 = base + 8j of a sub-step, then
-        // movmatrix transposes each 8x8 block.
+        // The warp's 32 output features k = m0 + 32q + (0..31) are TMEM
+        // lanes 32q..32q+31, in the order kperm() gives; a stage half
+        // covers kBK/2 reduction indices n, done in sub-steps of 32.  In a
+        // sub-step thread t reads 4 contiguous bytes (word t%4 of the
+        // warp's 16 bytes) of rows n = base + 8j + t/4, j = 0..3, from the
+        // TMA-staged tile.  Byte c of the word (k = 8(t%4) + 2c, +1) goes
+        // to 8x8 block c; movmatrix transposes each block so that a thread
+        // holds bf16 pairs along n, and block c fills TMEM lanes 8c..8c+7.
         constexpr int kSub = kBK / 64;  // sub-steps per stage half
-        const int64_t kq = m0 + 32 * q;
         const int rsub = lane >> 2, csub = lane & 3;
-        const uint8_t* pcol = packed + e * N * (K / 2) + kq / 2;
-        const uint8_t* scol = scales + e * N * (K / 32) + kq / 32;
-        const int ng = nk * kSub;  // sub-steps in this tile
-        uint4 pb[2][4];
-        uint32_t sb[2][4];
-        auto load = [&](int g, uint4* P, uint32_t* Sc) {
-          const int64_t nbase = (int64_t)(g / kSub) * kBK + (kBK / 2) * h + 32 * (g % kSub);
+        const uint8_t* scol = scales + e * N * (K / 32) + (m0 + 32 * q) / 32;
+        const int soff = (int)((m0 / 32) & 15) + q;  // this warp's byte in a scale box row
+        for (int ks = 0; ks < nk && ok; ++ks, ++wit) {
+          const int ws = wit % kWS;
+          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wit / kWS) & 1, abort, wait_limit_ns)))
+            break;
+          const uint8_t* wst = sW + ws * G::kWBytes;
+          const uint8_t* sst = sS + ws * G::kSBytes;
+          const int s = it % S;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int64_t n = nbase + 8 * j + rsub;
-            P[j] = ldg16(pcol + n * (K / 2));
-            Sc[j] = scol[n * (K / 32)];
-          }
-        };
-        load(0, pb[0], sb[0]);
-        if (ng > 1) load(1, pb[1], sb[1]);
-        for (int g0 = 0; g0 < ng && ok; g0 += 2) {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int g = g0 + u;
-            if (g >= ng || !ok) break;
-            const int sub_i = g % kSub;
+          for (int sub_i = 0; sub_i < kSub; ++sub_i) {
             uint32_t v[2][8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float sc = scale_f32(sb[u][j]);
-              const uint32_t w[4] = {pb[u][j].x, pb[u][j].y, pb[u][j].z, pb[u][j].w};
+              const int row = (kBK / 2) * h + 32 * sub_i + 8 * j + rsub;  // n within the stage
+              // 64-byte swizzle: 16-byte chunk q sits at chunk q ^ ((row >> 1) & 3)
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                  wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
+              const uint32_t sb = scales_by_tma
+                                      ? (uint32_t)sst[row * 16 + soff]
+                                      : (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)];
+              const float sc = scale_f32(sb);
 #pragma unroll
-              for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                  const uint32_t byte = (w[2 * r + b] >> (8 * csub)) & 0xFFu;
-                  v[r][2 * j + b] = movmatrix_trans(dequant_pair(byte, sc));
-                }
+              for (int c = 0; c < 4; ++c)
+                v[c >> 1][2 * j + (c & 1)] =
+                    movmatrix_trans(dequant_pair((w >> (8 * c)) & 0xFFu, sc));
             }
-            if (g + 2 < ng) load(g + 2, pb[u], sb[u]);
-            const int s = it % S;
+            if (sub_i == kSub - 1) {
+              // every byte of the slot is in registers: hand it back
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh->wempty[ws]);
+            }
             if (sub_i == 0) {
               if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
                 break;
@@ -421,14 +486,13 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
 #pragma unroll
             for (int r = 0; r < 2; ++r)
               tmem_st_16x128b_x4(tmem + ((uint32_t)(32 * q + 16 * r) << 16) + col, v[r]);
-            if (sub_i == kSub - 1) {
-              tmem_wait_st();
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
-              ++it;
-            }
           }
+          if (!ok) break;
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
+          ++it;
         }
       }
     }
@@ -444,7 +508,8 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act, const uint8_t
       tc_fence_after();
       const int64_t row0 = walk.row0;
       const int64_t rows = walk.row_end - row0 < kBN ? walk.row_end - row0 : kBN;
-      const int col = 32 * warp + lane;  // output feature within this CTA's 128
+      // output feature within this CTA's 128 (TMEM lane 32 warp + lane)
+      const int col = 32 * warp + (kDgrad ? kperm(lane) : lane);
 #pragma unroll 1
       for (int c = 0; c < (int)((rows + 31) / 32); ++c) {
         uint32_t v[32];
@@ -524,6 +589,21 @@ bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed weights viewed as bytes [rows, row_bytes]; boxes of box_cols bytes
+// x box_rows rows, with the given swizzle.
+bool make_byte_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                   int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 template <bool kDgrad, bool kPair>
@@ -532,13 +612,26 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
               cudaStream_t st) {
   using G = Geo<kPair>;
   const int64_t kin = kDgrad ? N : K, nout = kDgrad ? K : N;
-  CUtensorMap map;
+  constexpr uint32_t kSmem = kDgrad ? G::kSmemDgrad : G::kSmem;
+  CUtensorMap map, wmap = {}, smap = {};
   if (!make_act_map(&map, a, T, kin, G::kRowsB)) return MXQ_ERR_CUDA;
+  // The input gradient stages W by TMA; its scales too when their rows
+  // (K/32 bytes) are a whole number of 16-byte units.
+  int scales_by_tma = 0;
+  if constexpr (kDgrad) {
+    if (!make_byte_map(&wmap, packed, E * N, K / 2, 64, G::kBK, CU_TENSOR_MAP_SWIZZLE_64B))
+      return MXQ_ERR_CUDA;
+    if ((K / 32) % 16 == 0 && ((uintptr_t)scales & 15) == 0) {
+      if (!make_byte_map(&smap, scales, E * N, K / 32, 16, G::kBK, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return MXQ_ERR_CUDA;
+      scales_by_tma = 1;
+    }
+  }
   auto kernel = grouped_mm_tc_kernel<kDgrad, kPair>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   });
   if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
   // Upper bound on the tile count: every expert may add one ragged tile.
@@ -548,7 +641,7 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(units * G::kCG), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = G::kSmem;
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -557,9 +650,10 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, map, (const uint8_t*)packed,
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, map, wmap, smap, (const uint8_t*)packed,
                                        (const uint8_t*)scales, offs, T, E, N, K,
-                                       (__nv_bfloat16*)y, dev_status, g_wait_limit_ns.load());
+                                       (__nv_bfloat16*)y, dev_status, g_wait_limit_ns.load(),
+                                       scales_by_tma);
   return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
@@ -576,8 +670,12 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
                       int32_t* dev_status, cudaStream_t st) {
   const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
   const bool pair = nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2;
+  // (the input gradient's weight loads are TMA boxes: 16-byte aligned
+  // packed bytes, row coordinates below 2^31)
+  const bool w_ok = !transpose_w || (((uintptr_t)packed & 15) == 0 && E * N < (int64_t)1 << 31);
   const bool tc = kin % Geo<false>::kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
-                  ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31;
+                  ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31 &&
+                  w_ok;
   if (!tc)
     return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
                                      dev_status, st);
