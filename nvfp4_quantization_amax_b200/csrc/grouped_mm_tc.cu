@@ -453,30 +453,35 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
             break;
           const uint8_t* wst = sW + ws * G::kWBytes;
           const uint8_t* sst = sS + ws * G::kSBytes;
+          // All of the slot's reads first (16 independent shared loads in
+          // flight), then the slot goes back to the producer.
+          uint32_t wd[kSub][4];
+          float sc[kSub][4];
+#pragma unroll
+          for (int sub_i = 0; sub_i < kSub; ++sub_i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int row = (kBK / 2) * h + 32 * sub_i + 8 * j + rsub;  // n within the stage
+              // 64-byte swizzle: 16-byte chunk q sits at chunk q ^ ((row >> 1) & 3)
+              wd[sub_i][j] = *reinterpret_cast<const uint32_t*>(
+                  wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
+              const uint32_t sb = scales_by_tma
+                                      ? (uint32_t)sst[row * 16 + soff]
+                                      : (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)];
+              sc[sub_i][j] = scale_f32(sb);
+            }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->wempty[ws]);
           const int s = it % S;
 #pragma unroll
           for (int sub_i = 0; sub_i < kSub; ++sub_i) {
             uint32_t v[2][8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int row = (kBK / 2) * h + 32 * sub_i + 8 * j + rsub;  // n within the stage
-              // 64-byte swizzle: 16-byte chunk q sits at chunk q ^ ((row >> 1) & 3)
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                  wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
-              const uint32_t sb = scales_by_tma
-                                      ? (uint32_t)sst[row * 16 + soff]
-                                      : (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)];
-              const float sc = scale_f32(sb);
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
               for (int c = 0; c < 4; ++c)
                 v[c >> 1][2 * j + (c & 1)] =
-                    movmatrix_trans(dequant_pair((w >> (8 * c)) & 0xFFu, sc));
-            }
-            if (sub_i == kSub - 1) {
-              // every byte of the slot is in registers: hand it back
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&sh->wempty[ws]);
-            }
+                    movmatrix_trans(dequant_pair((wd[sub_i][j] >> (8 * c)) & 0xFFu, sc[sub_i][j]));
             if (sub_i == 0) {
               if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
                 break;
