@@ -76,6 +76,8 @@ def lib():
         L.orc_quantize_cache_packed.argtypes = [p, i, i64, i64, i, i, p, p]
         L.orc_dequantize_cache_packed.restype = i
         L.orc_dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i, p, i]
+        L.orc_w4a4_grouped_mm.restype = i
+        L.orc_w4a4_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, p, i64, p]
         L.orc_grouped_mm.restype = i
         L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
         _lib = L
@@ -223,6 +225,27 @@ def grouped_mm(a_bits, packed, scales, offs, transpose_w=False, rows=None):
         raise ValueError("oracle grouped_mm: rc=%d" % rc)
     return out
 
+
+
+def w4a4_grouped_mm(x_bits, packed, scales, offs, rows=None):
+    """Exact-sum grouped GEMM with the activations quantized to MXFP4 first:
+    out[i, n] = sum_k deq(mx_quantize(x))[t, k] W_e[n, k], t = rows[i]."""
+    x = _c(x_bits, np.uint16)
+    p = _c(packed, np.uint8)
+    s = _c(scales, np.uint8)
+    o = _c(offs, np.int32)
+    E, N, Kh = p.shape
+    K = 2 * Kh
+    T = x.shape[0]
+    if rows is None:
+        rows = np.arange(T, dtype=np.int64)
+    r = _c(rows, np.int64)
+    out = np.zeros((r.size, N), np.float64)
+    rc = lib().orc_w4a4_grouped_mm(_ptr(x), _ptr(p), _ptr(s), _ptr(o), T, E, N, K, _ptr(r),
+                                   r.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle w4a4_grouped_mm: rc=%d" % rc)
+    return out
 
 
 def nvfp4_global_scale(amax):

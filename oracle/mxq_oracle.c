@@ -641,3 +641,55 @@ int orc_nvfp4_quantize_mse(const void* x, int dtype, int64_t rows, int64_t K, ui
   *global_scale = (float)g;
   return orc_nvfp4_quantize_mse_rows(x, dtype, rows, K, g, packed, block_scales);
 }
+
+/* ------------------------------------------------------------------------ */
+/* W4A4 grouped GEMM: both operands MXFP4 ([MO] "W4A4 NVFP4 on FP4 tensor   */
+/* cores", here with the MX format of [MX]).                                 */
+/* ------------------------------------------------------------------------ */
+
+/* x: bf16 [T, K] activations, quantized row by row with orc_mx_quantize
+   (one E8M0 scale per 32 columns) and dequantized exactly; weights as in
+   orc_grouped_mm.  out[i][n] = sum_k deq(q(x))[t][k] W_e[n][k] for t =
+   rows[i], summed in double in index order (not rounded). */
+int orc_w4a4_grouped_mm(const uint16_t* x, const uint8_t* packed, const uint8_t* scales,
+                        const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
+                        const int64_t* rows, int64_t nrows, double* out) {
+  if (E < 1 || K % 32 != 0 || N < 1 || T < 0) return ORC_EARG;
+  if (orc_check_offs(offs, E, T) != ORC_OK) return ORC_EOFFS;
+  uint8_t* qp = (uint8_t*)malloc((size_t)(K / 2));
+  uint8_t* qs = (uint8_t*)malloc((size_t)(K / 32));
+  double* xa = (double*)malloc((size_t)K * sizeof(double));
+  double* w = (double*)malloc((size_t)(N * K) * sizeof(double));
+  int rc = ORC_OK;
+  if (!qp || !qs || !xa || !w) {
+    rc = ORC_EARG;
+    goto done;
+  }
+  for (int64_t e = 0; e < E; ++e) {
+    int64_t lo = e == 0 ? 0 : offs[e - 1], hi = offs[e];
+    int have = 0;
+    for (int64_t i = 0; i < nrows && !have; ++i) have = rows[i] >= lo && rows[i] < hi;
+    if (!have) continue;
+    const uint8_t* pe = packed + e * N * (K / 2);
+    const uint8_t* se = scales + e * N * (K / 32);
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k) w[n * K + k] = mx_element(pe, se, K, n, k);
+    for (int64_t i = 0; i < nrows; ++i) {
+      int64_t t = rows[i];
+      if (t < lo || t >= hi) continue;
+      orc_mx_quantize(x + t * K, ORC_BF16, 1, K, qp, qs);
+      for (int64_t k = 0; k < K; ++k) xa[k] = mx_element(qp, qs, K, 0, k);
+      for (int64_t n = 0; n < N; ++n) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += xa[k] * w[n * K + k];
+        out[i * N + n] = acc;
+      }
+    }
+  }
+done:
+  free(qp);
+  free(qs);
+  free(xa);
+  free(w);
+  return rc;
+}

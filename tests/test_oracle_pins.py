@@ -767,3 +767,45 @@ def test_mse_moves_codes_both_ways():
     _, s_max, _ = oracle.nvfp4_quantize(bits)
     diff = s_mse.astype(int) - s_max.astype(int)
     assert (diff < 0).any() and (diff > 0).any()
+
+
+# ----------------------------------------------------- W4A4 grouped GEMM
+
+def test_w4a4_matches_numpy_on_quantized_activations():
+    # the activations pass through the (pinned) MXFP4 quantizer; the product
+    # is then an ordinary matmul with the dequantized weights
+    xb, packed, scales, offs = small_moe()
+    qp, qs = oracle.mx_quantize(xb, "bf16")
+    xq = oracle.decode(oracle.mx_dequantize(qp, qs, "f32"), "f32")
+    W = dense_weights(packed, scales)
+    want = np.zeros((xb.shape[0], W.shape[1]))
+    lo = 0
+    for e, hi in enumerate(offs):
+        want[lo:hi] = xq[lo:hi] @ W[e].T
+        lo = hi
+    got = oracle.w4a4_grouped_mm(xb, packed, scales, offs)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_w4a4_differs_from_w4a16_by_the_activation_rounding():
+    # quantizing the activations changes the product: the MXFP4 cast moves
+    # an element by at most 2 scale units (clipping below 8 to 6, or
+    # rounding between 4 and 6) and a unit is at most amax / 4
+    xb, packed, scales, offs = small_moe()
+    y4 = oracle.w4a4_grouped_mm(xb, packed, scales, offs)
+    y16 = oracle.grouped_mm(xb, packed, scales, offs)
+    assert not np.allclose(y4, y16)
+    W = dense_weights(packed, scales)
+    bound = np.abs(oracle.decode(xb, "bf16")).max() / 2 * np.abs(W).sum(axis=2).max()
+    assert np.abs(y4 - y16).max() <= bound
+
+
+def test_w4a4_exact_on_representable_activations():
+    # activations already on the MXFP4 grid are left unchanged by the
+    # quantizer, so W4A4 equals the bf16-activation GEMM exactly
+    xb, packed, scales, offs = small_moe()
+    qp, qs = oracle.mx_quantize(xb, "bf16")
+    xg = oracle.mx_dequantize(qp, qs, "bf16")
+    y4 = oracle.w4a4_grouped_mm(xg, packed, scales, offs)
+    y16 = oracle.grouped_mm(xg, packed, scales, offs)
+    assert np.array_equal(y4, y16)
