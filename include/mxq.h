@@ -174,6 +174,26 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
                      int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                      int32_t* dev_status, void* stream);
 
+/* W4A4 grouped GEMM: MXFP4 activations times MXFP4 expert weights on the
+ * block-scaled tensor cores ([MO] "W4A4 NVFP4 on FP4 tensor cores", with
+ * the MX format of [MX]).
+ *
+ *  x_packed, x_scales  device, the activations as mx_quantize writes them:
+ *           [T, K/2] E2M1 bytes and [T, K/32] E8M0 bytes, rows grouped
+ *           contiguously by expert.
+ *  packed, scales, offs, dev_status  as mxfp4_grouped_mm (forward).
+ *  y        device, bf16 [T, N]: y[t, n] = sum_k xq[t, k] W_e[n, k] with xq
+ *           the dequantized activation; products are exact, the sum is
+ *           accumulated in f32 by the tensor core and rounded once to bf16.
+ *  Every pointer 16-byte aligned.
+ *  Errors: K % 32 != 0, E < 1, N < 1, T < 0 -> MXQ_ERR_SHAPE; null ->
+ *  MXQ_ERR_INVALID_ARG; misaligned -> MXQ_ERR_ALIGNMENT; K % 256 != 0 or
+ *  N % 128 != 0 (shapes this kernel does not tile) -> MXQ_ERR_UNSUPPORTED.
+ *  T == 0: no-op. */
+int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void* packed,
+                          const void* scales, const int32_t* offs, int64_t T, int64_t E, int64_t N,
+                          int64_t K, void* y, int32_t* dev_status, void* stream);
+
 /* Device workspace nvfp4_quantize needs (bytes, 16-byte aligned). */
 #define MXQ_NVFP4_WORKSPACE_BYTES 16
 

@@ -26,4 +26,5 @@ from ._abi import (  # noqa: F401
     quantize_cache_packed,
     set_wait_limit_ns,
     status_string,
+    w4a4_grouped_mm,
 )

@@ -56,6 +56,8 @@ def lib():
         L.quantize_cache_packed.argtypes = [p, i, i64, i64, i, i32, p, p, p]
         L.dequantize_cache_packed.restype = i
         L.dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i32, p, i, p]
+        L.mxfp4_w4a4_grouped_mm.restype = i
+        L.mxfp4_w4a4_grouped_mm.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p, p]
         L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64
         L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
@@ -265,6 +267,38 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
     rc = lib().mxfp4_grouped_mm(_ptr(a), _ptr(packed), _ptr(scales), _ptr(offs), T, E, N, K,
                                 1 if transpose_w else 0, _ptr(out), st, _stream(a.device))
     _check(rc, "mxfp4_grouped_mm")
+    return _to_host(out) if host else out
+
+
+def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=None,
+                    x_scales=None):
+    """W4A4 grouped GEMM: the bf16 activations x [T, K] are quantized to
+    MXFP4 (mx_quantize) and multiplied with the MXFP4 expert weights on the
+    block-scaled tensor cores.  Returns bf16 [T, N] (forward only).
+    x_packed / x_scales: optional preallocated [T, K/2] / [T, K/32] buffers
+    for the quantized activations."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("w4a4_grouped_mm: activations must be bf16")
+    x, host = _to_device(x)
+    packed, _ = _to_device(packed)
+    scales, _ = _to_device(scales)
+    offs, _ = _to_device(offs)
+    x, packed, scales = x.contiguous(), packed.contiguous(), scales.contiguous()
+    offs = offs.to(torch.int32).contiguous()
+    E, N, Kh = packed.shape
+    K = 2 * Kh
+    T = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("w4a4_grouped_mm: x must be [T, %d]" % K)
+    if tuple(scales.shape) != (E, N, K // 32) or offs.numel() != E:
+        raise ValueError("w4a4_grouped_mm: scales [E, N, K/32] and offs [E] expected")
+    xq, xs = mx_quantize(x, x_packed, x_scales)
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    rc = lib().mxfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(packed), _ptr(scales), _ptr(offs),
+                                     T, E, N, K, _ptr(out), st, _stream(x.device))
+    _check(rc, "mxfp4_w4a4_grouped_mm")
     return _to_host(out) if host else out
 
 

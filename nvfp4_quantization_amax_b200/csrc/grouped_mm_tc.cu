@@ -41,6 +41,7 @@
 #include "mxq_grouped.cuh"
 #include "mxq_launch.h"
 #include "sm100_primitives.cuh"
+#include "tmap.h"
 
 namespace mxq {
 
@@ -66,8 +67,8 @@ constexpr int kMmaWarp = 13;
 constexpr int kThreads = 14 * 32;
 constexpr uint32_t kStagingBytes = kBN * kBM * 2;   // 64 KB
 constexpr int kMaxSmemExperts = 4096;               // offs cached in smem up to this E
-constexpr int kMaxSmemExpertsDgrad = 256;           // (the input gradient's smem holds W stages)
-constexpr int kWStages = 3;                         // packed-weight stages of the input gradient
+constexpr int kMaxSmemExpertsW = 256;               // (when smem also holds weight slots)
+constexpr int kWStages = 3;                         // packed-weight slots staged by TMA
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 constexpr uint64_t kAbortSettleNs = 50000ull;
 
@@ -88,14 +89,16 @@ struct Geo {
   static constexpr int kStages = 4;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
-  // Input gradient: the packed weight tile of a stage (kBK rows n x 64
-  // bytes = 128 features k, 64-byte swizzled) and its scale bytes (a
-  // 16-byte box per row) arrive by TMA into kWStages slots.
-  static constexpr uint32_t kWBytes = kBK * 64;
-  static constexpr uint32_t kSBytes = kBK * 16;
-  static constexpr uint32_t kSmemDgrad = 1024 + kStages * kStageBytes +
-                                         kWStages * (kWBytes + kSBytes) + kStagingBytes + 256 +
-                                         4 * kMaxSmemExpertsDgrad;
+  // With weight staging, the packed weight tile of a stage (64 bytes by
+  // 128 rows: the input gradient's kBK rows n x 128 features k, or the
+  // pair forward's 128 rows n x 128 k, 64-byte swizzled) and its scale
+  // bytes (a 16-byte box per row) arrive by TMA into kWStages slots.
+  static constexpr int kWRows = 128;
+  static constexpr uint32_t kWBytes = kWRows * 64;
+  static constexpr uint32_t kSBytes = kWRows * 16;
+  static constexpr uint32_t kSmemW = 1024 + kStages * kStageBytes +
+                                     kWStages * (kWBytes + kSBytes) + kStagingBytes + 256 +
+                                     4 * kMaxSmemExpertsW;
   // Token count of a tile rounded to what the MMA accepts.
   __host__ __device__ static int64_t mma_n(int64_t rows) {
     return kPair ? (rows + 31) & ~31 : (rows + 15) & ~15;
@@ -184,16 +187,19 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
                      int32_t* dev_status, uint64_t wait_limit_ns, int scales_by_tma) {
   using G = Geo<kPair>;
   constexpr int S = G::kStages;
-  constexpr int kWS = kDgrad ? kWStages : 0;
+  // Weight staging by TMA: the input gradient always, the forward in pairs.
+  constexpr bool kWTma = kDgrad || kPair;
+  constexpr int kWS = kWTma ? kWStages : 0;
+  constexpr int kWBoxRows = kDgrad ? G::kBK : kBM;  // rows of a weight / scale box
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = smem;
-  uint8_t* sW = smem + S * G::kStageBytes;        // input gradient only
+  uint8_t* sW = smem + S * G::kStageBytes;        // weight slots (kWTma only)
   uint8_t* sS = sW + kWS * G::kWBytes;
   uint16_t* sY = (uint16_t*)(sS + kWS * G::kSBytes);
   Shared* sh = (Shared*)((uint8_t*)sY + kStagingBytes);
   int32_t* s_offs = (int32_t*)((uint8_t*)sh + 256);
-  constexpr int kOffsCache = kDgrad ? kMaxSmemExpertsDgrad : kMaxSmemExperts;
+  constexpr int kOffsCache = kWTma ? kMaxSmemExpertsW : kMaxSmemExperts;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0;  // 0 leads the pair
@@ -233,7 +239,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
   }
   if (warp == kTmaWarp && lane == 0) {
     prefetch_tmap(&tmap_act);
-    if constexpr (kDgrad) {
+    if constexpr (kWTma) {
       prefetch_tmap(&tmap_w);
       if (scales_by_tma) prefetch_tmap(&tmap_s);
     }
@@ -287,30 +293,39 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           bwait<kPair>(&sh->full_b[j % S], (j / S) & 1, &abort_local, kDrainLimitNs);
       }
     }
-    if constexpr (kDgrad) {
+    if constexpr (kWTma) {
       if (lane == 1) {
-        // ------------------------- weight producer (input gradient only)
-        // Stage ks of a tile: packed rows n = ks*kBK .. +kBK of expert e,
-        // bytes m0/2 .. +64 (this CTA's 128 features), and their scale
-        // bytes (a 16-byte box holding this CTA's 4).
-        const uint32_t tx = G::kWBytes + (scales_by_tma ? G::kSBytes : 0u);
+        // -------------------------------------------- weight producer
+        // Input gradient, stage ks of a tile: packed rows n = ks*kBK ..
+        // +kBK of expert e, bytes m0/2 .. +64 (this CTA's 128 features k).
+        // Forward: rows n = m0 .. +128 (this CTA's features), bytes
+        // ks*kBK/2 .. +64.  Scale bytes: the 16-byte box holding the 4 the
+        // stage needs, on the same rows.
+        const uint32_t tx = kWBoxRows * 64 + (scales_by_tma ? kWBoxRows * 16 : 0);
         TileWalker walk(t_offs, E, kBN, col_tiles);
         uint32_t wit = 0;
         for (int64_t tile = unit; !*abort && walk.seek(tile); tile += units) {
           const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;
           const int32_t wy = (int32_t)(walk.expert * N);
-          const int32_t sx = (int32_t)((m0 / 32) & ~(int64_t)15);
           bool ok = true;
           for (int ks = 0; ks < nk; ++ks, ++wit) {
             const int ws = wit % kWS;
             if (!(ok = bwait<kPair>(&sh->wempty[ws], ((wit / kWS) & 1) ^ 1, abort, wait_limit_ns)))
               break;
+            int32_t wx, sx, y0;
+            if constexpr (kDgrad) {
+              wx = (int32_t)(m0 / 2);
+              sx = (int32_t)((m0 / 32) & ~(int64_t)15);
+              y0 = wy + ks * kBK;
+            } else {
+              wx = ks * (kBK / 2);
+              sx = (ks * (kBK / 32)) & ~15;
+              y0 = wy + (int32_t)m0;
+            }
             mbar_arrive_expect_tx(&sh->wfull[ws], tx);
-            tma_load_2d(smem_addr(sW + ws * G::kWBytes), &tmap_w, (int32_t)(m0 / 2),
-                        wy + ks * kBK, &sh->wfull[ws]);
+            tma_load_2d(smem_addr(sW + ws * G::kWBytes), &tmap_w, wx, y0, &sh->wfull[ws]);
             if (scales_by_tma)
-              tma_load_2d(smem_addr(sS + ws * G::kSBytes), &tmap_s, sx, wy + ks * kBK,
-                          &sh->wfull[ws]);
+              tma_load_2d(smem_addr(sS + ws * G::kSBytes), &tmap_s, sx, y0, &sh->wfull[ws]);
           }
           if (!ok) break;
         }
@@ -374,7 +389,59 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
     for (int64_t tile = unit; ok && walk.seek(tile); tile += units) {
       const int64_t e = walk.expert;
       const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;  // this CTA's features
-      if constexpr (!kDgrad) {
+      if constexpr (!kDgrad && kWTma) {
+        // Thread = weight row n = m0 + 32q + lane (slot row 32q + lane);
+        // stage half h: k = ks*kBK + 64h .. +64, i.e. 16-byte chunks 2h and
+        // 2h+1 of the 64-byte slot row (64-byte swizzle), and scale bytes
+        // 4ks + 2h, +1 of the row's 16-byte scale box.
+        static_assert(kBK == 128, "weight staging of the forward assumes 128-deep stages");
+        const int row = 32 * q + lane;
+        const int swz = (row >> 1) & 3;
+        const uint8_t* srow = scales + (e * N + m0 + row) * (K / 32) + 2 * h;
+        for (int ks = 0; ks < nk && ok; ++ks, ++wit) {
+          const int ws = wit % kWS;
+          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wit / kWS) & 1, abort, wait_limit_ns)))
+            break;
+          const uint8_t* wrow = sW + ws * G::kWBytes + row * 64;
+          uint4 d[2];
+          uint32_t sb[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            d[c] = *reinterpret_cast<const uint4*>(wrow + 16 * ((2 * h + c) ^ swz));
+          if (scales_by_tma) {
+            const uint8_t* sp = sS + ws * G::kSBytes + row * 16 + ((4 * ks) & 15) + 2 * h;
+            sb[0] = sp[0];
+            sb[1] = sp[1];
+          } else {
+            sb[0] = srow[4 * ks];
+            sb[1] = srow[4 * ks + 1];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->wempty[ws]);
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t w[4] = {d[c].x, d[c].y, d[c].z, d[c].w};
+            const float sc = scale_f32(sb[c]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
+          }
+          const int s = it % S;
+          if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
+            break;
+          tc_fence_after();
+          const uint32_t col = kACol + G::kACols * s + 32 * h;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + col + 16 * c, v + 16 * c);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
+          ++it;
+        }
+      } else if constexpr (!kDgrad) {
         // Thread = weight row n; kBK/2 consecutive k (kBK/4 bytes, one or
         // two 16-byte loads, one scale per 32 k) per stage half.
         constexpr int kV = kBK / 64;  // 16-byte loads per thread per stage
@@ -561,52 +628,19 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
 
 // ------------------------------------------------------------------ host
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  });
-  return fn;
-}
-
 // Row-major bf16 [rows, cols] activations, boxes of 64 columns x box_rows
 // rows, 128-byte swizzle; rows past the end read as zero.
 bool make_act_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {kBox, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rows, cols, cols * 2, kBox,
+                      box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Packed weights viewed as bytes [rows, row_bytes]; boxes of box_cols bytes
 // x box_rows rows, with the given swizzle.
 bool make_byte_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
                    int box_cols, int box_rows, CUtensorMapSwizzle swz) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rows, row_bytes, row_bytes,
+                      box_cols, box_rows, swz);
 }
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
@@ -617,17 +651,19 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
               cudaStream_t st) {
   using G = Geo<kPair>;
   const int64_t kin = kDgrad ? N : K, nout = kDgrad ? K : N;
-  constexpr uint32_t kSmem = kDgrad ? G::kSmemDgrad : G::kSmem;
+  constexpr bool kWTma = kDgrad || kPair;
+  constexpr uint32_t kSmem = kWTma ? G::kSmemW : G::kSmem;
+  constexpr int kWBoxRows = kDgrad ? G::kBK : kBM;
   CUtensorMap map, wmap = {}, smap = {};
   if (!make_act_map(&map, a, T, kin, G::kRowsB)) return MXQ_ERR_CUDA;
-  // The input gradient stages W by TMA; its scales too when their rows
-  // (K/32 bytes) are a whole number of 16-byte units.
+  // The input gradient and the pair forward stage W by TMA; the scales
+  // too when their rows (K/32 bytes) are a whole number of 16-byte units.
   int scales_by_tma = 0;
-  if constexpr (kDgrad) {
-    if (!make_byte_map(&wmap, packed, E * N, K / 2, 64, G::kBK, CU_TENSOR_MAP_SWIZZLE_64B))
+  if constexpr (kWTma) {
+    if (!make_byte_map(&wmap, packed, E * N, K / 2, 64, kWBoxRows, CU_TENSOR_MAP_SWIZZLE_64B))
       return MXQ_ERR_CUDA;
     if ((K / 32) % 16 == 0 && ((uintptr_t)scales & 15) == 0) {
-      if (!make_byte_map(&smap, scales, E * N, K / 32, 16, G::kBK, CU_TENSOR_MAP_SWIZZLE_NONE))
+      if (!make_byte_map(&smap, scales, E * N, K / 32, 16, kWBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE))
         return MXQ_ERR_CUDA;
       scales_by_tma = 1;
     }
@@ -664,6 +700,8 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
 
 }  // namespace
 
+uint64_t get_wait_limit_ns() { return g_wait_limit_ns.load(); }
+
 uint64_t set_wait_limit_ns(uint64_t ns) {
   const uint64_t prev = g_wait_limit_ns;
   g_wait_limit_ns = ns;
@@ -674,13 +712,14 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                       int32_t* dev_status, cudaStream_t st) {
   const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
-  const bool pair = nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2;
-  // (the input gradient's weight loads are TMA boxes: 16-byte aligned
-  // packed bytes, row coordinates below 2^31)
-  const bool w_ok = !transpose_w || (((uintptr_t)packed & 15) == 0 && E * N < (int64_t)1 << 31);
+  // Weight loads by TMA (the input gradient, and the forward in pairs) need
+  // 16-byte aligned packed bytes and row coordinates below 2^31.
+  const bool w_ok = ((uintptr_t)packed & 15) == 0 && E * N < (int64_t)1 << 31;
+  const bool pair =
+      nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2 && w_ok;
   const bool tc = kin % Geo<false>::kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
                   ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31 &&
-                  w_ok;
+                  (w_ok || !transpose_w);
   if (!tc)
     return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
                                      dev_status, st);

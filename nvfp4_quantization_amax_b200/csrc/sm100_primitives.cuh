@@ -311,6 +311,54 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory descriptor of a non-swizzled K-major operand made of 8-row
+// x 16-byte core matrices stacked every sbo bytes (e.g. the 32 rows x 16
+// bytes that tcgen05.cp 32x128b reads).
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address
+  d |= (uint64_t)(16u >> 4) << 16;                    // leading byte offset (one core matrix)
+  d |= (uint64_t)((sbo & 0x3FFFFu) >> 4) << 32;       // stride byte offset
+  d |= (uint64_t)1 << 46;                             // descriptor version (sm_100)
+  return d;                                           // layout type 0: no swizzle
+}
+
+// Copy 32 rows x 128 bits from shared memory (descriptor) into TMEM lanes
+// 0..31 at taddr's columns, replicated into all four lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], both E2M1 (two per byte, K-major), with
+// one E8M0 scale per 32 K per row of A and of B read from TMEM (K = 64 per
+// instruction: two scales per row, selected by the descriptor's ids).
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf4 (block-scaled): E2M1 A and B
+// (K-major), E8M0 scales, f32 D; the two scale ids select the byte of the
+// TMEM scale word where this instruction's scales start.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t a_sf_id,
+                                                  uint32_t b_sf_id) {
+  return (b_sf_id << 4)              // B scale-factor id
+         | (1u << 7)                 // A format E2M1
+         | (1u << 10)                // B format E2M1
+         | ((uint32_t)(N >> 3) << 17)
+         | (1u << 23)                // scale format E8M0
+         | ((uint32_t)(M >> 4) << 24)
+         | (a_sf_id << 29);          // A scale-factor id
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B (K-major), f32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                   // D format f32

@@ -1,0 +1,361 @@
+// W4A4 grouped GEMM on the block-scaled tensor cores (sm_100a): both the
+// expert weights and the activations are MXFP4 (E2M1 codes, two per byte,
+// one E8M0 scale per 32 K), multiplied by tcgen05.mma kind::mxf4 with the
+// scales applied inside the tensor core ("NVIDIA Model Optimizer: from
+// mtq.quantize to a 4.95-bit DeepSeek-R1", section on W4A4 NVFP4 on FP4
+// tensor cores; here with the MX format of
+// "nemo_automodel.components.quantization.mxfp4").
+//
+//   y[t, n] = sum_k xq[t, k] W_e[n, k]   for t in expert e's rows
+//
+// xq is the activation after mx_quantize (its packed bytes and scales are
+// the inputs), so every product of codes is exact and the tensor core only
+// rounds the f32 accumulation; y is rounded once to bf16.
+//
+// Mapping (persistent, one CTA per SM, seven warps):
+//   D[m, j] (f32, TMEM) += A[m, k] (weights, smem) * B[j, k] (tokens, smem)
+// with m one of the CTA's 128 weight rows (TMEM lanes), j one of up to 256
+// tokens of the expert and k the reduction index, 256 per pipeline stage
+// (128 bytes of codes per row: one 128-byte-swizzled TMA row).
+//   * warp 4 (one lane) TMA-loads both code tiles of a stage;
+//   * warp 5 gathers the stage's scale bytes (8 per row: 128 weight rows
+//     and 256 token rows) from the row-major [rows, K/32] scale arrays and
+//     writes them into the tensor core's scale layout in shared memory:
+//     blocks of 128 rows x 4 scales, row r at byte 16 (r % 32) + 4 (r / 32)
+//     + the scale's index;
+//   * warp 6 (one lane) copies those blocks into TMEM (tcgen05.cp, 32 lanes
+//     x 128 bits, replicated to the four lane quarters) and issues four
+//     K=64 MMAs per stage, each selecting its pair of scales by byte id;
+//   * warps 0-3 drain D, round to bf16, stage the tile in shared memory and
+//     store the expert's rows.
+// Every mbarrier wait is bounded: on a time-out the CTA stops all roles,
+// drains what it issued, frees TMEM and reports MXQ_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "mxq.h"
+#include "mxq_device.cuh"
+#include "mxq_grouped.cuh"
+#include "mxq_launch.h"
+#include "sm100_primitives.cuh"
+#include "tmap.h"
+
+namespace mxq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kM = 128;                 // weight rows per tile (TMEM lanes)
+constexpr int kN = 256;                 // tokens per tile (MMA N)
+constexpr int kKB = 128;                // bytes of codes per row per stage (256 K)
+constexpr int kStages = 3;
+constexpr uint32_t kABytes = kM * kKB;            // 16 KB
+constexpr uint32_t kBBytes = kN * kKB;            // 32 KB
+constexpr uint32_t kSfBlock = 512;                // 128 rows x 4 scales
+constexpr uint32_t kSfaBytes = 2 * kSfBlock;      // 128 rows x 8 scales
+constexpr uint32_t kSfbBytes = 4 * kSfBlock;      // 256 rows x 8 scales
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr uint32_t kStagingBytes = kN * kM * 2;   // 64 KB of bf16 output
+constexpr int kMaxSmemExperts = 256;
+constexpr uint32_t kSmem = 1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
+constexpr int kTmemCols = 512;
+constexpr int kDCol = 0;                // accumulator: columns [0, 256)
+constexpr int kSfaCol = 256;            // A scales: 2 blocks x 4 columns
+constexpr int kSfbCol = 264;            // B scales: 4 blocks x 4 columns
+constexpr int kEpiWarps = 4;
+constexpr int kTmaWarp = 4;
+constexpr int kSfWarp = 5;
+constexpr int kMmaWarp = 6;
+constexpr int kThreads = 7 * 32;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+static_assert(kSmem <= 232448, "shared memory per CTA");
+
+struct Shared {
+  uint64_t full[kStages];   // codes (TMA bytes) and scales (warp 5) of a stage are in smem
+  uint64_t empty[kStages];  // the stage's MMAs (and scale copies) completed
+  uint64_t d_full, d_empty, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ int64_t mma_n(int64_t rows) { return (rows + 15) & ~15; }
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Byte offset of (row r, scale s) inside a 128-row block of the tensor
+// core's scale layout (s in 0..3).
+__device__ __forceinline__ uint32_t sf_offset(int r) { return 16 * (r & 31) + 4 * ((r >> 5) & 3); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               const uint8_t* __restrict__ x_scales, const uint8_t* __restrict__ w_scales,
+               const int32_t* __restrict__ offs, int64_t T, int64_t E, int64_t N, int64_t K,
+               __nv_bfloat16* __restrict__ y, int32_t* dev_status, uint64_t wait_limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint16_t* sY = (uint16_t*)(smem + kStages * kStageBytes);
+  Shared* sh = (Shared*)((uint8_t*)sY + kStagingBytes);
+  int32_t* s_offs = (int32_t*)((uint8_t*)sh + 256);
+  auto sA = [&](int s) { return smem + s * kStageBytes; };
+  auto sB = [&](int s) { return smem + s * kStageBytes + kABytes; };
+  auto sSfa = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes; };
+  auto sSfb = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes + kSfaBytes; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!offs_valid(offs, E, T)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && dev_status) *dev_status = MXQ_ERR_BAD_OFFS;
+    return;
+  }
+  const int32_t* t_offs = offs;
+  if (E <= kMaxSmemExperts) {
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) s_offs[e] = offs[e];
+    t_offs = s_offs;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->full[s], 2);  // TMA expect_tx arrive + scale warp arrive
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->d_full, 1);
+    mbar_init(&sh->d_empty, kEpiWarps);
+    mbar_init(&sh->drain, 1);
+    sh->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sh->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = sh->tmem_base;
+  volatile int* abort = &sh->abort;
+  const int nk = (int)(K / 256);
+  const int64_t col_tiles = N / kM;
+  const int64_t srow = K / 32;  // scale bytes per row
+
+  if (warp == kTmaWarp) {
+    // --------------------------------------------------- TMA producer
+    if (lane == 0) {
+      TileWalker walk(t_offs, E, kN, col_tiles);
+      uint32_t it = 0;
+      for (int64_t tile = blockIdx.x; !*abort && walk.seek(tile); tile += gridDim.x) {
+        const int32_t wy = (int32_t)(walk.expert * N + walk.col_tile * kM);
+        const int32_t xy = (int32_t)walk.row0;
+        bool ok = true;
+        for (int ks = 0; ks < nk; ++ks, ++it) {
+          const int s = it % kStages;
+          if (!(ok = mbar_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
+            break;
+          mbar_arrive_expect_tx(&sh->full[s], kABytes + kBBytes);
+          tma_load_2d(smem_addr(sA(s)), &tmap_w, ks * kKB, wy, &sh->full[s]);
+          tma_load_2d(smem_addr(sB(s)), &tmap_x, ks * kKB, xy, &sh->full[s]);
+        }
+        if (!ok) break;
+      }
+      int abort_local = 0;
+      for (uint32_t j = it > (uint32_t)kStages ? it - kStages : 0; j < it; ++j)
+        mbar_wait(&sh->full[j % kStages], (j / kStages) & 1, &abort_local, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == kSfWarp) {
+    // ------------------------------------------- scale-factor producer
+    // Stage ks needs scales 8ks .. 8ks+7 of every row: weight rows n0 + m
+    // (m = lane + 32i) and token rows row0 + r (r = lane + 32i, zero past
+    // the expert's rows).  Scales 0-3 go to block 0, 4-7 to block 1 (of
+    // each 128-row group).
+    TileWalker walk(t_offs, E, kN, col_tiles);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x) {
+      const int64_t rows = walk.row_end - walk.row0 < kN ? walk.row_end - walk.row0 : kN;
+      const uint8_t* wsc = w_scales + (walk.expert * N + walk.col_tile * kM) * srow;
+      const uint8_t* xsc = x_scales + walk.row0 * srow;
+      for (int ks = 0; ks < nk && ok; ++ks, ++it) {
+        const int s = it % kStages;
+        // independent loads first, then the slot wait, then the stores
+        uint2 wv[4], xv[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          wv[i] = __ldg(reinterpret_cast<const uint2*>(wsc + (lane + 32 * i) * srow + 8 * ks));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = lane + 32 * i;
+          xv[i] = r < rows ? __ldg(reinterpret_cast<const uint2*>(xsc + r * srow + 8 * ks))
+                           : make_uint2(0u, 0u);
+        }
+        if (!(ok = warp_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
+          break;
+        uint8_t* fa = sSfa(s);
+        uint8_t* fb = sSfb(s);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t o = sf_offset(lane + 32 * i);
+          *reinterpret_cast<uint32_t*>(fa + o) = wv[i].x;
+          *reinterpret_cast<uint32_t*>(fa + kSfBlock + o) = wv[i].y;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = lane + 32 * i;
+          const uint32_t o = sf_offset(r);
+          const int g = r >> 7;  // 128-row group
+          *reinterpret_cast<uint32_t*>(fb + g * kSfBlock + o) = xv[i].x;
+          *reinterpret_cast<uint32_t*>(fb + (2 + g) * kSfBlock + o) = xv[i].y;
+        }
+        fence_proxy_async_smem();  // visible to tcgen05.cp
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->full[s]);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      TileWalker walk(t_offs, E, kN, col_tiles);
+      uint32_t it = 0, lt = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x, ++lt) {
+        if (!(ok = mbar_wait(&sh->d_empty, (lt & 1) ^ 1, abort, wait_limit_ns))) break;
+        tc_fence_after();
+        const int64_t rows = walk.row_end - walk.row0 < kN ? walk.row_end - walk.row0 : kN;
+        const int n = (int)mma_n(rows);
+        for (int ks = 0; ks < nk; ++ks, ++it) {
+          const int s = it % kStages;
+          if (!(ok = mbar_wait(&sh->full[s], (it / kStages) & 1, abort, wait_limit_ns))) break;
+          tc_fence_after();
+          // scales of the stage into TMEM (A: blocks 0,1; B: (group, block)
+          // pairs (0,0) (1,0) (0,1) (1,1), 8 columns per block index)
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * b,
+                                   smem_desc_noswz(smem_addr(sSfa(s) + b * kSfBlock), 128));
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4 * b,
+                                   smem_desc_noswz(smem_addr(sSfb(s) + b * kSfBlock), 128));
+          const uint64_t adesc = smem_desc_sw128(smem_addr(sA(s)));
+          const uint64_t bdesc = smem_desc_sw128(smem_addr(sB(s)));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // K=64 step kk: 32 bytes into the 128-byte swizzled rows; its
+            // scales are 2kk, 2kk+1: block kk/2, byte 2(kk%2)
+            const uint32_t id = 2u * (kk & 1);
+            const uint32_t blk = kk >> 1;
+            const uint32_t sfa = (tmem + kSfaCol + 4 * blk) | (id << 30);
+            const uint32_t sfb = (tmem + kSfbCol + 8 * blk) | (id << 30);
+            mma_mxf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc_mxf4(kM, n, id, id),
+                        sfa, sfb, (ks | kk) != 0);
+          }
+          mma_commit(&sh->empty[s]);
+        }
+        if (ok) mma_commit(&sh->d_full);
+      }
+      mma_commit(&sh->drain);
+      int abort_local = 0;
+      mbar_wait(&sh->drain, 0, &abort_local, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- epilogue
+    TileWalker walk(t_offs, E, kN, col_tiles);
+    uint32_t lt = 0;
+    for (int64_t tile = blockIdx.x; walk.seek(tile); tile += gridDim.x, ++lt) {
+      if (epi_any(*abort != 0)) break;
+      const bool ok = mbar_wait(&sh->d_full, lt & 1, abort, wait_limit_ns);
+      if (epi_any(!ok)) break;
+      tc_fence_after();
+      const int64_t row0 = walk.row0;
+      const int64_t rows = walk.row_end - row0 < kN ? walk.row_end - row0 : kN;
+      const int col = 32 * warp + lane;  // output feature within the tile's 128
+#pragma unroll 1
+      for (int c = 0; c < (int)((rows + 31) / 32); ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+          sY[(32 * c + j) * kM + col] = (uint16_t)(pr & 0xFFFFu);
+          sY[(32 * c + j + 1) * kM + col] = (uint16_t)(pr >> 16);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->d_empty);
+      epi_bar();  // the whole tile is staged
+      __nv_bfloat16* yt = y + row0 * N + walk.col_tile * kM;
+      for (int r = 2 * warp + (lane >> 4); r < rows; r += 2 * kEpiWarps) {
+        const uint4 val = *reinterpret_cast<const uint4*>(sY + r * kM + 8 * (lane & 15));
+        *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort && dev_status) atomicExch(dev_status, MXQ_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+int launch_w4a4_grouped_mm(const void* xq, const void* xs, const void* packed, const void* scales,
+                           const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
+                           void* y, int32_t* dev_status, uint64_t wait_limit_ns, cudaStream_t st) {
+  CUtensorMap xmap, wmap;
+  if (!make_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, T, K / 2, K / 2, kKB, kN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, E * N, K / 2, K / 2, kKB, kM,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return MXQ_ERR_CUDA;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(w4a4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kSmem);
+  });
+  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
+  const int64_t sms = num_sms();
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  w4a4_tc_kernel<<<grid, kThreads, kSmem, st>>>(xmap, wmap, (const uint8_t*)xs,
+                                                (const uint8_t*)scales, offs, T, E, N, K,
+                                                (__nv_bfloat16*)y, dev_status, wait_limit_ns);
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+}  // namespace mxq

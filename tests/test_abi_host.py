@@ -171,3 +171,14 @@ def test_nvfp4_mse_validation(L):
     with pytest.raises(ValueError):
         import torch
         mxq.nvfp4_quantize(torch.zeros(2, 16, dtype=torch.bfloat16), rule="least")
+
+
+def test_w4a4_validation(L):
+    f = L.mxfp4_w4a4_grouped_mm
+    assert f(A1, A1, A2, A2, A2, 8, 0, 128, 256, A1, NULL, NULL) == ESHAPE  # E < 1
+    assert f(A1, A1, A2, A2, A2, 8, 2, 128, 48, A1, NULL, NULL) == ESHAPE  # K % 32
+    assert f(A1, A1, A2, A2, NULL, 8, 2, 128, 256, A1, NULL, NULL) == EARG  # offs
+    assert f(A1, A1, A2, A2, A2, 8, 2, 128, 96, A1, NULL, NULL) == EUNSUP  # K % 256
+    assert f(A1, A1, A2, A2, A2, 8, 2, 64, 256, A1, NULL, NULL) == EUNSUP  # N % 128
+    assert f(BAD, A1, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
+    assert f(A1, A1, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK  # T == 0

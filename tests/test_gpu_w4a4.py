@@ -1,0 +1,110 @@
+"""GPU parity of the W4A4 grouped GEMM (MXFP4 activations x MXFP4 weights
+on the block-scaled tensor cores) against the oracle, through the C ABI.
+
+The oracle quantizes the activations with its own MXFP4 quantizer and sums
+exactly in double; every product of codes is exact on the tensor core, so
+only the f32 accumulation and the final bf16 rounding differ.  Bar:
+max |y - ref| / max(|ref|, 1e-2 rms(ref)) <= 1e-2, as for the W4A16 GEMM.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_quantization_amax_b200 as mxq
+import oracle
+import synthetic as gen
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+TOL = 1e-2
+
+
+def bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def error(y, ref):
+    y = np.asarray(y, np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    return np.max(np.abs(y - ref) / np.maximum(np.abs(ref), 1e-2 * rms))
+
+
+def case(counts, N, K, seed=31, scale_lo=116, scale_hi=124):
+    E = len(counts)
+    offs = torch.tensor(np.cumsum(counts), dtype=torch.int32)
+    T = int(offs[-1])
+    packed, scales = gen.random_packed(E, N, K, scale_lo, scale_hi, workload=seed)
+    x = gen.normal_bf16(gen.seed_for(seed, 3), (T, K))
+    return x, packed, scales, offs
+
+
+def check(counts, N, K, rows=None, seed=31):
+    x, packed, scales, offs = case(counts, N, K, seed)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = mxq.w4a4_grouped_mm(x.to(DEV), packed.to(DEV), scales.to(DEV), offs.to(DEV),
+                            status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    T = x.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    ref = oracle.w4a4_grouped_mm(bits(x), packed.numpy(), scales.numpy(), offs.numpy(), rows)
+    yv = oracle.decode(bits(y)[rows], "bf16")
+    err = error(yv, ref)
+    assert err <= TOL, err
+    return y
+
+
+def test_w4a4_small_ragged():
+    check([200, 0, 37, 275], 256, 512)
+
+
+def test_w4a4_many_small_experts_and_one_tile_shapes():
+    check([int(c) for c in np.random.RandomState(5).randint(0, 41, size=40)], 128, 256)
+    check([1], 128, 256)
+    check([300], 384, 768)
+
+
+def test_w4a4_full_size_sampled():
+    # the benchmark GEMM: T=32768, E=32, N=2048, K=7168, multinomial counts
+    T, E, N, K = 32768, 32, 2048, 7168
+    counts = gen.expert_counts(T, E).numpy()
+    offs = torch.tensor(np.cumsum(counts), dtype=torch.int32)
+    W = gen.expert_weights(E, N, K, device=DEV, workload=5)
+    P, S = mxq.mx_quantize(W)
+    del W
+    x = gen.normal_bf16(gen.seed_for(5, 3), (T, K), device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = mxq.w4a4_grouped_mm(x, P, S, offs.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = np.array([0, 1, 255, 256, int(offs[0]) - 1, int(offs[0]), 12345, 20000, T - 1])
+    ref = oracle.w4a4_grouped_mm(bits(x), P.cpu().numpy(), S.cpu().numpy(), offs.numpy(), rows)
+    assert error(oracle.decode(bits(y)[rows], "bf16"), ref) <= TOL
+
+
+def test_w4a4_equals_w4a16_on_grid_activations():
+    # activations already on the MXFP4 grid: both GEMMs multiply the same
+    # numbers, so they agree within f32 accumulation order
+    x, packed, scales, offs = case([130, 126], 256, 512, seed=33)
+    xp, xs = mxq.mx_quantize(x.to(DEV))
+    xg = mxq.mx_dequantize(xp, xs)
+    args = (packed.to(DEV), scales.to(DEV), offs.to(DEV))
+    y4 = mxq.w4a4_grouped_mm(xg, *args).float()
+    y16 = mxq.mxfp4_grouped_mm(xg, *args).float()
+    rel = ((y4 - y16).abs().max() / y16.abs().max()).item()
+    assert rel <= 1e-2, rel
+
+
+def test_w4a4_bad_offs_and_unsupported_shapes():
+    x, packed, scales, offs = case([64, 64], 128, 256)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    bad = torch.tensor([100, 64], dtype=torch.int32, device=DEV)
+    y = torch.full((128, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    mxq.w4a4_grouped_mm(x.to(DEV), packed.to(DEV), scales.to(DEV), bad, out=y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == -6 and bool((y == 7.0).all())
+    x2, p2, s2, o2 = case([64], 128, 96)  # K % 256 != 0
+    with pytest.raises(mxq.MxqError) as ei:
+        mxq.w4a4_grouped_mm(x2.to(DEV), p2.to(DEV), s2.to(DEV), o2.to(DEV))
+    assert ei.value.status == -4
