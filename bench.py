@@ -225,6 +225,10 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
         calls["cache_unpack_" + f] = (
             lambda i=i, f=f, b=b, c=codes, s=sc: mxq.dequantize_cache_packed(
                 c, s, f, b, torch.bfloat16, step.kv_out[i]))
+    # W4A4: the benchmark GEMM with MXFP4 activations (quantized inside the call)
+    xq, xs = mxq.mx_quantize(step.x)
+    calls["w4a4_grouped_mm"] = lambda: mxq.w4a4_grouped_mm(step.x, step.P5, step.S5, step.offs,
+                                                           step.y, step.status, xq, xs)
     out = {}
     for name, fn in calls.items():
         for _ in range(2):
@@ -415,6 +419,7 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         nb = next_row_bytes()
         w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
         rows = {}
+        w4 = next_ms.pop("w4a4_grouped_mm", None)
         for n, ms in next_ms.items():
             gbs = nb[n] / (ms * 1e-3) / 1e9
             rows[n] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
@@ -425,6 +430,14 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         rows["nvfp4_quantize_mse"]["bound"] = "alu"
         rows["nvfp4_quantize_mse"]["g_candidates_per_s"] = round(
             126 * w / (next_ms["nvfp4_quantize_mse"] * 1e-3) / 1e9, 1)
+        if w4 is not None:
+            # fp4 peak: the measured bf16 burst x the nominal fp4 / bf16 ratio (9 / 2.25)
+            tf = gemm_flops() / (w4 * 1e-3) / 1e12
+            rows["w4a4_grouped_mm"] = {
+                "ms": round(w4, 4), "tflops": round(tf, 1),
+                "frac_of_fp4_peak": round(tf / (4.0 * peaks["bf16_tflops"]), 4),
+                "includes": "mx_quantize of the activations + the block-scaled GEMM",
+                "workload": "x bf16 [32768,7168], W MXFP4 [32,2048,7168], multinomial counts"}
         line["next_rows"] = rows
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)

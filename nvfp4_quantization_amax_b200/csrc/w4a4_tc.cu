@@ -195,48 +195,74 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     // Stage ks needs scales 8ks .. 8ks+7 of every row: weight rows n0 + m
     // (m = lane + 32i) and token rows row0 + r (r = lane + 32i, zero past
     // the expert's rows).  Scales 0-3 go to block 0, 4-7 to block 1 (of
-    // each 128-row group).
+    // each 128-row group).  The global loads run two stages ahead of the
+    // stores (a cursor of its own walks the same (tile, stage) sequence),
+    // so their latency overlaps the tensor core's work.
+    TileWalker pwalk(t_offs, E, kN, col_tiles);
+    int64_t ptile = blockIdx.x;
+    bool phave = pwalk.seek(ptile);
+    int pks = 0;
+    auto issue = [&](uint2 (&wv)[4], uint2 (&xv)[8]) {
+      if (!phave) return;
+      const int64_t rows = pwalk.row_end - pwalk.row0 < kN ? pwalk.row_end - pwalk.row0 : kN;
+      const uint8_t* wsc = w_scales + (pwalk.expert * N + pwalk.col_tile * kM) * srow + 8 * pks;
+      const uint8_t* xsc = x_scales + pwalk.row0 * srow + 8 * pks;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        wv[i] = __ldg(reinterpret_cast<const uint2*>(wsc + (lane + 32 * i) * srow));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = lane + 32 * i;
+        xv[i] = r < rows ? __ldg(reinterpret_cast<const uint2*>(xsc + r * srow))
+                         : make_uint2(0u, 0u);
+      }
+      if (++pks == nk) {
+        pks = 0;
+        ptile += gridDim.x;
+        phave = pwalk.seek(ptile);
+      }
+    };
+    auto store = [&](int s, const uint2 (&wv)[4], const uint2 (&xv)[8]) {
+      uint8_t* fa = sSfa(s);
+      uint8_t* fb = sSfb(s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t o = sf_offset(lane + 32 * i);
+        *reinterpret_cast<uint32_t*>(fa + o) = wv[i].x;
+        *reinterpret_cast<uint32_t*>(fa + kSfBlock + o) = wv[i].y;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = lane + 32 * i;
+        const uint32_t o = sf_offset(r);
+        const int g = r >> 7;  // 128-row group
+        *reinterpret_cast<uint32_t*>(fb + g * kSfBlock + o) = xv[i].x;
+        *reinterpret_cast<uint32_t*>(fb + (2 + g) * kSfBlock + o) = xv[i].y;
+      }
+      fence_proxy_async_smem();  // visible to tcgen05.cp
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->full[s]);
+    };
+    uint2 wa[4], xa[8], wb[4], xb[8];
+    issue(wa, xa);
+    issue(wb, xb);
     TileWalker walk(t_offs, E, kN, col_tiles);
     uint32_t it = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x) {
-      const int64_t rows = walk.row_end - walk.row0 < kN ? walk.row_end - walk.row0 : kN;
-      const uint8_t* wsc = w_scales + (walk.expert * N + walk.col_tile * kM) * srow;
-      const uint8_t* xsc = x_scales + walk.row0 * srow;
       for (int ks = 0; ks < nk && ok; ++ks, ++it) {
         const int s = it % kStages;
-        // independent loads first, then the slot wait, then the stores
-        uint2 wv[4], xv[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          wv[i] = __ldg(reinterpret_cast<const uint2*>(wsc + (lane + 32 * i) * srow + 8 * ks));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = lane + 32 * i;
-          xv[i] = r < rows ? __ldg(reinterpret_cast<const uint2*>(xsc + r * srow + 8 * ks))
-                           : make_uint2(0u, 0u);
-        }
         if (!(ok = warp_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
           break;
-        uint8_t* fa = sSfa(s);
-        uint8_t* fb = sSfb(s);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t o = sf_offset(lane + 32 * i);
-          *reinterpret_cast<uint32_t*>(fa + o) = wv[i].x;
-          *reinterpret_cast<uint32_t*>(fa + kSfBlock + o) = wv[i].y;
+        // item `it` was loaded into buffer it % 2; refill that buffer with
+        // item it + 2
+        if ((it & 1) == 0) {
+          store(s, wa, xa);
+          issue(wa, xa);
+        } else {
+          store(s, wb, xb);
+          issue(wb, xb);
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = lane + 32 * i;
-          const uint32_t o = sf_offset(r);
-          const int g = r >> 7;  // 128-row group
-          *reinterpret_cast<uint32_t*>(fb + g * kSfBlock + o) = xv[i].x;
-          *reinterpret_cast<uint32_t*>(fb + (2 + g) * kSfBlock + o) = xv[i].y;
-        }
-        fence_proxy_async_smem();  // visible to tcgen05.cp
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->full[s]);
       }
     }
   } else if (warp == kMmaWarp) {
