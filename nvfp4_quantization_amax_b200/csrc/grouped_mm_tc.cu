@@ -219,13 +219,15 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&sh->full_a[s], kDqWarps * G::kCG);
+      // with weight staging each stage is decoded by the 4 warps of one
+      // stage-parity group, otherwise by all 8 (two halves of the stage)
+      mbar_init(&sh->full_a[s], (kWTma ? kDqWarps / 2 : kDqWarps) * G::kCG);
       mbar_init(&sh->full_b[s], 1);
       mbar_init(&sh->empty[s], 1);
     }
     for (int s = 0; s < kWS; ++s) {
       mbar_init(&sh->wfull[s], 1);
-      mbar_init(&sh->wempty[s], kDqWarps);
+      mbar_init(&sh->wempty[s], kDqWarps / 2);
     }
     mbar_init(&sh->d_full, 1);
     mbar_init(&sh->d_empty, kEpiWarps * G::kCG);
@@ -381,66 +383,76 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
   } else if (warp >= kEpiWarps) {
     // -------------------------------------------- dequantization (A)
     const int q = warp & 3;                  // TMEM lane quarter
-    const int h = (warp - kEpiWarps) >> 2;   // which half of the 64-wide stage
+    // which half of a stage (no weight staging), or which stage parity
+    // (weight staging: warps h = 0 decode even stages, h = 1 odd ones)
+    const int h = (warp - kEpiWarps) >> 2;
+    uint32_t it_base = 0;  // stages of the tiles before this one
     TileWalker walk(t_offs, E, kBN, col_tiles);
-    uint32_t it = 0;
-    uint32_t wit = 0;  // weight-slot ring position (input gradient)
+    uint32_t it = 0;  // stage counter of the unstaged forward
     bool ok = true;
     for (int64_t tile = unit; ok && walk.seek(tile); tile += units) {
       const int64_t e = walk.expert;
       const int64_t m0 = walk.col_tile * G::kTileM + rank * kBM;  // this CTA's features
       if constexpr (!kDgrad && kWTma) {
         // Thread = weight row n = m0 + 32q + lane (slot row 32q + lane);
-        // stage half h: k = ks*kBK + 64h .. +64, i.e. 16-byte chunks 2h and
-        // 2h+1 of the 64-byte slot row (64-byte swizzle), and scale bytes
-        // 4ks + 2h, +1 of the row's 16-byte scale box.
+        // the warp decodes every other stage (parity h): k = ks*kBK ..
+        // +128, the four 16-byte chunks of the 64-byte slot row (64-byte
+        // swizzle) and scale bytes 4ks .. 4ks+3 of the row's 16-byte scale
+        // box, in two halves of 64 k.  The other parity group's decode
+        // overlaps this group's TMEM-store wait.
         static_assert(kBK == 128, "weight staging of the forward assumes 128-deep stages");
         const int row = 32 * q + lane;
         const int swz = (row >> 1) & 3;
-        const uint8_t* srow = scales + (e * N + m0 + row) * (K / 32) + 2 * h;
-        for (int ks = 0; ks < nk && ok; ++ks, ++wit) {
-          const int ws = wit % kWS;
-          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wit / kWS) & 1, abort, wait_limit_ns)))
+        const uint8_t* srow = scales + (e * N + m0 + row) * (K / 32);
+        for (int ks = h; ks < nk && ok; ks += 2) {
+          const uint32_t wi = it_base + ks;  // stage index (weight slots and A slots)
+          const int ws = wi % kWS;
+          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wi / kWS) & 1, abort, wait_limit_ns)))
             break;
           const uint8_t* wrow = sW + ws * G::kWBytes + row * 64;
-          uint4 d[2];
-          uint32_t sb[2];
+          uint4 d[4];
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-            d[c] = *reinterpret_cast<const uint4*>(wrow + 16 * ((2 * h + c) ^ swz));
-          if (scales_by_tma) {
-            const uint8_t* sp = sS + ws * G::kSBytes + row * 16 + ((4 * ks) & 15) + 2 * h;
-            sb[0] = sp[0];
-            sb[1] = sp[1];
-          } else {
-            sb[0] = srow[4 * ks];
-            sb[1] = srow[4 * ks + 1];
-          }
+          for (int c = 0; c < 4; ++c)
+            d[c] = *reinterpret_cast<const uint4*>(wrow + 16 * (c ^ swz));
+          uint32_t sb4;
+          if (scales_by_tma)
+            sb4 = *reinterpret_cast<const uint32_t*>(sS + ws * G::kSBytes + row * 16 + ((4 * ks) & 15));
+          else
+            sb4 = *reinterpret_cast<const uint32_t*>(srow + 4 * ks);
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh->wempty[ws]);
-          uint32_t v[32];
+          const int s = wi % S;
+          bool waited = false;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint32_t w[4] = {d[c].x, d[c].y, d[c].z, d[c].w};
-            const float sc = scale_f32(sb[c]);
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
+            for (int c = 0; c < 2; ++c) {
+              const uint4 dd = d[2 * hh + c];
+              const uint32_t w[4] = {dd.x, dd.y, dd.z, dd.w};
+              const float sc = scale_f32((sb4 >> (8 * (2 * hh + c))) & 0xFFu);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
+            }
+            if (!waited) {
+              if (!(ok = warp_wait<kPair>(&sh->empty[s], ((wi / S) & 1) ^ 1, abort, wait_limit_ns)))
+                break;
+              tc_fence_after();
+              waited = true;
+            }
+            const uint32_t col = kACol + G::kACols * s + 32 * hh;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + col + 16 * c, v + 16 * c);
           }
-          const int s = it % S;
-          if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
-            break;
-          tc_fence_after();
-          const uint32_t col = kACol + G::kACols * s + 32 * h;
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tmem_st_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + col + 16 * c, v + 16 * c);
+          if (!ok) break;
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
-          ++it;
         }
+        it_base += nk;
       } else if constexpr (!kDgrad) {
         // Thread = weight row n; kBK/2 consecutive k (kBK/4 bytes, one or
         // two 16-byte loads, one scale per 32 k) per stage half.
@@ -503,33 +515,32 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
         }
       } else {
         // The warp's 32 output features k = m0 + 32q + (0..31) are TMEM
-        // lanes 32q..32q+31, in the order kperm() gives; a stage half
-        // covers kBK/2 reduction indices n, done in sub-steps of 32.  In a
+        // lanes 32q..32q+31, in the order kperm() gives; the warp decodes
+        // every other stage (parity h), all kBK reduction indices n of it,
+        // in sub-steps of 32.  In a
         // sub-step thread t reads 4 contiguous bytes (word t%4 of the
         // warp's 16 bytes) of rows n = base + 8j + t/4, j = 0..3, from the
         // TMA-staged tile.  Byte c of the word (k = 8(t%4) + 2c, +1) goes
         // to 8x8 block c; movmatrix transposes each block so that a thread
         // holds bf16 pairs along n, and block c fills TMEM lanes 8c..8c+7.
-        constexpr int kSub = kBK / 64;  // sub-steps per stage half
         const int rsub = lane >> 2, csub = lane & 3;
         const uint8_t* scol = scales + e * N * (K / 32) + (m0 + 32 * q) / 32;
         const int soff = (int)((m0 / 32) & 15) + q;  // this warp's byte in a scale box row
-        for (int ks = 0; ks < nk && ok; ++ks, ++wit) {
-          const int ws = wit % kWS;
-          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wit / kWS) & 1, abort, wait_limit_ns)))
+        constexpr int kSubAll = kBK / 32;  // sub-steps of 32 rows n per stage
+        for (int ks = h; ks < nk && ok; ks += 2) {
+          const uint32_t wi = it_base + ks;
+          const int ws = wi % kWS;
+          if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wi / kWS) & 1, abort, wait_limit_ns)))
             break;
           const uint8_t* wst = sW + ws * G::kWBytes;
           const uint8_t* sst = sS + ws * G::kSBytes;
-          // All of the slot's reads first (16 independent shared loads in
-          // flight), then the slot goes back to the producer.
-          uint32_t wd[kSub][4];
-          float sc[kSub][4];
+          uint32_t wd[kSubAll][4];
+          float sc[kSubAll][4];
 #pragma unroll
-          for (int sub_i = 0; sub_i < kSub; ++sub_i)
+          for (int sub_i = 0; sub_i < kSubAll; ++sub_i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int row = (kBK / 2) * h + 32 * sub_i + 8 * j + rsub;  // n within the stage
-              // 64-byte swizzle: 16-byte chunk q sits at chunk q ^ ((row >> 1) & 3)
+              const int row = 32 * sub_i + 8 * j + rsub;  // n within the stage
               wd[sub_i][j] = *reinterpret_cast<const uint32_t*>(
                   wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
               const uint32_t sb = scales_by_tma
@@ -539,9 +550,9 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
             }
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh->wempty[ws]);
-          const int s = it % S;
+          const int s = wi % S;
 #pragma unroll
-          for (int sub_i = 0; sub_i < kSub; ++sub_i) {
+          for (int sub_i = 0; sub_i < kSubAll; ++sub_i) {
             uint32_t v[2][8];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -550,11 +561,11 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
                 v[c >> 1][2 * j + (c & 1)] =
                     movmatrix_trans(dequant_pair((wd[sub_i][j] >> (8 * c)) & 0xFFu, sc[sub_i][j]));
             if (sub_i == 0) {
-              if (!(ok = warp_wait<kPair>(&sh->empty[s], ((it / S) & 1) ^ 1, abort, wait_limit_ns)))
+              if (!(ok = warp_wait<kPair>(&sh->empty[s], ((wi / S) & 1) ^ 1, abort, wait_limit_ns)))
                 break;
               tc_fence_after();
             }
-            const uint32_t col = kACol + G::kACols * s + (kBK / 4) * h + 16 * sub_i;
+            const uint32_t col = kACol + G::kACols * s + 16 * sub_i;
 #pragma unroll
             for (int r = 0; r < 2; ++r)
               tmem_st_16x128b_x4(tmem + ((uint32_t)(32 * q + 16 * r) << 16) + col, v[r]);
@@ -564,8 +575,8 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           tc_fence_before();
           __syncwarp();
           if (lane == 0) arrive_leader<kPair>(&sh->full_a[s]);
-          ++it;
         }
+        it_base += nk;
       }
     }
   } else {
