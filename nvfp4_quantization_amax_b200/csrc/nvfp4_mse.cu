@@ -14,9 +14,10 @@
 // code wins.  A code whose d_c underflows to zero is skipped.  With g = 0
 // (an all-zero tensor) the output is the max rule's: scale 1.0, zero codes.
 //
-// Work split: kLanes lanes share a block, each trying every kLanes-th code,
-// and combine (error, code) with shuffles; the lane holding the best code's
-// first slot then writes the block's eight code bytes and its scale byte.
+// Work split: kLanes lanes share a block, each trying every kLanes-th code
+// (only the codes that can win: see the pruning below), and combine (error,
+// code) with shuffles; the lane of the first slot then writes the block's
+// eight code bytes and its scale byte.
 // This is ALU work (126 candidates x 16 divisions and fmas per block), so
 // the grid is one thread per (block, lane slot) and the CTA scheduler
 // balances the waves.
@@ -78,12 +79,45 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
     best_c = 1;
     if (valid) {
       double wd[16];
+      float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) wd[i] = (double)w[i];
-      for (int c = 1 + slot; c <= 126; c += kLanes) {
+      for (int i = 0; i < 16; ++i) {
+        wd[i] = (double)w[i];
+        amax = fmaxf(amax, fabsf(w[i]));
+      }
+      // Codes are visited from the top down, and only where they can win:
+      //  * from c_top = the smallest code whose quotient amax / d rounds to
+      //    at most 0.25 (every weight's code is then 0, so every larger code
+      //    reconstructs all zeros with exactly the same error and loses the
+      //    tie to c_top); 126 if there is none;
+      //  * down to the first code whose clipping error alone exceeds the
+      //    best sum so far: with 6d < amax the largest weight is cut to 6d,
+      //    so the sum is at least (amax - 6d)^2 (exact in double; the
+      //    accumulated sum is within 2^-49 of the exact one), and it only
+      //    grows as d shrinks.
+      // Visiting in decreasing order with <= keeps the smallest code among
+      // equal sums, as the full ascending sweep does.
+      auto all_zero = [&](int c) {
+        const float dc = s_d[c];
+        return dc != 0.0f && __fdiv_rn(amax, dc) <= 0.25f;
+      };
+      int c_top = 126;
+      if (all_zero(126)) {
+        int lo = 1, hi = 126;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (all_zero(mid)) hi = mid;
+          else lo = mid + 1;
+        }
+        c_top = lo;
+      }
+      const double amax_d = (double)amax;
+      for (int c = c_top - slot; c >= 1; c -= kLanes) {
         const float d = s_d[c];
-        if (d == 0.0f) continue;
+        if (d == 0.0f) break;  // d only shrinks further down
         const double dd = (double)d;
+        const double t = amax_d - 6.0 * dd;
+        if (t > 0.0 && t * t * (1.0 - 0x1p-40) > best) break;
         double err = 0.0;
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
@@ -94,7 +128,7 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
           const double e1 = fma(f16_to_f64(h2 >> 16), dd, -wd[i + 1]);
           err = fma(e1, e1, err);
         }
-        if (err < best) {  // strict: the first (smallest) code keeps a tie
+        if (err <= best) {  // descending: a tie goes to the smaller code
           best = err;
           best_c = c;
         }

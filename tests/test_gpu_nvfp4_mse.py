@@ -96,3 +96,22 @@ def test_mse_full_expert_weight():
     energy = (x.double() ** 2).view(-1, 16).sum(dim=1)
     assert bool((e_mse <= e_max * (1 + 1e-6) + 1e-12 * energy).all())
     assert float(e_mse.sum()) < float(e_max.sum())
+
+
+def test_mse_ties_and_pruning_edges():
+    # blocks where many scale codes tie (a single nonzero weight, constant
+    # blocks, values on the E2M1 grid) and blocks whose weights are tiny or
+    # huge next to the tensor maximum (the top and bottom of the code range)
+    rows = []
+    vals = [2.0 ** k for k in range(-12, 6)] + [3.0, 0.75, 1.5, 6.0, 0.1, 7.0]
+    for v in vals:
+        b = np.zeros(16)
+        b[5] = v
+        rows.append(b)
+        rows.append(np.full(16, v))
+        rows.append(np.array([6, 4, 3, 2, 1.5, 1, 0.5, 0, -6, -4, -3, -2, -1.5, -1, -0.5, 0.0]) * v)
+    x = torch.tensor(np.concatenate(rows).reshape(-1, 64), dtype=torch.float32)
+    x[0, 0] = 2000.0  # the tensor maximum: small blocks sit near the bottom codes
+    for dtype in (torch.bfloat16, torch.float32):
+        xd = x.to(dtype)
+        check(xd.to(DEV), "bf16" if dtype == torch.bfloat16 else "f32")
