@@ -127,6 +127,29 @@ __device__ __forceinline__ uint32_t e2m1x2(float a, float b) {
   return r;
 }
 
+// E2M1 codes (one byte, a in the low nibble) of the binary32 quotients
+// a / d and b / d, exactly as e2m1x2(__fdiv_rn(a, d), __fdiv_rn(b, d)), with
+// the divisions only where they can matter.  r = fl32(1 / d), d in
+// [2^-126, 2^126) (so r is a normal number).  a * r is within 2^-22
+// (relative) of the rounded quotient v; scaling it by 1 -+ 2^-19 gives a
+// bracket that contains v, and where the (monotone) cast gives the same
+// codes at both ends of the bracket it gives them for v too.  Otherwise a
+// quotient lies within ~2^-19 of an E2M1 decision point and the IEEE
+// divisions decide.  Signs (including -0 and underflow to zero) follow a and
+// b in both paths.
+__device__ __forceinline__ uint32_t e2m1x2_quot(float a, float b, float d, float r) {
+  const float va = a * r, vb = b * r;
+  const uint32_t lo = e2m1x2(va * (1.0f - 0x1p-19f), vb * (1.0f - 0x1p-19f));
+  const uint32_t hi = e2m1x2(va * (1.0f + 0x1p-19f), vb * (1.0f + 0x1p-19f));
+  if (lo == hi) return lo;
+  return e2m1x2(__fdiv_rn(a, d), __fdiv_rn(b, d));
+}
+
+// Whether e2m1x2_quot may be used with divisor d.
+__device__ __forceinline__ bool quot_fast_ok(float d) {
+  return d >= 0x1p-126f && d < 0x1p126f;
+}
+
 // Eight f32 -> four bytes of E2M1 codes, element 2j in the low nibble of
 // byte j.
 __device__ __forceinline__ uint32_t e2m1x8(const float* v) {

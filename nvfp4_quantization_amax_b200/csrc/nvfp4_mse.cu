@@ -118,11 +118,14 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
         const double dd = (double)d;
         const double t = amax_d - 6.0 * dd;
         if (t > 0.0 && t * t * (1.0 - 0x1p-40) > best) break;
+        const bool fast = quot_fast_ok(d);
+        const float r = fast ? __frcp_rn(d) : 0.0f;
         double err = 0.0;
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const uint32_t h2 =
-              e2m1x2_to_f16x2(e2m1x2(__fdiv_rn(w[i], d), __fdiv_rn(w[i + 1], d)));
+          const uint32_t h2 = e2m1x2_to_f16x2(
+              fast ? e2m1x2_quot(w[i], w[i + 1], d, r)
+                   : e2m1x2(__fdiv_rn(w[i], d), __fdiv_rn(w[i + 1], d)));
           const double e0 = fma(f16_to_f64(h2 & 0xFFFFu), dd, -wd[i]);
           err = fma(e0, e0, err);
           const double e1 = fma(f16_to_f64(h2 >> 16), dd, -wd[i + 1]);
@@ -155,9 +158,22 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
     for (int i = 0; i < 16; ++i) {
       // a zero weight (either sign) gives code 0, also when d underflowed;
       // a tiny negative weight keeps its sign bit
-      v[i] = w[i] == 0.0f ? 0.0f : __fdiv_rn(w[i], d);
+      v[i] = w[i] == 0.0f ? 0.0f : w[i];
     }
-    codes = make_uint2(e2m1x8(v), e2m1x8(v + 8));
+    if (quot_fast_ok(d)) {
+      const float r = __frcp_rn(d);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        lo |= e2m1x2_quot(v[2 * j], v[2 * j + 1], d, r) << (8 * j);
+        hi |= e2m1x2_quot(v[8 + 2 * j], v[8 + 2 * j + 1], d, r) << (8 * j);
+      }
+      codes = make_uint2(lo, hi);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = v[i] == 0.0f ? 0.0f : __fdiv_rn(v[i], d);
+      codes = make_uint2(e2m1x8(v), e2m1x8(v + 8));
+    }
   }
   packed[blk] = codes;
   block_scales[blk] = (uint8_t)best_c;
