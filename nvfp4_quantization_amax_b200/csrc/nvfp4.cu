@@ -62,10 +62,16 @@ nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restr
   __shared__ uint32_t s_max[kNvThreads / 32];
   uint32_t m = 0;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
-  for (int64_t it = (int64_t)blockIdx.x * kNvThreads + threadIdx.x; it < n_items; it += stride) {
-    uint4 a, b;
-    load_vec8<DT>(x, it, a, b);
-    m = max(m, amax8<DT>(a, b));
+  // kNvUnroll independent 16-byte loads in flight per thread
+  for (int64_t base = (int64_t)blockIdx.x * kNvThreads + threadIdx.x; base < n_items;
+       base += stride * kNvUnroll) {
+    uint4 a[kNvUnroll], b[kNvUnroll];
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u)
+      if (base + u * stride < n_items) load_vec8<DT>(x, base + u * stride, a[u], b[u]);
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u)
+      if (base + u * stride < n_items) m = max(m, amax8<DT>(a[u], b[u]));
   }
   m = __reduce_max_sync(0xffffffffu, m);
   if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
@@ -180,7 +186,7 @@ template <int DT>
 void run_amax(const void* x, int64_t n_items, uint32_t* amax_word, cudaStream_t st) {
   clear_word_kernel<<<1, 1, 0, st>>>(amax_word);
   if (n_items > 0) {
-    nvfp4_amax_kernel<DT><<<grid_for(n_items, kNvThreads * 4, 8), kNvThreads, 0, st>>>(
+    nvfp4_amax_kernel<DT><<<grid_for(n_items, kNvThreads * kNvUnroll, 8), kNvThreads, 0, st>>>(
         x, n_items, amax_word);
   }
 }
