@@ -382,3 +382,12 @@ def test_nvfp4_zero_and_ragged():
     assert float(g.item()) == wg
     assert_bits_equal(u8(p), wp, "packed")
     assert_bits_equal(u8(s), ws, "scales")
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_small_remainders(transpose_w):
+    # experts just above a multiple of the 256-row tile (remainders of 1,
+    # 31, 32, 33, 63, 64 and 65 rows), one-row and empty experts: every
+    # ragged tail the CTA-pair tiling meets
+    counts = [257, 287, 288, 289, 319, 320, 321, 576, 600, 64, 1, 0, 512]
+    check_gemm(counts, 256, 512, transpose_w)
