@@ -40,6 +40,10 @@ W_SHAPE = (64, 2048, 7168)
 KV_SHAPE = (4, 8192, 512)
 CACHE_RUNS = (("fp8", 128), ("mxfp4", 32), ("nvfp4", 16))
 T, E, N, K = 32768, 32, 2048, 7168
+WORKLOAD = ("mx_quantize + mx_dequantize of expert weights bf16 [64,2048,7168]; "
+            "quantize_cache fp8/128, mxfp4/32, nvfp4/16 of KV bf16 [4,8192,512]; "
+            "MXFP4 grouped GEMM fwd + dgrad, x [32768,7168], W [32,2048,7168], "
+            "multinomial expert counts")
 
 
 def algorithmic_bytes():
@@ -395,10 +399,7 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 / Box-Muller inputs of the configured shapes)",
         "config": {
-            "workload": "mx_quantize + mx_dequantize of expert weights bf16 [64,2048,7168]; "
-                        "quantize_cache fp8/128, mxfp4/32, nvfp4/16 of KV bf16 [4,8192,512]; "
-                        "MXFP4 grouped GEMM fwd + dgrad, x [32768,7168], W [32,2048,7168], "
-                        "multinomial expert counts",
+            "workload": WORKLOAD,
             "hbm_fraction_nominal_8tbs": round(gbs / world / 8000.0, 4),
             "l2": "no flush; every kernel's inputs were last touched >126 MB of traffic earlier",
             "parallelism": "replicas" if world > 1 else "single GPU",
@@ -508,8 +509,10 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "bounded sample of the GPU arm's "
-                                                        "workload on the scalar CPU oracle"},
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD,
+                       "sample": "each step times the scalar CPU oracle on a bounded sample of "
+                                 "this workload (rows of the same tensors), single thread"},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
