@@ -78,6 +78,10 @@ def lib():
         L.orc_dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i, p, i]
         L.orc_w4a4_grouped_mm.restype = i
         L.orc_w4a4_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, p, i64, p]
+        L.orc_nvfp4_quantize_rows.restype = i
+        L.orc_nvfp4_quantize_rows.argtypes = [p, i, i64, i64, d, p, p]
+        L.orc_nvfp4_w4a4_grouped_mm.restype = i
+        L.orc_nvfp4_w4a4_grouped_mm.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, i64, p]
         L.orc_grouped_mm.restype = i
         L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
         _lib = L
@@ -351,3 +355,39 @@ def nvfp4_quantize_mse(x_bits, dtype="bf16", g=None):
     if rc != 0:
         raise ValueError("oracle nvfp4_quantize_mse: bad arguments rc=%d" % rc)
     return packed, bs, g
+
+
+def nvfp4_quantize_rows(x_bits, g, dtype="bf16"):
+    """NVFP4 codes and block scales of rows with a given per-tensor scale g."""
+    x = _c(x_bits, _BITS[dtype])
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    packed = np.empty(x.shape[:-1] + (K // 2,), np.uint8)
+    bs = np.empty(x.shape[:-1] + (K // 16,), np.uint8)
+    rc = lib().orc_nvfp4_quantize_rows(_ptr(x), DTYPES[dtype], rows, K, float(g), _ptr(packed),
+                                       _ptr(bs))
+    if rc != 0:
+        raise ValueError("oracle nvfp4_quantize_rows: bad arguments rc=%d" % rc)
+    return packed, bs
+
+
+def nvfp4_w4a4_grouped_mm(x_bits, packed, block_scales, w_global, offs, rows=None):
+    """Exact-sum grouped GEMM of NVFP4 activations (x quantized as one
+    tensor) with NVFP4 expert weights (one global scale per expert)."""
+    x = _c(x_bits, np.uint16)
+    p = _c(packed, np.uint8)
+    s = _c(block_scales, np.uint8)
+    gw = _c(w_global, np.float32)
+    o = _c(offs, np.int32)
+    E, N, Kh = p.shape
+    K = 2 * Kh
+    T = x.shape[0]
+    if rows is None:
+        rows = np.arange(T, dtype=np.int64)
+    r = _c(rows, np.int64)
+    out = np.zeros((r.size, N), np.float64)
+    rc = lib().orc_nvfp4_w4a4_grouped_mm(_ptr(x), _ptr(p), _ptr(s), _ptr(gw), _ptr(o), T, E, N, K,
+                                         _ptr(r), r.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle nvfp4_w4a4_grouped_mm: rc=%d" % rc)
+    return out

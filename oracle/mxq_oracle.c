@@ -693,3 +693,102 @@ done:
   free(w);
   return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* W4A4 NVFP4 grouped GEMM ([MO] "W4A4 NVFP4 on FP4 tensor cores").          */
+/* ------------------------------------------------------------------------ */
+
+/* NVFP4 quantize of rows with a given per-tensor scale g (that of the
+   whole tensor the rows belong to): the per-block steps of
+   orc_nvfp4_quantize.  g == 0 (an all-zero tensor) gives codes 0 and block
+   scales 1.0. */
+int orc_nvfp4_quantize_rows(const void* x, int dtype, int64_t rows, int64_t K, double g,
+                            uint8_t* packed, uint8_t* block_scales) {
+  if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < K / 16; ++b) {
+      int64_t base = r * K + b * 16;
+      double amax_b = 0.0;
+      for (int i = 0; i < 16; ++i) {
+        double a = fabs(load_elem(x, dtype, base + i));
+        if (a > amax_b) amax_b = a;
+      }
+      double s = g == 0.0 ? 1.0 : orc_nvfp4_block_scale(amax_b, g);
+      block_scales[r * (K / 16) + b] = orc_encode_e4m3(s);
+      double d = f32_mul(s, g);
+      for (int j = 0; j < 8; ++j) {
+        int nib[2] = {0, 0};
+        for (int h = 0; h < 2 && g != 0.0; ++h) {
+          double xi = load_elem(x, dtype, base + 2 * j + h);
+          nib[h] = (orc_e2m1_code(fabs(f32_div(xi, d))) & 7) | (xi < 0.0 ? 8 : 0);
+        }
+        packed[r * (K / 2) + b * 8 + j] = (uint8_t)(nib[0] | (nib[1] << 4));
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* Value of NVFP4 element k of a row: E2M1 code * E4M3 block scale * g,
+   exact in double. */
+static double nv_element(const uint8_t* packed_row, const uint8_t* scales_row, int64_t k,
+                         double g) {
+  uint8_t byte = packed_row[k / 2];
+  int nib = (k % 2 == 0) ? (byte & 15) : (byte >> 4);
+  return E2M1_TABLE[nib] * orc_decode_e4m3(scales_row[k / 16]) * g;
+}
+
+/* x: bf16 [T, K] activations, NVFP4-quantized as one tensor (its global
+   scale from max |x| over all of x), then dequantized exactly; weights:
+   packed [E, N, K/2], E4M3 block scales [E, N, K/16] and one global scale
+   per expert.  out[i][n] = sum_k deq(q(x))[t][k] * deq(W_e)[n][k] for t =
+   rows[i], summed in double in index order (not rounded). */
+int orc_nvfp4_w4a4_grouped_mm(const uint16_t* x, const uint8_t* packed, const uint8_t* bscales,
+                              const float* w_global, const int32_t* offs, int64_t T, int64_t E,
+                              int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                              double* out) {
+  if (E < 1 || K % 16 != 0 || N < 1 || T < 0) return ORC_EARG;
+  if (orc_check_offs(offs, E, T) != ORC_OK) return ORC_EOFFS;
+  double amax = 0.0;
+  for (int64_t i = 0; i < T * K; ++i) {
+    double a = fabs(decode_bf16(x[i]));
+    if (a > amax) amax = a;
+  }
+  double gx = amax == 0.0 ? 0.0 : orc_nvfp4_global_scale(amax);
+  uint8_t* qp = (uint8_t*)malloc((size_t)(K / 2));
+  uint8_t* qs = (uint8_t*)malloc((size_t)(K / 16));
+  double* xa = (double*)malloc((size_t)K * sizeof(double));
+  double* w = (double*)malloc((size_t)(N * K) * sizeof(double));
+  int rc = ORC_OK;
+  if (!qp || !qs || !xa || !w) {
+    rc = ORC_EARG;
+    goto done;
+  }
+  for (int64_t e = 0; e < E; ++e) {
+    int64_t lo = e == 0 ? 0 : offs[e - 1], hi = offs[e];
+    int have = 0;
+    for (int64_t i = 0; i < nrows && !have; ++i) have = rows[i] >= lo && rows[i] < hi;
+    if (!have) continue;
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k)
+        w[n * K + k] = nv_element(packed + (e * N + n) * (K / 2), bscales + (e * N + n) * (K / 16),
+                                  k, (double)w_global[e]);
+    for (int64_t i = 0; i < nrows; ++i) {
+      int64_t t = rows[i];
+      if (t < lo || t >= hi) continue;
+      orc_nvfp4_quantize_rows(x + t * K, ORC_BF16, 1, K, gx, qp, qs);
+      for (int64_t k = 0; k < K; ++k) xa[k] = nv_element(qp, qs, k, gx);
+      for (int64_t n = 0; n < N; ++n) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += xa[k] * w[n * K + k];
+        out[i * N + n] = acc;
+      }
+    }
+  }
+done:
+  free(qp);
+  free(qs);
+  free(xa);
+  free(w);
+  return rc;
+}

@@ -809,3 +809,44 @@ def test_w4a4_exact_on_representable_activations():
     y4 = oracle.w4a4_grouped_mm(xg, packed, scales, offs)
     y16 = oracle.grouped_mm(xg, packed, scales, offs)
     assert np.array_equal(y4, y16)
+
+
+# --------------------------------------------- W4A4 NVFP4 grouped GEMM
+
+def nv_dense(packed, bscales, g):
+    """float64 values of NVFP4 storage (numpy, from the table and torch's
+    E4M3 decode)."""
+    tab = full_table()
+    codes = np.stack([packed & 15, packed >> 4], axis=-1).reshape(packed.shape[:-1] + (-1,))
+    sc = torch.from_numpy(np.ascontiguousarray(bscales)).view(torch.float8_e4m3fn).double().numpy()
+    return tab[codes] * np.repeat(sc, 16, axis=-1) * g
+
+
+def test_nvfp4_quantize_rows_equals_whole_tensor():
+    x = torch.cat([gen.kv_cache((1, 3, 64)).view(3, 64), gen.mixed_blocks(3, 64)])
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    p2, s2 = oracle.nvfp4_quantize_rows(bits[2:5], g)
+    assert np.array_equal(p2, p[2:5]) and np.array_equal(s2, s[2:5])
+
+
+def test_nvfp4_w4a4_matches_numpy():
+    xb, packed_mx, scales_mx, offs = small_moe()
+    E, N = packed_mx.shape[0], packed_mx.shape[1]
+    K = 2 * packed_mx.shape[2]
+    # NVFP4 weights: each expert quantized as its own tensor
+    W = gen.expert_weights(E, N, K).view(torch.int16).numpy().view(np.uint16)
+    wp, ws, wg = [], [], []
+    for e in range(E):
+        p, s, g = oracle.nvfp4_quantize(W[e])
+        wp.append(p); ws.append(s); wg.append(g)
+    wp, ws, wg = np.stack(wp), np.stack(ws), np.array(wg, np.float32)
+    xp, xs, xg = oracle.nvfp4_quantize(xb)
+    xq = nv_dense(xp, xs, xg)
+    want = np.zeros((xb.shape[0], N))
+    lo = 0
+    for e, hi in enumerate(offs):
+        want[lo:hi] = xq[lo:hi] @ nv_dense(wp[e], ws[e], float(wg[e])).T
+        lo = hi
+    got = oracle.nvfp4_w4a4_grouped_mm(xb, wp, ws, wg, offs)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
