@@ -233,6 +233,17 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
     xq, xs = mxq.mx_quantize(step.x)
     calls["w4a4_grouped_mm"] = lambda: mxq.w4a4_grouped_mm(step.x, step.P5, step.S5, step.offs,
                                                            step.y, step.status, xq, xs)
+    # ... and in NVFP4 (each expert's weight quantized as its own tensor)
+    import synthetic as gen
+    W5 = gen.expert_weights(E, N, K, device=dev, workload=5)
+    nvq = [mxq.nvfp4_quantize(W5[e]) for e in range(E)]
+    del W5
+    nvp = torch.stack([q[0] for q in nvq])
+    nvs = torch.stack([q[1] for q in nvq])
+    nvg = torch.cat([q[2] for q in nvq])
+    del nvq
+    calls["nvfp4_w4a4_grouped_mm"] = lambda: mxq.nvfp4_w4a4_grouped_mm(
+        step.x, nvp, nvs, nvg, step.offs, step.y, step.status)
     out = {}
     for name, fn in calls.items():
         for _ in range(2):
@@ -421,6 +432,7 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
         rows = {}
         w4 = next_ms.pop("w4a4_grouped_mm", None)
+        nv4 = next_ms.pop("nvfp4_w4a4_grouped_mm", None)
         for n, ms in next_ms.items():
             gbs = nb[n] / (ms * 1e-3) / 1e9
             rows[n] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
@@ -439,6 +451,13 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
                 "frac_of_fp4_peak": round(tf / (4.0 * peaks["bf16_tflops"]), 4),
                 "includes": "mx_quantize of the activations + the block-scaled GEMM",
                 "workload": "x bf16 [32768,7168], W MXFP4 [32,2048,7168], multinomial counts"}
+        if nv4 is not None:
+            tf = gemm_flops() / (nv4 * 1e-3) / 1e12
+            rows["nvfp4_w4a4_grouped_mm"] = {
+                "ms": round(nv4, 4), "tflops": round(tf, 1),
+                "frac_of_fp4_peak": round(tf / (4.0 * peaks["bf16_tflops"]), 4),
+                "includes": "nvfp4_quantize of the activations (two passes) + the block-scaled GEMM",
+                "workload": "x bf16 [32768,7168], W NVFP4 [32,2048,7168], multinomial counts"}
         line["next_rows"] = rows
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)

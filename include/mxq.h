@@ -194,6 +194,29 @@ int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void
                           const void* scales, const int32_t* offs, int64_t T, int64_t E, int64_t N,
                           int64_t K, void* y, int32_t* dev_status, void* stream);
 
+/* W4A4 grouped GEMM in NVFP4: activations and expert weights both NVFP4 on
+ * the block-scaled tensor cores ([MO] "W4A4 NVFP4 on FP4 tensor cores";
+ * two-level format of [MO] "NVFP4 in the code: two scales and a nibble").
+ *
+ *  x_packed, x_block_scales, x_global_scale  device, the activations as
+ *           nvfp4_quantize writes them for the whole [T, K] tensor: [T, K/2]
+ *           E2M1 bytes, [T, K/16] E4M3 bytes, one float g_x.
+ *  packed, block_scales  device, [E, N, K/2] and [E, N, K/16] bytes: each
+ *           expert's weight in NVFP4 (e.g. nvfp4_quantize of W_e).
+ *  w_global_scales  device, float [E]: each expert's g.
+ *  offs, dev_status, y  as mxfp4_w4a4_grouped_mm.
+ *  y[t, n] = g_x g_w[e] sum_k (code * s_b)_x[t, k] (code * s_b)_w[n, k]: the
+ *  tensor core multiplies codes and block scales exactly and accumulates in
+ *  f32; the product of the two global scales multiplies the f32 sum, and y is
+ *  rounded to bf16.
+ *  Errors as mxfp4_w4a4_grouped_mm (K % 16 != 0 -> MXQ_ERR_SHAPE; K % 256 or
+ *  N % 128 nonzero -> MXQ_ERR_UNSUPPORTED). */
+int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
+                          const float* x_global_scale, const void* packed,
+                          const void* block_scales, const float* w_global_scales,
+                          const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K, void* y,
+                          int32_t* dev_status, void* stream);
+
 /* Device workspace nvfp4_quantize needs (bytes, 16-byte aligned). */
 #define MXQ_NVFP4_WORKSPACE_BYTES 16
 

@@ -21,6 +21,7 @@ from ._abi import (  # noqa: F401
     mxfp4_grouped_mm,
     nvfp4_dequantize,
     nvfp4_quantize,
+    nvfp4_w4a4_grouped_mm,
     dequantize_cache_packed,
     quantize_cache,
     quantize_cache_packed,

@@ -58,6 +58,8 @@ def lib():
         L.dequantize_cache_packed.argtypes = [p, p, i64, i64, i, i32, p, i, p]
         L.mxfp4_w4a4_grouped_mm.restype = i
         L.mxfp4_w4a4_grouped_mm.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p, p]
+        L.nvfp4_w4a4_grouped_mm.restype = i
+        L.nvfp4_w4a4_grouped_mm.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p]
         L.mxq_set_wait_limit_ns.restype = ctypes.c_uint64
         L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         _lib = L
@@ -299,6 +301,43 @@ def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=Non
     rc = lib().mxfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(packed), _ptr(scales), _ptr(offs),
                                      T, E, N, K, _ptr(out), st, _stream(x.device))
     _check(rc, "mxfp4_w4a4_grouped_mm")
+    return _to_host(out) if host else out
+
+
+def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=None,
+                          status=None):
+    """W4A4 grouped GEMM in NVFP4: the bf16 activations x [T, K] are
+    quantized to NVFP4 as one tensor (nvfp4_quantize) and multiplied with the
+    NVFP4 expert weights (packed [E, N, K/2], E4M3 block scales [E, N, K/16],
+    float32 global scales [E]) on the block-scaled tensor cores.  Returns
+    bf16 [T, N]."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("nvfp4_w4a4_grouped_mm: activations must be bf16")
+    x, host = _to_device(x)
+    packed, _ = _to_device(packed)
+    block_scales, _ = _to_device(block_scales)
+    w_global_scales, _ = _to_device(w_global_scales)
+    offs, _ = _to_device(offs)
+    x, packed, block_scales = x.contiguous(), packed.contiguous(), block_scales.contiguous()
+    w_global_scales = w_global_scales.to(torch.float32).contiguous()
+    offs = offs.to(torch.int32).contiguous()
+    E, N, Kh = packed.shape
+    K = 2 * Kh
+    T = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("nvfp4_w4a4_grouped_mm: x must be [T, %d]" % K)
+    if (tuple(block_scales.shape) != (E, N, K // 16) or offs.numel() != E or
+            w_global_scales.numel() != E):
+        raise ValueError("nvfp4_w4a4_grouped_mm: block_scales [E, N, K/16], global scales [E] "
+                         "and offs [E] expected")
+    xq, xs, xg = nvfp4_quantize(x)
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    rc = lib().nvfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(xg), _ptr(packed),
+                                     _ptr(block_scales), _ptr(w_global_scales), _ptr(offs),
+                                     T, E, N, K, _ptr(out), st, _stream(x.device))
+    _check(rc, "nvfp4_w4a4_grouped_mm")
     return _to_host(out) if host else out
 
 

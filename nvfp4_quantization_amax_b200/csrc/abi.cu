@@ -149,6 +149,25 @@ int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void
                                 dev_status, get_wait_limit_ns(), (cudaStream_t)stream);
 }
 
+int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
+                          const float* x_global_scale, const void* packed,
+                          const void* block_scales, const float* w_global_scales,
+                          const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K, void* y,
+                          int32_t* dev_status, void* stream) {
+  if (T < 0 || E < 1 || N < 1 || K < 16 || K % 16 != 0) return MXQ_ERR_SHAPE;
+  if (!packed || !block_scales || !w_global_scales || !offs) return MXQ_ERR_INVALID_ARG;
+  if (T == 0) return MXQ_OK;
+  if (!x_packed || !x_block_scales || !x_global_scale || !y) return MXQ_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 128 != 0 || T >= ((int64_t)1 << 31) || E * N >= ((int64_t)1 << 31))
+    return MXQ_ERR_UNSUPPORTED;
+  if (!aligned16(x_packed) || !aligned16(x_block_scales) || !aligned16(packed) ||
+      !aligned16(block_scales) || !aligned16(y))
+    return MXQ_ERR_ALIGNMENT;
+  return launch_nvfp4_w4a4_grouped_mm(x_packed, x_block_scales, x_global_scale, packed,
+                                      block_scales, w_global_scales, offs, T, E, N, K, y,
+                                      dev_status, get_wait_limit_ns(), (cudaStream_t)stream);
+}
+
 int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
                    void* block_scales, float* global_scale, void* workspace, void* stream) {
   if (!valid_dtype(x_dtype)) return MXQ_ERR_INVALID_ARG;

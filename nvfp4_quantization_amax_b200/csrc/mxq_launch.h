@@ -37,6 +37,11 @@ int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const 
                             int64_t rows, int64_t K, void* out, int dt, cudaStream_t st);
 uint64_t set_wait_limit_ns(uint64_t ns);
 uint64_t get_wait_limit_ns();
+int launch_nvfp4_w4a4_grouped_mm(const void* xq, const void* xs, const float* xg,
+                                 const void* packed, const void* scales, const float* wg,
+                                 const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
+                                 void* y, int32_t* dev_status, uint64_t wait_limit_ns,
+                                 cudaStream_t st);
 int launch_w4a4_grouped_mm(const void* xq, const void* xs, const void* packed, const void* scales,
                            const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
                            void* y, int32_t* dev_status, uint64_t wait_limit_ns, cudaStream_t st);

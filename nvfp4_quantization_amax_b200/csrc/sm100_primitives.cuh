@@ -345,16 +345,30 @@ __device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// NVFP4 form: E2M1 A and B with one UE4M3 scale per 16 K per row (K = 64
+// per instruction: four scales per row, one whole TMEM word).
+__device__ __forceinline__ void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Instruction descriptor of kind::mxf4 (block-scaled): E2M1 A and B
 // (K-major), E8M0 scales, f32 D; the two scale ids select the byte of the
 // TMEM scale word where this instruction's scales start.
 __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t a_sf_id,
-                                                  uint32_t b_sf_id) {
+                                                  uint32_t b_sf_id, bool e8m0_scales = true) {
   return (b_sf_id << 4)              // B scale-factor id
          | (1u << 7)                 // A format E2M1
          | (1u << 10)                // B format E2M1
          | ((uint32_t)(N >> 3) << 17)
-         | (1u << 23)                // scale format E8M0
+         | ((e8m0_scales ? 1u : 0u) << 23)  // scale format: E8M0, else UE4M3
          | ((uint32_t)(M >> 4) << 24)
          | (a_sf_id << 29);          // A scale-factor id
 }

@@ -36,6 +36,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "mxq.h"
 #include "mxq_device.cuh"
@@ -53,20 +54,37 @@ using namespace sm100;
 constexpr int kM = 128;                 // weight rows per tile (TMEM lanes)
 constexpr int kN = 256;                 // tokens per tile (MMA N)
 constexpr int kKB = 128;                // bytes of codes per row per stage (256 K)
-constexpr int kStages = 3;
+constexpr int kMaxStages = 3;
 constexpr uint32_t kABytes = kM * kKB;            // 16 KB
 constexpr uint32_t kBBytes = kN * kKB;            // 32 KB
 constexpr uint32_t kSfBlock = 512;                // 128 rows x 4 scales
-constexpr uint32_t kSfaBytes = 2 * kSfBlock;      // 128 rows x 8 scales
-constexpr uint32_t kSfbBytes = 4 * kSfBlock;      // 256 rows x 8 scales
-constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr uint32_t kStagingBytes = kN * kM * 2;   // 64 KB of bf16 output
 constexpr int kMaxSmemExperts = 256;
-constexpr uint32_t kSmem = 1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
 constexpr int kTmemCols = 512;
 constexpr int kDCol = 0;                // accumulator: columns [0, 256)
-constexpr int kSfaCol = 256;            // A scales: 2 blocks x 4 columns
-constexpr int kSfbCol = 264;            // B scales: 4 blocks x 4 columns
+constexpr int kSfaCol = 256;            // A scales: 4 columns per block
+
+// The two block-scaled formats: MXFP4 (one E8M0 scale per 32 K; a stage's
+// 8 scales per row fill 2 blocks, each MMA uses half a TMEM word) and NVFP4
+// (one UE4M3 scale per 16 K; 16 scales per row, 4 blocks, each MMA uses a
+// whole word).
+template <bool kNV>
+struct W4Fmt {
+  static constexpr int kScalesPerRow = kNV ? 16 : 8;       // per stage (256 K)
+  static constexpr int kBlocks = kScalesPerRow / 4;         // per 128-row group
+  static constexpr uint32_t kSfaBytes = kBlocks * kSfBlock;
+  static constexpr uint32_t kSfbBytes = 2 * kBlocks * kSfBlock;  // two 128-row groups
+  static constexpr int kSfbCol = kSfaCol + 4 * kBlocks;
+  // NVFP4 stages are larger (twice the scale bytes): two fit beside the
+  // output staging, which the operand feed of this kernel tolerates.
+  static constexpr int kStages = kNV ? 2 : 3;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr uint32_t kSmem =
+      1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+  static_assert(kSfbCol + 8 * kBlocks <= kTmemCols, "TMEM columns");
+};
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kSfWarp = 5;
@@ -74,12 +92,10 @@ constexpr int kMmaWarp = 6;
 constexpr int kThreads = 7 * 32;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
-static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
-static_assert(kSmem <= 232448, "shared memory per CTA");
 
 struct Shared {
-  uint64_t full[kStages];   // codes (TMA bytes) and scales (warp 5) of a stage are in smem
-  uint64_t empty[kStages];  // the stage's MMAs (and scale copies) completed
+  uint64_t full[kMaxStages];   // codes (TMA bytes) and scales (warp 5) of a stage are in smem
+  uint64_t empty[kMaxStages];  // the stage's MMAs (and scale copies) completed
   uint64_t d_full, d_empty, drain;
   uint32_t tmem_base;
   int abort;
@@ -112,11 +128,18 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // core's scale layout (s in 0..3).
 __device__ __forceinline__ uint32_t sf_offset(int r) { return 16 * (r & 31) + 4 * ((r >> 5) & 3); }
 
+template <bool kNV>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const uint8_t* __restrict__ x_scales, const uint8_t* __restrict__ w_scales,
+               const float* __restrict__ x_global, const float* __restrict__ w_global,
                const int32_t* __restrict__ offs, int64_t T, int64_t E, int64_t N, int64_t K,
                __nv_bfloat16* __restrict__ y, int32_t* dev_status, uint64_t wait_limit_ns) {
+  using F = W4Fmt<kNV>;
+  constexpr int kStages = F::kStages;
+  constexpr uint32_t kStageBytes = F::kStageBytes;
+  constexpr uint32_t kSfaBytes = F::kSfaBytes;
+  constexpr int kSfbCol = F::kSfbCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint16_t* sY = (uint16_t*)(smem + kStages * kStageBytes);
@@ -164,7 +187,7 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   volatile int* abort = &sh->abort;
   const int nk = (int)(K / 256);
   const int64_t col_tiles = N / kM;
-  const int64_t srow = K / 32;  // scale bytes per row
+  const int64_t srow = K / (kNV ? 16 : 32);  // scale bytes per row
 
   if (warp == kTmaWarp) {
     // --------------------------------------------------- TMA producer
@@ -198,23 +221,24 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     // each 128-row group).  The global loads run two stages ahead of the
     // stores (a cursor of its own walks the same (tile, stage) sequence),
     // so their latency overlaps the tensor core's work.
+    using SV = typename std::conditional<kNV, uint4, uint2>::type;  // a row's scales of a stage
+    constexpr int kSPR = F::kScalesPerRow;
     TileWalker pwalk(t_offs, E, kN, col_tiles);
     int64_t ptile = blockIdx.x;
     bool phave = pwalk.seek(ptile);
     int pks = 0;
-    auto issue = [&](uint2 (&wv)[4], uint2 (&xv)[8]) {
+    auto issue = [&](SV (&wv)[4], SV (&xv)[8]) {
       if (!phave) return;
       const int64_t rows = pwalk.row_end - pwalk.row0 < kN ? pwalk.row_end - pwalk.row0 : kN;
-      const uint8_t* wsc = w_scales + (pwalk.expert * N + pwalk.col_tile * kM) * srow + 8 * pks;
-      const uint8_t* xsc = x_scales + pwalk.row0 * srow + 8 * pks;
+      const uint8_t* wsc = w_scales + (pwalk.expert * N + pwalk.col_tile * kM) * srow + kSPR * pks;
+      const uint8_t* xsc = x_scales + pwalk.row0 * srow + kSPR * pks;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        wv[i] = __ldg(reinterpret_cast<const uint2*>(wsc + (lane + 32 * i) * srow));
+        wv[i] = __ldg(reinterpret_cast<const SV*>(wsc + (lane + 32 * i) * srow));
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = lane + 32 * i;
-        xv[i] = r < rows ? __ldg(reinterpret_cast<const uint2*>(xsc + r * srow))
-                         : make_uint2(0u, 0u);
+        xv[i] = r < rows ? __ldg(reinterpret_cast<const SV*>(xsc + r * srow)) : SV{};
       }
       if (++pks == nk) {
         pks = 0;
@@ -222,28 +246,43 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         phave = pwalk.seek(ptile);
       }
     };
-    auto store = [&](int s, const uint2 (&wv)[4], const uint2 (&xv)[8]) {
+    // word b of a row's scales (scales 4b..4b+3) goes to block b; B blocks
+    // are ordered (group 0, block b), (group 1, block b) for b = 0, 1, ...
+    auto words = [](const SV& v, uint32_t (&w)[F::kBlocks]) {
+      if constexpr (kNV) {
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+      } else {
+        w[0] = v.x; w[1] = v.y;
+      }
+    };
+    auto store = [&](int s, const SV (&wv)[4], const SV (&xv)[8]) {
       uint8_t* fa = sSfa(s);
       uint8_t* fb = sSfb(s);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t o = sf_offset(lane + 32 * i);
-        *reinterpret_cast<uint32_t*>(fa + o) = wv[i].x;
-        *reinterpret_cast<uint32_t*>(fa + kSfBlock + o) = wv[i].y;
+        uint32_t w[F::kBlocks];
+        words(wv[i], w);
+#pragma unroll
+        for (int b = 0; b < F::kBlocks; ++b)
+          *reinterpret_cast<uint32_t*>(fa + b * kSfBlock + o) = w[b];
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = lane + 32 * i;
         const uint32_t o = sf_offset(r);
         const int g = r >> 7;  // 128-row group
-        *reinterpret_cast<uint32_t*>(fb + g * kSfBlock + o) = xv[i].x;
-        *reinterpret_cast<uint32_t*>(fb + (2 + g) * kSfBlock + o) = xv[i].y;
+        uint32_t w[F::kBlocks];
+        words(xv[i], w);
+#pragma unroll
+        for (int b = 0; b < F::kBlocks; ++b)
+          *reinterpret_cast<uint32_t*>(fb + (2 * b + g) * kSfBlock + o) = w[b];
       }
       fence_proxy_async_smem();  // visible to tcgen05.cp
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->full[s]);
     };
-    uint2 wa[4], xa[8], wb[4], xb[8];
+    SV wa[4], xa[8], wb[4], xb[8];
     issue(wa, xa);
     issue(wb, xb);
     TileWalker walk(t_offs, E, kN, col_tiles);
@@ -283,25 +322,31 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
           // scales of the stage into TMEM (A: blocks 0,1; B: (group, block)
           // pairs (0,0) (1,0) (0,1) (1,1), 8 columns per block index)
 #pragma unroll
-          for (int b = 0; b < 2; ++b)
+          for (int b = 0; b < F::kBlocks; ++b)
             tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * b,
                                    smem_desc_noswz(smem_addr(sSfa(s) + b * kSfBlock), 128));
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
+          for (int b = 0; b < 2 * F::kBlocks; ++b)
             tmem_cp_32x128b_warpx4(tmem + kSfbCol + 4 * b,
                                    smem_desc_noswz(smem_addr(sSfb(s) + b * kSfBlock), 128));
           const uint64_t adesc = smem_desc_sw128(smem_addr(sA(s)));
           const uint64_t bdesc = smem_desc_sw128(smem_addr(sB(s)));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            // K=64 step kk: 32 bytes into the 128-byte swizzled rows; its
-            // scales are 2kk, 2kk+1: block kk/2, byte 2(kk%2)
-            const uint32_t id = 2u * (kk & 1);
-            const uint32_t blk = kk >> 1;
+            // K=64 step kk: 32 bytes into the 128-byte swizzled rows.  MX:
+            // its scales are 2kk, 2kk+1 (block kk/2, byte 2(kk%2)); NV: its
+            // scales are 4kk..4kk+3 (block kk, the whole word)
+            const uint32_t id = kNV ? 0u : 2u * (kk & 1);
+            const uint32_t blk = kNV ? kk : kk >> 1;
             const uint32_t sfa = (tmem + kSfaCol + 4 * blk) | (id << 30);
             const uint32_t sfb = (tmem + kSfbCol + 8 * blk) | (id << 30);
-            mma_mxf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc_mxf4(kM, n, id, id),
-                        sfa, sfb, (ks | kk) != 0);
+            const uint32_t idesc = idesc_mxf4(kM, n, id, id, !kNV);
+            if constexpr (kNV)
+              mma_nvf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb,
+                          (ks | kk) != 0);
+            else
+              mma_mxf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb,
+                          (ks | kk) != 0);
           }
           mma_commit(&sh->empty[s]);
         }
@@ -324,11 +369,17 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       const int64_t row0 = walk.row0;
       const int64_t rows = walk.row_end - row0 < kN ? walk.row_end - row0 : kN;
       const int col = 32 * warp + lane;  // output feature within the tile's 128
+      // NV: the product of the two per-tensor scales, applied in f32
+      const float gg = kNV ? __fmul_rn(x_global[0], w_global[walk.expert]) : 1.0f;
 #pragma unroll 1
       for (int c = 0; c < (int)((rows + 31) / 32); ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
         tmem_wait_ld();
+        if constexpr (kNV) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gg);
+        }
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
@@ -357,31 +408,50 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   if (threadIdx.x == 0 && *abort && dev_status) atomicExch(dev_status, MXQ_ERR_TIMEOUT);
 }
 
-}  // namespace
-
-int launch_w4a4_grouped_mm(const void* xq, const void* xs, const void* packed, const void* scales,
-                           const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
-                           void* y, int32_t* dev_status, uint64_t wait_limit_ns, cudaStream_t st) {
+template <bool kNV>
+int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* packed,
+                const void* scales, const float* wg, const int32_t* offs, int64_t T, int64_t E,
+                int64_t N, int64_t K, void* y, int32_t* dev_status, uint64_t wait_limit_ns,
+                cudaStream_t st) {
+  using F = W4Fmt<kNV>;
   CUtensorMap xmap, wmap;
   if (!make_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, T, K / 2, K / 2, kKB, kN,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, E * N, K / 2, K / 2, kKB, kM,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return MXQ_ERR_CUDA;
+  auto kernel = w4a4_tc_kernel<kNV>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(w4a4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kSmem);
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F::kSmem);
   });
   if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
   const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
   const int64_t sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
-  w4a4_tc_kernel<<<grid, kThreads, kSmem, st>>>(xmap, wmap, (const uint8_t*)xs,
-                                                (const uint8_t*)scales, offs, T, E, N, K,
-                                                (__nv_bfloat16*)y, dev_status, wait_limit_ns);
+  kernel<<<grid, kThreads, F::kSmem, st>>>(xmap, wmap, (const uint8_t*)xs, (const uint8_t*)scales,
+                                           xg, wg, offs, T, E, N, K, (__nv_bfloat16*)y,
+                                           dev_status, wait_limit_ns);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_w4a4_grouped_mm(const void* xq, const void* xs, const void* packed, const void* scales,
+                           const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
+                           void* y, int32_t* dev_status, uint64_t wait_limit_ns, cudaStream_t st) {
+  return launch_w4a4<false>(xq, xs, nullptr, packed, scales, nullptr, offs, T, E, N, K, y,
+                            dev_status, wait_limit_ns, st);
+}
+
+int launch_nvfp4_w4a4_grouped_mm(const void* xq, const void* xs, const float* xg,
+                                 const void* packed, const void* scales, const float* wg,
+                                 const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
+                                 void* y, int32_t* dev_status, uint64_t wait_limit_ns,
+                                 cudaStream_t st) {
+  return launch_w4a4<true>(xq, xs, xg, packed, scales, wg, offs, T, E, N, K, y, dev_status,
+                           wait_limit_ns, st);
 }
 
 }  // namespace mxq

@@ -182,3 +182,14 @@ def test_w4a4_validation(L):
     assert f(A1, A1, A2, A2, A2, 8, 2, 64, 256, A1, NULL, NULL) == EUNSUP  # N % 128
     assert f(BAD, A1, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
     assert f(A1, A1, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK  # T == 0
+
+
+def test_nvfp4_w4a4_validation(L):
+    f = L.nvfp4_w4a4_grouped_mm
+    assert f(A1, A1, A2, A2, A2, A2, A2, 8, 0, 128, 256, A1, NULL, NULL) == ESHAPE  # E < 1
+    assert f(A1, A1, A2, A2, A2, A2, A2, 8, 2, 128, 40, A1, NULL, NULL) == ESHAPE  # K % 16
+    assert f(A1, A1, A2, A2, A2, NULL, A2, 8, 2, 128, 256, A1, NULL, NULL) == EARG  # w scales
+    assert f(A1, A1, NULL, A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EARG  # x scale
+    assert f(A1, A1, A2, A2, A2, A2, A2, 8, 2, 128, 96, A1, NULL, NULL) == EUNSUP
+    assert f(BAD, A1, A2, A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
+    assert f(A1, A1, A2, A2, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK

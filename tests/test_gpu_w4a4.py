@@ -108,3 +108,50 @@ def test_w4a4_bad_offs_and_unsupported_shapes():
     with pytest.raises(mxq.MxqError) as ei:
         mxq.w4a4_grouped_mm(x2.to(DEV), p2.to(DEV), s2.to(DEV), o2.to(DEV))
     assert ei.value.status == -4
+
+
+# ---------------------------------------------------------------- NVFP4
+
+def nv_weights(E, N, K, seed=41):
+    """Random NVFP4 weight storage from the seeded generator: code bytes,
+    E4M3 block-scale bytes in [0x30, 0x40] (0.5 .. 2.0) and per-expert
+    global scales."""
+    packed = gen.random_bytes(E * N * (K // 2), gen.seed_for(seed, 1)).view(E, N, K // 2)
+    u = gen.uniform(gen.seed_for(seed, 2), E * N * (K // 16))
+    bs = (u * 17).floor().clamp_(max=16).to(torch.uint8).add_(0x30).view(E, N, K // 16)
+    gw = torch.tensor([0.01 * (1 + e / E) for e in range(E)], dtype=torch.float32)
+    return packed, bs, gw
+
+
+def nv_check(counts, N, K, rows=None, seed=41):
+    E = len(counts)
+    offs = torch.tensor(np.cumsum(counts), dtype=torch.int32)
+    T = int(offs[-1])
+    packed, bs, gw = nv_weights(E, N, K, seed)
+    x = gen.normal_bf16(gen.seed_for(seed, 3), (T, K))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = mxq.nvfp4_w4a4_grouped_mm(x.to(DEV), packed.to(DEV), bs.to(DEV), gw.to(DEV),
+                                  offs.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    ref = oracle.nvfp4_w4a4_grouped_mm(bits(x), packed.numpy(), bs.numpy(), gw.numpy(),
+                                       offs.numpy(), rows)
+    err = error(oracle.decode(bits(y)[rows], "bf16"), ref)
+    assert err <= TOL, err
+
+
+def test_nvfp4_w4a4_small_ragged():
+    nv_check([200, 0, 37, 275], 256, 512)
+
+
+def test_nvfp4_w4a4_many_small_experts():
+    nv_check([int(c) for c in np.random.RandomState(7).randint(0, 41, size=24)], 128, 256)
+    nv_check([300], 384, 768)
+
+
+def test_nvfp4_w4a4_full_size_sampled():
+    T, E, N, K = 32768, 32, 2048, 7168
+    counts = gen.expert_counts(T, E).numpy()
+    rows = [0, 1, 255, 256, int(np.cumsum(counts)[0]), 20000, T - 1]
+    nv_check(list(counts), N, K, rows=rows)
