@@ -1,16 +1,18 @@
-// W4A4 grouped GEMM on the block-scaled tensor cores (sm_100a): both the
-// expert weights and the activations are MXFP4 (E2M1 codes, two per byte,
-// one E8M0 scale per 32 K), multiplied by tcgen05.mma kind::mxf4 with the
-// scales applied inside the tensor core ("NVIDIA Model Optimizer: from
-// mtq.quantize to a 4.95-bit DeepSeek-R1", section on W4A4 NVFP4 on FP4
-// tensor cores; here with the MX format of
-// "nemo_automodel.components.quantization.mxfp4").
-//
-//   y[t, n] = sum_k xq[t, k] W_e[n, k]   for t in expert e's rows
-//
-// xq is the activation after mx_quantize (its packed bytes and scales are
-// the inputs), so every product of codes is exact and the tensor core only
-// rounds the f32 accumulation; y is rounded once to bf16.
+// W4A4 grouped GEMMs on the block-scaled tensor cores (sm_100a): both the
+// expert weights and the activations are 4-bit E2M1 codes (two per byte)
+// with block scales, multiplied by tcgen05.mma with the scales applied
+// inside the tensor core ("NVIDIA Model Optimizer: from mtq.quantize to a
+// 4.95-bit DeepSeek-R1", section on W4A4 NVFP4 on FP4 tensor cores).  Two
+// formats share the kernel:
+//   MXFP4: one E8M0 scale per 32 K ("nemo_automodel.components.quantization.
+//          mxfp4"), kind::mxf4, y = sum_k xq[t, k] W_e[n, k];
+//   NVFP4: one UE4M3 scale per 16 K plus a per-tensor f32 scale for the
+//          activations and one per expert weight ("NVFP4 in the code: two
+//          scales and a nibble"), kind::mxf4nvf4, y = g_x g_w[e] sum_k ...
+// The activations come quantized (mx_quantize / nvfp4_quantize), so every
+// product of codes and block scales is exact and the tensor core only
+// rounds the f32 accumulation; y is rounded once to bf16 (NVFP4: after the
+// f32 product with g_x g_w[e]).
 //
 // Mapping (persistent, one CTA per SM, seven warps):
 //   D[m, j] (f32, TMEM) += A[m, k] (weights, smem) * B[j, k] (tokens, smem)
@@ -18,14 +20,14 @@
 // tokens of the expert and k the reduction index, 256 per pipeline stage
 // (128 bytes of codes per row: one 128-byte-swizzled TMA row).
 //   * warp 4 (one lane) TMA-loads both code tiles of a stage;
-//   * warp 5 gathers the stage's scale bytes (8 per row: 128 weight rows
-//     and 256 token rows) from the row-major [rows, K/32] scale arrays and
-//     writes them into the tensor core's scale layout in shared memory:
-//     blocks of 128 rows x 4 scales, row r at byte 16 (r % 32) + 4 (r / 32)
-//     + the scale's index;
+//   * warp 5 gathers the stage's scale bytes (8 or 16 per row: 128 weight
+//     rows and 256 token rows) from the row-major [rows, K/32 or K/16] scale
+//     arrays and writes them into the tensor core's scale layout in shared
+//     memory: blocks of 128 rows x 4 scales, row r at byte 16 (r % 32) +
+//     4 (r / 32) + the scale's index;
 //   * warp 6 (one lane) copies those blocks into TMEM (tcgen05.cp, 32 lanes
 //     x 128 bits, replicated to the four lane quarters) and issues four
-//     K=64 MMAs per stage, each selecting its pair of scales by byte id;
+//     K=64 MMAs per stage, each selecting its scales by block and byte id;
 //   * warps 0-3 drain D, round to bf16, stage the tile in shared memory and
 //     store the expert's rows.
 // Every mbarrier wait is bounded: on a time-out the CTA stops all roles,
