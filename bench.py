@@ -519,6 +519,62 @@ def cpu_baseline(budget_s):
                        "GEMM: 8 rows x 256 outputs x 7168" % (n1, n2, n3, t1 + t2 + t3))}
 
 
+def run_sweep(args):
+    """Bandwidth sweep over row counts of the mixed-block workload x bf16
+    [R, 7168] (normal, subnormal-range, zero and single-spike 32-blocks):
+    mx_quantize, mx_dequantize and quantize_cache in the three formats, device
+    time per call (CUDA events, median of 5 after 2 warm-up calls; L2 is
+    flushed before each timed call).  Prints one JSON line."""
+    import torch
+
+    import nvfp4_quantization_amax_b200 as mxq
+    import synthetic as gen
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    C = 7168
+    r_max = 1 << min(args.sweep_max_log2, 21)
+    x = gen.mixed_blocks(r_max, C, device=dev)
+    out = torch.empty_like(x)
+    packed = torch.empty((r_max, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((r_max, C // 32), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows_out = []
+    logs = list(range(10, min(args.sweep_max_log2, 20) + 1, 2))
+    if args.sweep_max_log2 >= 21:
+        logs.append(21)
+    for lg in logs:
+        R = 1 << lg
+        xr, outr, pr, sr = x[:R], out[:R], packed[:R], scales[:R]
+        mxq.mx_quantize(xr, pr, sr)
+        n = R * C
+        calls = {
+            "mx_quantize": (lambda: mxq.mx_quantize(xr, pr, sr), n * 2 + n // 2 + n // 32),
+            "mx_dequantize": (lambda: mxq.mx_dequantize(pr, sr, torch.bfloat16, outr),
+                              n // 2 + n // 32 + n * 2),
+        }
+        for f, b in CACHE_RUNS:
+            calls["qc_" + f] = ((lambda f=f, b=b: mxq.quantize_cache(xr, f, b, outr)), n * 4)
+        row = {"rows": R}
+        for name, (fn, nbytes) in calls.items():
+            for _ in range(2):
+                fn()
+            ts = []
+            for _ in range(5):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = sorted(ts)[2]
+            row[name] = {"ms": round(ms, 4), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+        rows_out.append(row)
+    print(json.dumps({"sweep": "mixed blocks bf16 [R, 7168]", "peak_hbm_gbs":
+                      load_peaks()[0]["hbm_gbs"], "rows": rows_out}), flush=True)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -546,12 +602,18 @@ def main():
     ap.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the step: the mixed-block bandwidth sweep over row counts")
+    ap.add_argument("--sweep-max-log2", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    if args.impl == "reference":
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_gpu(args, rank, world)

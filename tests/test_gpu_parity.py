@@ -391,3 +391,18 @@ def test_grouped_mm_small_remainders(transpose_w):
     # ragged tail the CTA-pair tiling meets
     counts = [257, 287, 288, 289, 319, 320, 321, 576, 600, 64, 1, 0, 512]
     check_gemm(counts, 256, 512, transpose_w)
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_scale_rows_not_16_byte_multiples(transpose_w):
+    # K = 768: 24 scale bytes per weight row, so the weight tiles are staged
+    # by TMA but their scale bytes are read from global memory
+    check_gemm([130, 300, 90], N=256, K=768, transpose_w=transpose_w)
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_more_experts_than_the_offs_cache(transpose_w):
+    # 300 experts (more than the shared-memory copy of offs holds): the tile
+    # walks read offs from global memory
+    counts = [int(c) for c in np.random.RandomState(3).randint(0, 9, size=300)]
+    check_gemm(counts, N=256, K=256, transpose_w=transpose_w)
