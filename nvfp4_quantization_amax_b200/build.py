@@ -8,6 +8,7 @@ Every .cu under csrc/ is compiled for sm_100a only
 nvfp4_quantization_amax_b200/libmxq.so next to this file.  Object files go to
 _build/ beside it.  nvcc cross-compiles, so no GPU is needed to build.
 """
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -35,16 +36,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_dep = max(os.path.getmtime(p) for p in _deps())
-    objs = []
+    objs, jobs = [], []
     for src in sources:
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         stale = (force or not os.path.exists(obj) or
                  os.path.getmtime(obj) < max(os.path.getmtime(src), newest_dep))
         if stale:
-            cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + \
-                  ["-c", src, "-o", obj]
-            subprocess.check_call(cmd)
+            jobs.append([NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) +
+                        ["-c", src, "-o", obj])
+    # translation units compile independently: one nvcc per source, in parallel
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
+        for f in [ex.submit(subprocess.check_call, cmd) for cmd in jobs]:
+            f.result()
     if force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB)
                                                 for o in objs):
         tmp = LIB + ".tmp%d" % os.getpid()
