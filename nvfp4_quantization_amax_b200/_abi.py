@@ -84,15 +84,19 @@ def _stream(dev):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
-def _to_device(t):
-    """(device tensor, was_on_host).  Host tensors are moved to the current
-    CUDA device; pinned ones without blocking the host."""
+def _to_device(t, dev=None):
+    """(device tensor, was_on_host) for an input.  A host tensor is moved to
+    `dev` (default: the current CUDA device), a pinned one without blocking
+    the host; a CUDA tensor must already be on `dev`."""
     if t.is_cuda:
+        if dev is not None and t.device != dev:
+            raise ValueError("input on %s, the call runs on %s" % (t.device, dev))
         return t, False
     if not torch.cuda.is_available():
         raise RuntimeError("no CUDA device: libmxq runs only on the GPU")
-    return t.to(torch.device("cuda", torch.cuda.current_device()),
-                non_blocking=t.is_pinned()), True
+    if dev is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return t.to(dev, non_blocking=t.is_pinned()), True
 
 
 def _to_host(t):
@@ -100,6 +104,55 @@ def _to_host(t):
     out.copy_(t, non_blocking=True)
     torch.cuda.current_stream(t.device).synchronize()
     return out
+
+
+def _out(t, shape, dtype, dev, name):
+    """(device buffer, host target) for an output of `shape` and `dtype` of
+    a call that runs on `dev`.  None: a new device tensor.  A contiguous
+    tensor of that dtype and element count on `dev`: itself.  The same on
+    the host: a new device tensor, copied into it by _result.  Anything else
+    raises before a launch, so no kernel ever writes outside a buffer."""
+    shape = tuple(int(v) for v in shape)
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=dev), None
+    n = 1
+    for v in shape:
+        n *= v
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, not %s" % (name, dtype, t.dtype))
+    if t.numel() != n:
+        raise ValueError("%s must hold %d elements (shape %s), not %d"
+                         % (name, n, list(shape), t.numel()))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.is_cuda:
+        if t.device != dev:
+            raise ValueError("%s is on %s, the call runs on %s" % (name, t.device, dev))
+        return t, None
+    return torch.empty(shape, dtype=dtype, device=dev).view(t.shape), t
+
+
+def _result(buf, target, to_host):
+    """What the caller gets back for one output: the host tensor it passed
+    (now filled); a pinned host copy when its inputs came from the host;
+    else the device buffer."""
+    if target is not None:
+        target.copy_(buf, non_blocking=target.is_pinned())
+        torch.cuda.current_stream(buf.device).synchronize()
+        return target
+    return _to_host(buf) if to_host else buf
+
+
+def _device_word(t, dtype, min_numel, dev, name):
+    """Pointer of an optional device-side scratch or status buffer."""
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_cuda or t.device != dev:
+        raise ValueError("%s must be a tensor on %s" % (name, dev))
+    if t.dtype != dtype or t.numel() < min_numel or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous %s tensor of at least %d elements"
+                         % (name, dtype, min_numel))
+    return _ptr(t)
 
 
 def _ptr(t):
@@ -119,16 +172,13 @@ def mx_quantize(x, packed=None, scales=None):
     x = x.contiguous()
     K = x.shape[-1]
     rows = x.numel() // K if K else 0
-    if packed is None:
-        packed = torch.empty(x.shape[:-1] + (K // 2,), dtype=torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty(x.shape[:-1] + (K // 32,), dtype=torch.uint8, device=x.device)
+    lead = tuple(x.shape[:-1])
+    packed, hp = _out(packed, lead + (K // 2,), torch.uint8, x.device, "packed")
+    scales, hs = _out(scales, lead + (K // 32,), torch.uint8, x.device, "scales")
     rc = lib().mx_quantize(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed), _ptr(scales),
                            _stream(x.device))
     _check(rc, "mx_quantize")
-    if host:
-        return _to_host(packed), _to_host(scales)
-    return packed, scales
+    return _result(packed, hp, host), _result(scales, hs, host)
 
 
 def mx_dequantize(packed, scales, dtype=torch.bfloat16, out=None):
@@ -136,7 +186,7 @@ def mx_dequantize(packed, scales, dtype=torch.bfloat16, out=None):
     if dtype not in _DTYPES:
         raise TypeError("mx_dequantize: unsupported dtype %s" % dtype)
     packed, host = _to_device(packed)
-    scales, _ = _to_device(scales)
+    scales, _ = _to_device(scales, packed.device)
     packed = packed.contiguous()
     scales = scales.contiguous()
     Kh = packed.shape[-1]
@@ -144,12 +194,11 @@ def mx_dequantize(packed, scales, dtype=torch.bfloat16, out=None):
     rows = packed.numel() // Kh if Kh else 0
     if scales.numel() != rows * (K // 32):
         raise ValueError("mx_dequantize: scales must have shape [..., K/32]")
-    if out is None:
-        out = torch.empty(packed.shape[:-1] + (K,), dtype=dtype, device=packed.device)
+    out, ho = _out(out, tuple(packed.shape[:-1]) + (K,), dtype, packed.device, "out")
     rc = lib().mx_dequantize(_ptr(packed), _ptr(scales), rows, K, _ptr(out), _DTYPES[dtype],
                              _stream(packed.device))
     _check(rc, "mx_dequantize")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 def quantize_cache(values, format, block_size, out=None):
@@ -163,12 +212,11 @@ def quantize_cache(values, format, block_size, out=None):
     values = values.contiguous()
     C = values.shape[-1] if values.dim() else 1
     rows = values.numel() // C if C else 0
-    if out is None:
-        out = torch.empty_like(values)
+    out, ho = _out(out, tuple(values.shape), values.dtype, values.device, "out")
     rc = lib().quantize_cache(_ptr(values), _ptr(out), _DTYPES[values.dtype], rows, C,
                               _FORMATS[format], int(block_size), _stream(values.device))
     _check(rc, "quantize_cache")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 def quantize_cache_packed(values, format, block_size, codes=None, scales=None):
@@ -189,17 +237,14 @@ def quantize_cache_packed(values, format, block_size, codes=None, scales=None):
     B = int(block_size)
     lead = tuple(values.shape[:-1])
     dev = values.device
-    if codes is None:
-        codes = torch.empty(lead + (C if format == "fp8" else C // 2,), dtype=torch.uint8,
-                            device=dev)
-    if scales is None:
-        scales = torch.empty(lead + (C // B if B > 0 else 0,), dtype=torch.uint8, device=dev)
+    if B < 1:
+        raise ValueError("quantize_cache_packed: block_size must be >= 1")
+    codes, hc = _out(codes, lead + (C if format == "fp8" else C // 2,), torch.uint8, dev, "codes")
+    scales, hs = _out(scales, lead + (C // B,), torch.uint8, dev, "scales")
     rc = lib().quantize_cache_packed(_ptr(values), _DTYPES[values.dtype], rows, C,
                                      _FORMATS[format], B, _ptr(codes), _ptr(scales), _stream(dev))
     _check(rc, "quantize_cache_packed")
-    if host:
-        return _to_host(codes), _to_host(scales)
-    return codes, scales
+    return _result(codes, hc, host), _result(scales, hs, host)
 
 
 def dequantize_cache_packed(codes, scales, format, block_size, dtype=torch.bfloat16, out=None):
@@ -209,19 +254,18 @@ def dequantize_cache_packed(codes, scales, format, block_size, dtype=torch.bfloa
     if format not in _FORMATS:
         raise ValueError("dequantize_cache_packed: format must be one of %s" % sorted(_FORMATS))
     codes, host = _to_device(codes)
-    scales, _ = _to_device(scales)
+    scales, _ = _to_device(scales, codes.device)
     codes, scales = codes.contiguous(), scales.contiguous()
     B = int(block_size)
     C = scales.shape[-1] * B
     rows = scales.numel() // scales.shape[-1] if scales.shape[-1] else 0
     if codes.numel() != rows * (C if format == "fp8" else C // 2):
         raise ValueError("dequantize_cache_packed: codes do not match the scales' shape")
-    if out is None:
-        out = torch.empty(tuple(scales.shape[:-1]) + (C,), dtype=dtype, device=codes.device)
+    out, ho = _out(out, tuple(scales.shape[:-1]) + (C,), dtype, codes.device, "out")
     rc = lib().dequantize_cache_packed(_ptr(codes), _ptr(scales), rows, C, _FORMATS[format], B,
                                        _ptr(out), _DTYPES[dtype], _stream(codes.device))
     _check(rc, "dequantize_cache_packed")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 class CacheQuantization(torch.autograd.Function):
@@ -250,9 +294,9 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
     if a.dtype != torch.bfloat16:
         raise TypeError("mxfp4_grouped_mm: activations must be bf16")
     a, host = _to_device(a)
-    packed, _ = _to_device(packed)
-    scales, _ = _to_device(scales)
-    offs, _ = _to_device(offs)
+    packed, _ = _to_device(packed, a.device)
+    scales, _ = _to_device(scales, a.device)
+    offs, _ = _to_device(offs, a.device)
     a, packed, scales = a.contiguous(), packed.contiguous(), scales.contiguous()
     offs = offs.to(torch.int32).contiguous()
     E, N, Kh = packed.shape
@@ -263,13 +307,12 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
         raise ValueError("mxfp4_grouped_mm: a must be [T, %d]" % kin)
     if tuple(scales.shape) != (E, N, K // 32) or offs.numel() != E:
         raise ValueError("mxfp4_grouped_mm: scales [E, N, K/32] and offs [E] expected")
-    if out is None:
-        out = torch.empty((T, nout), dtype=torch.bfloat16, device=a.device)
-    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    out, ho = _out(out, (T, nout), torch.bfloat16, a.device, "out")
+    st = _device_word(status, torch.int32, 1, a.device, "status")
     rc = lib().mxfp4_grouped_mm(_ptr(a), _ptr(packed), _ptr(scales), _ptr(offs), T, E, N, K,
                                 1 if transpose_w else 0, _ptr(out), st, _stream(a.device))
     _check(rc, "mxfp4_grouped_mm")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=None,
@@ -282,9 +325,9 @@ def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=Non
     if x.dtype != torch.bfloat16:
         raise TypeError("w4a4_grouped_mm: activations must be bf16")
     x, host = _to_device(x)
-    packed, _ = _to_device(packed)
-    scales, _ = _to_device(scales)
-    offs, _ = _to_device(offs)
+    packed, _ = _to_device(packed, x.device)
+    scales, _ = _to_device(scales, x.device)
+    offs, _ = _to_device(offs, x.device)
     x, packed, scales = x.contiguous(), packed.contiguous(), scales.contiguous()
     offs = offs.to(torch.int32).contiguous()
     E, N, Kh = packed.shape
@@ -294,14 +337,16 @@ def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=Non
         raise ValueError("w4a4_grouped_mm: x must be [T, %d]" % K)
     if tuple(scales.shape) != (E, N, K // 32) or offs.numel() != E:
         raise ValueError("w4a4_grouped_mm: scales [E, N, K/32] and offs [E] expected")
+    for t, name in ((x_packed, "x_packed"), (x_scales, "x_scales")):
+        if t is not None and not (t.is_cuda and t.device == x.device):
+            raise ValueError("w4a4_grouped_mm: %s must be a tensor on %s" % (name, x.device))
     xq, xs = mx_quantize(x, x_packed, x_scales)
-    if out is None:
-        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
-    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    out, ho = _out(out, (T, N), torch.bfloat16, x.device, "out")
+    st = _device_word(status, torch.int32, 1, x.device, "status")
     rc = lib().mxfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(packed), _ptr(scales), _ptr(offs),
                                      T, E, N, K, _ptr(out), st, _stream(x.device))
     _check(rc, "mxfp4_w4a4_grouped_mm")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=None,
@@ -314,10 +359,10 @@ def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=No
     if x.dtype != torch.bfloat16:
         raise TypeError("nvfp4_w4a4_grouped_mm: activations must be bf16")
     x, host = _to_device(x)
-    packed, _ = _to_device(packed)
-    block_scales, _ = _to_device(block_scales)
-    w_global_scales, _ = _to_device(w_global_scales)
-    offs, _ = _to_device(offs)
+    packed, _ = _to_device(packed, x.device)
+    block_scales, _ = _to_device(block_scales, x.device)
+    w_global_scales, _ = _to_device(w_global_scales, x.device)
+    offs, _ = _to_device(offs, x.device)
     x, packed, block_scales = x.contiguous(), packed.contiguous(), block_scales.contiguous()
     w_global_scales = w_global_scales.to(torch.float32).contiguous()
     offs = offs.to(torch.int32).contiguous()
@@ -331,14 +376,13 @@ def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=No
         raise ValueError("nvfp4_w4a4_grouped_mm: block_scales [E, N, K/16], global scales [E] "
                          "and offs [E] expected")
     xq, xs, xg = nvfp4_quantize(x)
-    if out is None:
-        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
-    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    out, ho = _out(out, (T, N), torch.bfloat16, x.device, "out")
+    st = _device_word(status, torch.int32, 1, x.device, "status")
     rc = lib().nvfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(xg), _ptr(packed),
                                      _ptr(block_scales), _ptr(w_global_scales), _ptr(offs),
                                      T, E, N, K, _ptr(out), st, _stream(x.device))
     _check(rc, "nvfp4_w4a4_grouped_mm")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
 
 
 NVFP4_WORKSPACE_BYTES = 16
@@ -363,21 +407,19 @@ def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspa
     K = x.shape[-1]
     rows = x.numel() // K if K else 0
     dev = x.device
-    if packed is None:
-        packed = torch.empty(x.shape[:-1] + (K // 2,), dtype=torch.uint8, device=dev)
-    if block_scales is None:
-        block_scales = torch.empty(x.shape[:-1] + (K // 16,), dtype=torch.uint8, device=dev)
-    if global_scale is None:
-        global_scale = torch.empty(1, dtype=torch.float32, device=dev)
+    lead = tuple(x.shape[:-1])
+    packed, hp = _out(packed, lead + (K // 2,), torch.uint8, dev, "packed")
+    block_scales, hb = _out(block_scales, lead + (K // 16,), torch.uint8, dev, "block_scales")
+    global_scale, hg = _out(global_scale, (1,), torch.float32, dev, "global_scale")
     if workspace is None:
         workspace = torch.empty(NVFP4_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    ws = _device_word(workspace, torch.uint8, NVFP4_WORKSPACE_BYTES, dev, "workspace")
     fn = lib().nvfp4_quantize if rule == "max" else lib().nvfp4_quantize_mse
     rc = fn(_ptr(x), _DTYPES[x.dtype], rows, K, _ptr(packed), _ptr(block_scales),
-            _ptr(global_scale), _ptr(workspace), _stream(dev))
+            _ptr(global_scale), ws, _stream(dev))
     _check(rc, "nvfp4_quantize" if rule == "max" else "nvfp4_quantize_mse")
-    if host:
-        return _to_host(packed), _to_host(block_scales), _to_host(global_scale)
-    return packed, block_scales, global_scale
+    return (_result(packed, hp, host), _result(block_scales, hb, host),
+            _result(global_scale, hg, host))
 
 
 def nvfp4_dequantize(packed, block_scales, global_scale, dtype=torch.bfloat16, out=None):
@@ -385,8 +427,8 @@ def nvfp4_dequantize(packed, block_scales, global_scale, dtype=torch.bfloat16, o
     if dtype not in _DTYPES:
         raise TypeError("nvfp4_dequantize: unsupported dtype %s" % dtype)
     packed, host = _to_device(packed)
-    block_scales, _ = _to_device(block_scales)
-    global_scale, _ = _to_device(global_scale)
+    block_scales, _ = _to_device(block_scales, packed.device)
+    global_scale, _ = _to_device(global_scale, packed.device)
     packed, block_scales = packed.contiguous(), block_scales.contiguous()
     global_scale = global_scale.to(torch.float32).contiguous()
     Kh = packed.shape[-1]
@@ -394,9 +436,10 @@ def nvfp4_dequantize(packed, block_scales, global_scale, dtype=torch.bfloat16, o
     rows = packed.numel() // Kh if Kh else 0
     if block_scales.numel() != rows * (K // 16):
         raise ValueError("nvfp4_dequantize: block_scales must have shape [..., K/16]")
-    if out is None:
-        out = torch.empty(packed.shape[:-1] + (K,), dtype=dtype, device=packed.device)
+    if global_scale.numel() < 1:
+        raise ValueError("nvfp4_dequantize: global_scale must hold one float32")
+    out, ho = _out(out, tuple(packed.shape[:-1]) + (K,), dtype, packed.device, "out")
     rc = lib().nvfp4_dequantize(_ptr(packed), _ptr(block_scales), _ptr(global_scale), rows, K,
                                 _ptr(out), _DTYPES[dtype], _stream(packed.device))
     _check(rc, "nvfp4_dequantize")
-    return _to_host(out) if host else out
+    return _result(out, ho, host)
