@@ -4,7 +4,9 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "mxq.h"
 #include "mxq_launch.h"
@@ -24,6 +26,32 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+int resident_ctas(const void* kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int, size_t>, int> cached;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const auto key = std::make_tuple(kernel, dev, threads, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  const auto it = cached.find(key);
+  if (it != cached.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+      n < 1) {
+    (void)cudaGetLastError();  // not sticky; keep it out of the launch checks
+    n = 1;
+  }
+  cached[key] = n;
+  return n;
+}
+
+int wave_grid(const void* kernel, int threads, int64_t n_units, int64_t per_cta) {
+  int64_t need = (n_units + per_cta - 1) / per_cta;
+  const int64_t wave = (int64_t)num_sms() * resident_ctas(kernel, threads, 0);
+  if (need > wave) need = wave;
+  return (int)(need < 1 ? 1 : need);
 }
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }

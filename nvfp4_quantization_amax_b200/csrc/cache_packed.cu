@@ -263,21 +263,21 @@ unpack_cache_general_kernel(const uint8_t* __restrict__ codes, const uint8_t* __
   }
 }
 
-int grid_over(int64_t n_units, int per_block) {
-  int64_t need = (n_units + per_block - 1) / per_block;
-  const int64_t cap = (int64_t)num_sms() * (2048 / kThreads);
-  if (need > cap) need = cap;
-  return (int)(need < 1 ? 1 : need);
+template <class Kernel>
+int grid_over(Kernel kernel, int64_t n_units, int per_block) {
+  return wave_grid((const void*)kernel, kThreads, n_units, per_block);
 }
 
 template <int DT, int FMT, int LPB>
 void launch_fast(const void* in, void* codes, uint8_t* scales, void* out, bool pack,
                  int64_t n_items, cudaStream_t st) {
-  const int grid = grid_over(n_items, kThreads * kUnroll);
+  const int per = kThreads * kUnroll;
   if (pack)
-    pack_cache_kernel<DT, FMT, LPB><<<grid, kThreads, 0, st>>>(in, codes, scales, n_items);
+    pack_cache_kernel<DT, FMT, LPB><<<grid_over(pack_cache_kernel<DT, FMT, LPB>, n_items, per),
+                                      kThreads, 0, st>>>(in, codes, scales, n_items);
   else
-    unpack_cache_kernel<DT, FMT, LPB><<<grid, kThreads, 0, st>>>(codes, scales, out, n_items);
+    unpack_cache_kernel<DT, FMT, LPB><<<grid_over(unpack_cache_kernel<DT, FMT, LPB>, n_items, per),
+                                        kThreads, 0, st>>>(codes, scales, out, n_items);
 }
 
 template <int DT, int FMT>
@@ -296,13 +296,14 @@ void launch_fmt(const void* in, void* codes, uint8_t* scales, void* out, bool pa
     return;
   }
   const int64_t n_groups = rows * (C / B);
-  const int grid = grid_over(n_groups, kThreads);
   if (pack)
-    pack_cache_general_kernel<DT, FMT><<<grid, kThreads, 0, st>>>(in, (uint8_t*)codes, scales,
-                                                                  n_groups, B);
+    pack_cache_general_kernel<DT, FMT>
+        <<<grid_over(pack_cache_general_kernel<DT, FMT>, n_groups, kThreads), kThreads, 0, st>>>(
+            in, (uint8_t*)codes, scales, n_groups, B);
   else
-    unpack_cache_general_kernel<DT, FMT><<<grid, kThreads, 0, st>>>((const uint8_t*)codes,
-                                                                    scales, out, n_groups, B);
+    unpack_cache_general_kernel<DT, FMT>
+        <<<grid_over(unpack_cache_general_kernel<DT, FMT>, n_groups, kThreads), kThreads, 0, st>>>(
+            (const uint8_t*)codes, scales, out, n_groups, B);
 }
 
 template <int DT>

@@ -298,51 +298,72 @@ quantize_cache_general_kernel(const void* __restrict__ in, void* __restrict__ ou
 
 // ------------------------------------------------------------ launchers
 
-static int grid_for(int64_t n_units, int per_block) {
-  int64_t need = (n_units + per_block - 1) / per_block;
-  int64_t cap = (int64_t)num_sms() * (2048 / kThreads);
-  if (need > cap) need = cap;
-  return (int)(need < 1 ? 1 : need);
+template <class Kernel>
+static int grid_for(Kernel kernel, int64_t n_units, int per_block) {
+  return wave_grid((const void*)kernel, kThreads, n_units, per_block);
 }
 
 int launch_mx_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed, void* scales,
                        cudaStream_t st) {
-  int64_t n_items = rows * (K / 8);
-  int grid = grid_for(n_items, kThreads * kUnroll);
+  const int64_t n_items = rows * (K / 8);
+  const int per = kThreads * kUnroll;
   auto* p = (uint32_t*)packed;
   auto* s = (uint8_t*)scales;
   switch (dt) {
-    case kBF16: mx_quantize_kernel<kBF16><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
-    case kF16: mx_quantize_kernel<kF16><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
-    default: mx_quantize_kernel<kF32><<<grid, kThreads, 0, st>>>(x, p, s, n_items); break;
+    case kBF16:
+      mx_quantize_kernel<kBF16><<<grid_for(mx_quantize_kernel<kBF16>, n_items, per), kThreads, 0,
+                                  st>>>(x, p, s, n_items);
+      break;
+    case kF16:
+      mx_quantize_kernel<kF16><<<grid_for(mx_quantize_kernel<kF16>, n_items, per), kThreads, 0,
+                                 st>>>(x, p, s, n_items);
+      break;
+    default:
+      mx_quantize_kernel<kF32><<<grid_for(mx_quantize_kernel<kF32>, n_items, per), kThreads, 0,
+                                 st>>>(x, p, s, n_items);
+      break;
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 int launch_mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t K, void* out,
                          int dt, cudaStream_t st) {
-  int64_t n_items = rows * (K / 8);
-  int grid = grid_for(n_items, kThreads * kUnroll);
+  const int64_t n_items = rows * (K / 8);
+  const int per = kThreads * kUnroll;
   auto* p = (const uint32_t*)packed;
   auto* s = (const uint8_t*)scales;
   switch (dt) {
-    case kBF16: mx_dequantize_kernel<kBF16><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
-    case kF16: mx_dequantize_kernel<kF16><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
-    default: mx_dequantize_kernel<kF32><<<grid, kThreads, 0, st>>>(p, s, out, n_items); break;
+    case kBF16:
+      mx_dequantize_kernel<kBF16><<<grid_for(mx_dequantize_kernel<kBF16>, n_items, per), kThreads,
+                                    0, st>>>(p, s, out, n_items);
+      break;
+    case kF16:
+      mx_dequantize_kernel<kF16><<<grid_for(mx_dequantize_kernel<kF16>, n_items, per), kThreads,
+                                   0, st>>>(p, s, out, n_items);
+      break;
+    default:
+      mx_dequantize_kernel<kF32><<<grid_for(mx_dequantize_kernel<kF32>, n_items, per), kThreads,
+                                   0, st>>>(p, s, out, n_items);
+      break;
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+template <int DT, int FMT, int LPB>
+static void launch_cache_lpb(const void* in, void* out, int64_t n_items, cudaStream_t st) {
+  const int grid = grid_for(quantize_cache_kernel<DT, FMT, LPB>, n_items, kThreads * kUnroll);
+  quantize_cache_kernel<DT, FMT, LPB><<<grid, kThreads, 0, st>>>(in, out, n_items);
+}
+
 template <int DT, int FMT>
 static void launch_cache_fast(const void* in, void* out, int64_t n_items, int lpb, cudaStream_t st) {
-  int grid = grid_for(n_items, kThreads * kUnroll);
   switch (lpb) {
-    case 1: quantize_cache_kernel<DT, FMT, 1><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
-    case 2: quantize_cache_kernel<DT, FMT, 2><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
-    case 4: quantize_cache_kernel<DT, FMT, 4><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
-    case 8: quantize_cache_kernel<DT, FMT, 8><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
-    case 16: quantize_cache_kernel<DT, FMT, 16><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
-    default: quantize_cache_kernel<DT, FMT, 32><<<grid, kThreads, 0, st>>>(in, out, n_items); break;
+    case 1: launch_cache_lpb<DT, FMT, 1>(in, out, n_items, st); break;
+    case 2: launch_cache_lpb<DT, FMT, 2>(in, out, n_items, st); break;
+    case 4: launch_cache_lpb<DT, FMT, 4>(in, out, n_items, st); break;
+    case 8: launch_cache_lpb<DT, FMT, 8>(in, out, n_items, st); break;
+    case 16: launch_cache_lpb<DT, FMT, 16>(in, out, n_items, st); break;
+    default: launch_cache_lpb<DT, FMT, 32>(in, out, n_items, st); break;
   }
 }
 
@@ -353,8 +374,8 @@ static void launch_cache(const void* in, void* out, int64_t rows, int64_t C, int
     launch_cache_fast<DT, FMT>(in, out, rows * (C / 8), B / 8, st);
   } else {
     int64_t n_groups = rows * ((C + B - 1) / B);
-    quantize_cache_general_kernel<DT, FMT><<<grid_for(n_groups, kThreads), kThreads, 0, st>>>(
-        in, out, rows, C, B);
+    const int grid = grid_for(quantize_cache_general_kernel<DT, FMT>, n_groups, kThreads);
+    quantize_cache_general_kernel<DT, FMT><<<grid, kThreads, 0, st>>>(in, out, rows, C, B);
   }
 }
 

@@ -145,7 +145,37 @@ __device__ __forceinline__ uint32_t e2m1x2_quot(float a, float b, float d, float
   return e2m1x2(__fdiv_rn(a, d), __fdiv_rn(b, d));
 }
 
-// Whether e2m1x2_quot may be used with divisor d.
+// E2M1 codes of the eight binary32 quotients w_j / d by IEEE division
+// (element 2j in the low nibble of byte j).  Out of line: it is the rare
+// path of e2m1x8_quot.
+static __device__ __noinline__ uint32_t e2m1x8_div(float w0, float w1, float w2, float w3,
+                                                   float w4, float w5, float w6, float w7,
+                                                   float d) {
+  return e2m1x2(__fdiv_rn(w0, d), __fdiv_rn(w1, d)) |
+         (e2m1x2(__fdiv_rn(w2, d), __fdiv_rn(w3, d)) << 8) |
+         (e2m1x2(__fdiv_rn(w4, d), __fdiv_rn(w5, d)) << 16) |
+         (e2m1x2(__fdiv_rn(w6, d), __fdiv_rn(w7, d)) << 24);
+}
+
+// The codes of e2m1x8_div with the divisions only where they can matter:
+// the bracket of e2m1x2_quot for eight quotients at once, with one check.
+// Its ends are w * r_lo and w * r_hi, r_lo = fl(r (1 - 2^-19)) and
+// r_hi = fl(r (1 + 2^-19)), r = fl(1 / d): each end lies within 5 * 2^-24
+// (relative) of v (1 -+ 2^-19), so on the far side of the rounded quotient
+// v, and equal codes at both ends are the codes of v.  d in [2^-126, 2^126).
+__device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d) {
+  const float r = __frcp_rn(d);
+  const float r_lo = r * (1.0f - 0x1p-19f), r_hi = r * (1.0f + 0x1p-19f);
+  uint32_t a = 0, b = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    a |= e2m1x2(w[2 * j] * r_lo, w[2 * j + 1] * r_lo) << (8 * j);
+    b |= e2m1x2(w[2 * j] * r_hi, w[2 * j + 1] * r_hi) << (8 * j);
+  }
+  return a == b ? a : e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
+}
+
+// Whether e2m1x2_quot / e2m1x8_quot may be used with divisor d.
 __device__ __forceinline__ bool quot_fast_ok(float d) {
   return d >= 0x1p-126f && d < 0x1p126f;
 }

@@ -2,6 +2,7 @@
 // translation units.  Arguments reaching these functions are validated.
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -9,6 +10,14 @@ namespace mxq {
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+// CTAs of `kernel` that fit on one SM at `threads` threads and `smem` bytes
+// of dynamic shared memory (occupancy query, cached per kernel and device;
+// 1 if the query fails).
+int resident_ctas(const void* kernel, int threads, size_t smem);
+// Grid of a grid-stride streaming kernel: one CTA per per_cta units, at
+// most one full wave (SMs x resident CTAs), so that no CTA waits for a
+// second wave.
+int wave_grid(const void* kernel, int threads, int64_t n_units, int64_t per_cta);
 
 int launch_mx_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed, void* scales,
                        cudaStream_t st);

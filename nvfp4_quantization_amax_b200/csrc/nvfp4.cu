@@ -9,8 +9,10 @@
 // CTA on the magnitude bits, which order like the values), then the
 // streaming quantize pass (same item/lane layout as the MXFP4 pack, with a
 // block of 16 held by two lanes).  Every binary32 operation the recipe names
-// (the divisions and products) is the IEEE-rounded one (div.rn / mul.rn), so
-// the codes match a plain float32 implementation bit for bit.
+// (the divisions and products) is the IEEE-rounded one (div.rn / mul.rn), or
+// gives provably the same E2M1 code (the guarded reciprocal quotient of
+// e2m1x8_quot), so the codes match a plain float32 implementation bit for
+// bit.
 #include <mutex>
 
 #include "mxq_device.cuh"
@@ -122,14 +124,16 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
         sbyte = e4m3x2(q, 0.0f) & 0xFFu;
         const float s = f16lo(e4m3x2_to_f16x2(sbyte));
         const float d = __fmul_rn(s, g);
-        float v[8];
+        float w[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           uint32_t bits = elem_bits<DT>(va[u], vb[u], j);
           if (bits == negzero) bits = 0u;  // -0.0 carries no sign into the code
-          v[j] = __fdiv_rn(elem_to_f32<DT>(bits), d);  // keeps the sign on underflow
+          w[j] = elem_to_f32<DT>(bits);
         }
-        codes = e2m1x8(v);
+        // E2M1 of the binary32 quotients w / d (the sign is kept on underflow)
+        codes = quot_fast_ok(d) ? e2m1x8_quot(w, d)
+                                : e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
       }
       packed[item] = codes;
       if ((lane & 1) == 0) block_scales[item >> 1] = (uint8_t)sbyte;
@@ -175,19 +179,17 @@ nvfp4_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __re
   }
 }
 
-int grid_for(int64_t n_units, int per_block, int resident) {
-  int64_t need = (n_units + per_block - 1) / per_block;
-  int64_t cap = (int64_t)num_sms() * resident;
-  if (need > cap) need = cap;
-  return (int)(need < 1 ? 1 : need);
+template <class Kernel>
+int grid_for(Kernel kernel, int64_t n_units, int per_block) {
+  return wave_grid((const void*)kernel, kNvThreads, n_units, per_block);
 }
 
 template <int DT>
 void run_amax(const void* x, int64_t n_items, uint32_t* amax_word, cudaStream_t st) {
   clear_word_kernel<<<1, 1, 0, st>>>(amax_word);
   if (n_items > 0) {
-    nvfp4_amax_kernel<DT><<<grid_for(n_items, kNvThreads * kNvUnroll, 8), kNvThreads, 0, st>>>(
-        x, n_items, amax_word);
+    const int grid = grid_for(nvfp4_amax_kernel<DT>, n_items, kNvThreads * kNvUnroll);
+    nvfp4_amax_kernel<DT><<<grid, kNvThreads, 0, st>>>(x, n_items, amax_word);
   }
 }
 
@@ -196,7 +198,8 @@ int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* blo
                  float* global_scale, uint32_t* amax_word, cudaStream_t st) {
   const int64_t n_items = rows * (K / 8);
   run_amax<DT>(x, n_items, amax_word, st);
-  nvfp4_quantize_kernel<DT><<<grid_for(n_items, kNvThreads * kNvUnroll, 4), kNvThreads, 0, st>>>(
+  const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items, kNvThreads * kNvUnroll);
+  nvfp4_quantize_kernel<DT><<<grid, kNvThreads, 0, st>>>(
       x, (uint32_t*)packed, (uint8_t*)block_scales, global_scale, amax_word, n_items);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
@@ -256,13 +259,22 @@ void launch_nvfp4_amax(const void* x, int dt, int64_t n_elems, uint32_t* amax_wo
 int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                             int64_t rows, int64_t K, void* out, int dt, cudaStream_t st) {
   const int64_t n_items = rows * (K / 8);
-  const int grid = grid_for(n_items, kNvThreads * kNvUnroll, 8);
+  const int per = kNvThreads * kNvUnroll;
   auto* p = (const uint32_t*)packed;
   auto* s = (const uint8_t*)block_scales;
   switch (dt) {
-    case kBF16: nvfp4_dequantize_kernel<kBF16><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
-    case kF16: nvfp4_dequantize_kernel<kF16><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
-    default: nvfp4_dequantize_kernel<kF32><<<grid, kNvThreads, 0, st>>>(p, s, global_scale, out, n_items); break;
+    case kBF16:
+      nvfp4_dequantize_kernel<kBF16><<<grid_for(nvfp4_dequantize_kernel<kBF16>, n_items, per),
+                                       kNvThreads, 0, st>>>(p, s, global_scale, out, n_items);
+      break;
+    case kF16:
+      nvfp4_dequantize_kernel<kF16><<<grid_for(nvfp4_dequantize_kernel<kF16>, n_items, per),
+                                      kNvThreads, 0, st>>>(p, s, global_scale, out, n_items);
+      break;
+    default:
+      nvfp4_dequantize_kernel<kF32><<<grid_for(nvfp4_dequantize_kernel<kF32>, n_items, per),
+                                      kNvThreads, 0, st>>>(p, s, global_scale, out, n_items);
+      break;
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
