@@ -127,24 +127,6 @@ __device__ __forceinline__ uint32_t e2m1x2(float a, float b) {
   return r;
 }
 
-// E2M1 codes (one byte, a in the low nibble) of the binary32 quotients
-// a / d and b / d, exactly as e2m1x2(__fdiv_rn(a, d), __fdiv_rn(b, d)), with
-// the divisions only where they can matter.  r = fl32(1 / d), d in
-// [2^-126, 2^126) (so r is a normal number).  a * r is within 2^-22
-// (relative) of the rounded quotient v; scaling it by 1 -+ 2^-19 gives a
-// bracket that contains v, and where the (monotone) cast gives the same
-// codes at both ends of the bracket it gives them for v too.  Otherwise a
-// quotient lies within ~2^-19 of an E2M1 decision point and the IEEE
-// divisions decide.  Signs (including -0 and underflow to zero) follow a and
-// b in both paths.
-__device__ __forceinline__ uint32_t e2m1x2_quot(float a, float b, float d, float r) {
-  const float va = a * r, vb = b * r;
-  const uint32_t lo = e2m1x2(va * (1.0f - 0x1p-19f), vb * (1.0f - 0x1p-19f));
-  const uint32_t hi = e2m1x2(va * (1.0f + 0x1p-19f), vb * (1.0f + 0x1p-19f));
-  if (lo == hi) return lo;
-  return e2m1x2(__fdiv_rn(a, d), __fdiv_rn(b, d));
-}
-
 // E2M1 codes of the eight binary32 quotients w_j / d by IEEE division
 // (element 2j in the low nibble of byte j).  Out of line: it is the rare
 // path of e2m1x8_quot.
@@ -157,15 +139,25 @@ static __device__ __noinline__ uint32_t e2m1x8_div(float w0, float w1, float w2,
          (e2m1x2(__fdiv_rn(w6, d), __fdiv_rn(w7, d)) << 24);
 }
 
-// The codes of e2m1x8_div with the divisions only where they can matter:
-// the bracket of e2m1x2_quot for eight quotients at once, with one check.
-// Its ends are w * r_lo and w * r_hi, r_lo = fl(r (1 - 2^-19)) and
-// r_hi = fl(r (1 + 2^-19)), r = fl(1 / d): each end lies within 5 * 2^-24
-// (relative) of v (1 -+ 2^-19), so on the far side of the rounded quotient
-// v, and equal codes at both ends are the codes of v.  d in [2^-126, 2^126).
-__device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d) {
+// Bracket factors of a divisor d in [2^-126, 2^126) (quot_fast_ok):
+// r = fl(1 / d), r_lo = fl(r (1 - 2^-19)), r_hi = fl(r (1 + 2^-19)).
+__device__ __forceinline__ void bracket_factors(float d, float& r_lo, float& r_hi) {
   const float r = __frcp_rn(d);
-  const float r_lo = r * (1.0f - 0x1p-19f), r_hi = r * (1.0f + 0x1p-19f);
+  r_lo = r * (1.0f - 0x1p-19f);
+  r_hi = r * (1.0f + 0x1p-19f);
+}
+
+// The codes of e2m1x8_div, with the divisions only where they can matter.
+// For the rounded quotient v = fl(w / d), the products w * r_lo and
+// w * r_hi (binary32) each lie within 5 * 2^-24 (relative) of
+// v (1 -+ 2^-19), so they bracket v from below and above in magnitude, with
+// its sign.  The cast to E2M1 is monotone, so where it gives the same codes
+// at both ends of the brackets it gives them for v too; otherwise some
+// quotient lies within ~2^-19 of an E2M1 decision point and the IEEE
+// divisions decide.  Quotients near the binary32 underflow threshold are far
+// below the first decision point (0.25): every end then casts to a zero
+// magnitude with the sign of w, as v does.
+__device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d, float r_lo, float r_hi) {
   uint32_t a = 0, b = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -175,7 +167,14 @@ __device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d) {
   return a == b ? a : e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
 }
 
-// Whether e2m1x2_quot / e2m1x8_quot may be used with divisor d.
+__device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d) {
+  float r_lo, r_hi;
+  bracket_factors(d, r_lo, r_hi);
+  return e2m1x8_quot(w, d, r_lo, r_hi);
+}
+
+// Whether the bracket (e2m1x8_quot) may be used with divisor d: then r is
+// a normal number.
 __device__ __forceinline__ bool quot_fast_ok(float d) {
   return d >= 0x1p-126f && d < 0x1p126f;
 }

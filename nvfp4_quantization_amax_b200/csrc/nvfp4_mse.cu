@@ -118,14 +118,21 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
         const double dd = (double)d;
         const double t = amax_d - 6.0 * dd;
         if (t > 0.0 && t * t * (1.0 - 0x1p-40) > best) break;
-        const bool fast = quot_fast_ok(d);
-        const float r = fast ? __frcp_rn(d) : 0.0f;
+        // the 16 E2M1 codes of fl32(w / d), eight per word
+        uint32_t q[2];
+        if (quot_fast_ok(d)) {
+          float r_lo, r_hi;
+          bracket_factors(d, r_lo, r_hi);
+          q[0] = e2m1x8_quot(w, d, r_lo, r_hi);
+          q[1] = e2m1x8_quot(w + 8, d, r_lo, r_hi);
+        } else {
+          q[0] = e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
+          q[1] = e2m1x8_div(w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15], d);
+        }
         double err = 0.0;
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const uint32_t h2 = e2m1x2_to_f16x2(
-              fast ? e2m1x2_quot(w[i], w[i + 1], d, r)
-                   : e2m1x2(__fdiv_rn(w[i], d), __fdiv_rn(w[i + 1], d)));
+          const uint32_t h2 = e2m1x2_to_f16x2((q[i >> 3] >> (4 * (i & 7))) & 0xFFu);
           const double e0 = fma(f16_to_f64(h2 & 0xFFFFu), dd, -wd[i]);
           err = fma(e0, e0, err);
           const double e1 = fma(f16_to_f64(h2 >> 16), dd, -wd[i + 1]);
@@ -161,14 +168,9 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
       v[i] = w[i] == 0.0f ? 0.0f : w[i];
     }
     if (quot_fast_ok(d)) {
-      const float r = __frcp_rn(d);
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        lo |= e2m1x2_quot(v[2 * j], v[2 * j + 1], d, r) << (8 * j);
-        hi |= e2m1x2_quot(v[8 + 2 * j], v[8 + 2 * j + 1], d, r) << (8 * j);
-      }
-      codes = make_uint2(lo, hi);
+      float r_lo, r_hi;
+      bracket_factors(d, r_lo, r_hi);
+      codes = make_uint2(e2m1x8_quot(v, d, r_lo, r_hi), e2m1x8_quot(v + 8, d, r_lo, r_hi));
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = v[i] == 0.0f ? 0.0f : __fdiv_rn(v[i], d);
