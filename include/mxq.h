@@ -15,6 +15,10 @@
  *  - Return value: MXQ_OK (0) or a negative mxq_status.  Argument errors are
  *    detected on the host before anything is launched and leave every output
  *    untouched.  MXQ_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *  - Outputs never alias: an output buffer that overlaps an input or another
+ *    output of the same call (by the byte extents the sizes give) is
+ *    MXQ_ERR_INVALID_ARG.  Sizes whose byte extents do not fit in 62 bits
+ *    are MXQ_ERR_SHAPE.
  *  - Element dtypes are mxq_dtype values; floating-point results are rounded
  *    to nearest-even with subnormals kept and overflow to +-infinity.
  *  - Inputs are expected to be finite; NaN/Inf inputs give unspecified

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <initializer_list>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -67,6 +68,30 @@ static bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
   return x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
 }
 
+// A byte extent of a call's buffer: where it starts and how long it is.
+struct Extent {
+  const void* p;
+  int64_t bytes;
+};
+
+// Whether every output extent is disjoint from every other extent (inputs
+// may overlap one another).  Null or empty extents take no part.
+static bool no_alias(std::initializer_list<Extent> outputs, std::initializer_list<Extent> inputs) {
+  for (auto o = outputs.begin(); o != outputs.end(); ++o) {
+    if (!o->p || o->bytes <= 0) continue;
+    for (auto q = o + 1; q != outputs.end(); ++q)
+      if (q->p && q->bytes > 0 && overlap(o->p, o->bytes, q->p, q->bytes)) return false;
+    for (const Extent& i : inputs)
+      if (i.p && i.bytes > 0 && overlap(o->p, o->bytes, i.p, i.bytes)) return false;
+  }
+  return true;
+}
+
+// rows x cols elements of up to 8 bytes have a byte extent below 2^62.
+static bool fits(int64_t rows, int64_t cols) {
+  return rows >= 0 && cols >= 0 && (cols == 0 || rows <= ((int64_t)1 << 59) / cols);
+}
+
 }  // namespace mxq
 
 using namespace mxq;
@@ -79,7 +104,11 @@ int mx_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packe
   if (rows < 0 || K < 0 || K % 32 != 0) return MXQ_ERR_SHAPE;
   if (rows == 0 || K == 0) return MXQ_OK;
   if (!x || !packed || !scales) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(packed)) return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{packed, rows * K / 2}, {scales, rows * K / 32}},
+                {{x, rows * K * elem_bytes(x_dtype)}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_mx_quantize(x, x_dtype, rows, K, packed, scales, (cudaStream_t)stream);
 }
 
@@ -89,7 +118,11 @@ int mx_dequantize(const void* packed, const void* scales, int64_t rows, int64_t 
   if (rows < 0 || K < 0 || K % 32 != 0) return MXQ_ERR_SHAPE;
   if (rows == 0 || K == 0) return MXQ_OK;
   if (!packed || !scales || !out) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (!aligned16(packed) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{out, rows * K * elem_bytes(out_dtype)}},
+                {{packed, rows * K / 2}, {scales, rows * K / 32}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_mx_dequantize(packed, scales, rows, K, out, out_dtype, (cudaStream_t)stream);
 }
 
@@ -101,6 +134,7 @@ int quantize_cache(const void* in, void* out, int dtype, int64_t rows, int64_t c
   if (rows < 0 || channels < 0 || block_size < 1) return MXQ_ERR_SHAPE;
   if (rows == 0 || channels == 0) return MXQ_OK;
   if (!in || !out) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, channels)) return MXQ_ERR_SHAPE;
   int64_t bytes = rows * channels * elem_bytes(dtype);
   if (overlap(in, bytes, out, bytes)) return MXQ_ERR_INVALID_ARG;
   if (!elem_aligned(in, dtype) || !elem_aligned(out, dtype)) return MXQ_ERR_ALIGNMENT;
@@ -130,7 +164,12 @@ int quantize_cache_packed(const void* in, int dtype, int64_t rows, int64_t chann
   if (rc != MXQ_OK) return rc;
   if (rows == 0 || channels == 0) return MXQ_OK;
   if (!in || !codes || !scales) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, channels)) return MXQ_ERR_SHAPE;
   if (!elem_aligned(in, dtype)) return MXQ_ERR_ALIGNMENT;
+  const int64_t code_bytes = format == MXQ_FMT_FP8 ? rows * channels : rows * channels / 2;
+  if (!no_alias({{codes, code_bytes}, {scales, rows * (channels / block_size)}},
+                {{in, rows * channels * elem_bytes(dtype)}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_quantize_cache_packed(in, dtype, rows, channels, format, block_size, codes, scales,
                                       packed_fast(block_size, in, codes), (cudaStream_t)stream);
 }
@@ -142,7 +181,12 @@ int dequantize_cache_packed(const void* codes, const void* scales, int64_t rows,
   if (rc != MXQ_OK) return rc;
   if (rows == 0 || channels == 0) return MXQ_OK;
   if (!codes || !scales || !out) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, channels)) return MXQ_ERR_SHAPE;
   if (!elem_aligned(out, out_dtype)) return MXQ_ERR_ALIGNMENT;
+  const int64_t code_bytes = format == MXQ_FMT_FP8 ? rows * channels : rows * channels / 2;
+  if (!no_alias({{out, rows * channels * elem_bytes(out_dtype)}},
+                {{codes, code_bytes}, {scales, rows * (channels / block_size)}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_dequantize_cache_packed(codes, scales, rows, channels, format, block_size, out,
                                         out_dtype, packed_fast(block_size, out, codes),
                                         (cudaStream_t)stream);
@@ -156,7 +200,15 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
   if (!packed || !scales || !offs) return MXQ_ERR_INVALID_ARG;
   if (T == 0) return MXQ_OK;
   if (!a || !y) return MXQ_ERR_INVALID_ARG;
+  if (!fits(T, N > K ? N : K) || !fits(E, N) || !fits(E * N, K)) return MXQ_ERR_SHAPE;
   if (E > 65536) return MXQ_ERR_UNSUPPORTED;
+  {
+    const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
+    if (!no_alias({{y, T * nout * 2}, {dev_status, 4}},
+                  {{a, T * kin * 2}, {packed, E * N * K / 2}, {scales, E * N * K / 32},
+                   {offs, E * 4}}))
+      return MXQ_ERR_INVALID_ARG;
+  }
   return launch_grouped_mm(a, packed, scales, offs, T, E, N, K, transpose_w, y, dev_status,
                            (cudaStream_t)stream);
 }
@@ -168,11 +220,16 @@ int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void
   if (!packed || !scales || !offs) return MXQ_ERR_INVALID_ARG;
   if (T == 0) return MXQ_OK;
   if (!x_packed || !x_scales || !y) return MXQ_ERR_INVALID_ARG;
+  if (!fits(T, N > K ? N : K) || !fits(E, N) || !fits(E * N, K)) return MXQ_ERR_SHAPE;
   if (K % 256 != 0 || N % 128 != 0 || T >= ((int64_t)1 << 31) || E * N >= ((int64_t)1 << 31))
     return MXQ_ERR_UNSUPPORTED;
   if (!aligned16(x_packed) || !aligned16(x_scales) || !aligned16(packed) || !aligned16(scales) ||
       !aligned16(y))
     return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{y, T * N * 2}, {dev_status, 4}},
+                {{x_packed, T * K / 2}, {x_scales, T * K / 32}, {packed, E * N * K / 2},
+                 {scales, E * N * K / 32}, {offs, E * 4}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_w4a4_grouped_mm(x_packed, x_scales, packed, scales, offs, T, E, N, K, y,
                                 dev_status, get_wait_limit_ns(), (cudaStream_t)stream);
 }
@@ -186,11 +243,17 @@ int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
   if (!packed || !block_scales || !w_global_scales || !offs) return MXQ_ERR_INVALID_ARG;
   if (T == 0) return MXQ_OK;
   if (!x_packed || !x_block_scales || !x_global_scale || !y) return MXQ_ERR_INVALID_ARG;
+  if (!fits(T, N > K ? N : K) || !fits(E, N) || !fits(E * N, K)) return MXQ_ERR_SHAPE;
   if (K % 256 != 0 || N % 128 != 0 || T >= ((int64_t)1 << 31) || E * N >= ((int64_t)1 << 31))
     return MXQ_ERR_UNSUPPORTED;
   if (!aligned16(x_packed) || !aligned16(x_block_scales) || !aligned16(packed) ||
       !aligned16(block_scales) || !aligned16(y))
     return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{y, T * N * 2}, {dev_status, 4}},
+                {{x_packed, T * K / 2}, {x_block_scales, T * K / 16}, {x_global_scale, 4},
+                 {packed, E * N * K / 2}, {block_scales, E * N * K / 16},
+                 {w_global_scales, E * 4}, {offs, E * 4}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_nvfp4_w4a4_grouped_mm(x_packed, x_block_scales, x_global_scale, packed,
                                       block_scales, w_global_scales, offs, T, E, N, K, y,
                                       dev_status, get_wait_limit_ns(), (cudaStream_t)stream);
@@ -202,8 +265,13 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
   if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
   if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
     return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4},
+                 {workspace, MXQ_NVFP4_WORKSPACE_BYTES}},
+                {{x, rows * K * elem_bytes(x_dtype)}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_nvfp4_quantize(x, x_dtype, rows, K, packed, block_scales, global_scale,
                                (uint32_t*)workspace, (cudaStream_t)stream);
 }
@@ -214,8 +282,13 @@ int nvfp4_quantize_mse(const void* x, int x_dtype, int64_t rows, int64_t K, void
   if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
   if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
     return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4},
+                 {workspace, MXQ_NVFP4_WORKSPACE_BYTES}},
+                {{x, rows * K * elem_bytes(x_dtype)}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_nvfp4_quantize_mse(x, x_dtype, rows, K, packed, block_scales, global_scale,
                                    (uint32_t*)workspace, (cudaStream_t)stream);
 }
@@ -226,7 +299,11 @@ int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, 
   if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
   if (!global_scale) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))) return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4}},
+                {{x, rows * K * elem_bytes(x_dtype)}}))
+    return MXQ_ERR_INVALID_ARG;
   int status = MXQ_OK;
   uint32_t* scratch = noalloc_scratch(MXQ_NVFP4_WORKSPACE_BYTES, &status);
   if (!scratch) return status;
@@ -240,7 +317,11 @@ int nvfp4_dequantize(const void* packed, const void* block_scales, const float* 
   if (rows < 0 || K < 0 || K % 16 != 0) return MXQ_ERR_SHAPE;
   if (rows == 0 || K == 0) return MXQ_OK;
   if (!packed || !block_scales || !global_scale || !out) return MXQ_ERR_INVALID_ARG;
+  if (!fits(rows, K)) return MXQ_ERR_SHAPE;
   if (!aligned16(packed) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  if (!no_alias({{out, rows * K * elem_bytes(out_dtype)}},
+                {{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4}}))
+    return MXQ_ERR_INVALID_ARG;
   return launch_nvfp4_dequantize(packed, block_scales, global_scale, rows, K, out, out_dtype,
                                  (cudaStream_t)stream);
 }

@@ -193,3 +193,41 @@ def test_nvfp4_w4a4_validation(L):
     assert f(A1, A1, A2, A2, A2, A2, A2, 8, 2, 128, 96, A1, NULL, NULL) == EUNSUP
     assert f(BAD, A1, A2, A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
     assert f(A1, A1, A2, A2, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK
+
+
+A3 = ctypes.c_void_p(0x30000)  # never dereferenced
+BIG = 1 << 40
+
+
+def test_outputs_that_alias_are_rejected(L):
+    # x [4, 64] bf16 at A1 (512 bytes): packed inside it
+    assert L.mx_quantize(A1, 0, 4, 64, ctypes.c_void_p(0x10100), A2, NULL) == EARG
+    assert L.mx_quantize(A1, 0, 4, 64, A2, ctypes.c_void_p(0x20010), NULL) == EARG  # scales in packed
+    assert L.mx_dequantize(A1, A2, 4, 64, A1, 0, NULL) == EARG  # out over packed
+    assert L.mx_dequantize(A1, A2, 4, 64, ctypes.c_void_p(0x1FF00), 0, NULL) == EARG  # out reaches scales
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, A3, ctypes.c_void_p(0x30010), NULL) == EARG
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, ctypes.c_void_p(0x20080), A1, A3, NULL) == EARG
+    assert L.nvfp4_quantize_mse(A1, 0, 4, 64, A2, A2, A3, ctypes.c_void_p(0x30010), NULL) == EARG
+    assert L.nvfp4_quantize_noalloc(A1, 0, 4, 64, A2, ctypes.c_void_p(0x20010), A3, NULL) == EARG
+    assert L.nvfp4_dequantize(A1, A2, A3, 4, 64, ctypes.c_void_p(0x1FF80), 0, NULL) == EARG
+    q, d = L.quantize_cache_packed, L.dequantize_cache_packed
+    assert q(A1, 0, 4, 64, 0, 32, A1, A2, NULL) == EARG  # codes over the input
+    assert q(A1, 0, 4, 64, 1, 32, A2, ctypes.c_void_p(0x20020), NULL) == EARG  # scales in codes
+    assert d(A1, A2, 4, 64, 2, 16, ctypes.c_void_p(0x1FFF0), 0, NULL) == EARG
+    # grouped GEMMs: y over the activations, or the status word inside y
+    assert L.mxfp4_grouped_mm(A1, A2, A3, A3, 8, 2, 128, 256, 0, A1, NULL, NULL) == EARG
+    assert L.mxfp4_grouped_mm(A1, A2, A3, A3, 8, 2, 128, 256, 0, ctypes.c_void_p(0x40000),
+                              ctypes.c_void_p(0x40010), NULL) == EARG
+    assert L.mxfp4_w4a4_grouped_mm(A1, A1, A2, A2, A3, 8, 2, 128, 256, A1, NULL, NULL) == EARG
+    assert L.nvfp4_w4a4_grouped_mm(A1, A1, A1, A2, A2, A2, A3, 8, 2, 128, 256, A3, NULL,
+                                   NULL) == EARG
+
+
+def test_sizes_beyond_62_bits_are_rejected(L):
+    assert L.mx_quantize(A1, 0, BIG, BIG, A2, A3, NULL) == ESHAPE
+    assert L.mx_dequantize(A1, A2, BIG, BIG, A3, 0, NULL) == ESHAPE
+    assert L.quantize_cache(A1, A2, 0, BIG, BIG, 0, 32, NULL) == ESHAPE
+    assert L.nvfp4_quantize(A1, 0, BIG, BIG, A2, A2, A3, A3, NULL) == ESHAPE
+    assert L.nvfp4_dequantize(A1, A2, A3, BIG, BIG, A3, 0, NULL) == ESHAPE
+    assert L.quantize_cache_packed(A1, 0, BIG, 1 << 30, 0, 32, A2, A3, NULL) == ESHAPE
+    assert L.mxfp4_grouped_mm(A1, A2, A3, A3, BIG, 2, 128, BIG, 0, A1, NULL, NULL) == ESHAPE
