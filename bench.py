@@ -333,31 +333,34 @@ def run_gpu(args, rank, world):
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
     step = Step(torch, mxq, gen, dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in step.names]
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
     if int(step.status.item()) != 0:
         raise RuntimeError("grouped GEMM reported status %d" % int(step.status.item()))
 
-    per = {n: [] for n in step.names}
+    # One pair of events per kernel and step, read after the closing
+    # synchronize: the host queues the steps back to back, so no kernel
+    # starts on an idle GPU and no event pair spans host launch overhead.
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in step.names]
+          for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(gpu_id(torch, dev)) as clk:
         start.record()
-        for _ in range(args.steps):
-            step.run(ev)
-            torch.cuda.synchronize()  # read this step's events
-            for n, (a, b) in zip(step.names, ev):
-                per[n].append(a.elapsed_time(b))
+        for k in range(args.steps):
+            step.run(ev[k])
         stop.record()
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    if int(step.status.item()) != 0:
+        raise RuntimeError("grouped GEMM reported status %d" % int(step.status.item()))
     total_ms = start.elapsed_time(stop)
-    kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
+    kern_ms = {n: sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps)) / args.steps
+               for i, n in enumerate(step.names)}
     red = max_over_ranks([total_ms] + [kern_ms[n] for n in step.names], dev)
     total_ms = red[0]
     kern_ms = dict(zip(step.names, red[1:]))
