@@ -211,7 +211,8 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
     """Device time (ms, mean over reps, max over ranks) of the next-row
     kernels: NVFP4 two-level quantize (max and mse block-scale rules) and
     dequantize on the expert weights; packed cache quantize / unpack on the
-    three KV-cache tensors.  Timed after, and outside, the main step."""
+    three KV-cache tensors; the W4A4 GEMMs.  Timed after, and outside, the
+    main step, each call on an L2 flushed before it."""
     packed, bscales, g = mxq.nvfp4_quantize(step.W)
     packed2, bscales2, g2 = mxq.nvfp4_quantize(step.W)
     ws = torch.empty(16, dtype=torch.uint8, device=dev)
@@ -244,18 +245,24 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
     del nvq
     calls["nvfp4_w4a4_grouped_mm"] = lambda: mxq.nvfp4_w4a4_grouped_mm(
         step.x, nvp, nvs, nvg, step.offs, step.y, step.status)
+    # Before each timed call a 256 MB write flushes L2 (126 MB) and keeps the
+    # GPU busy while the host queues the call, so each event pair holds the
+    # call's own kernels on cold inputs and no host launch overhead.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     out = {}
     for name, fn in calls.items():
         for _ in range(2):
             fn()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
         torch.cuda.synchronize()
-        a.record()
-        for _ in range(reps):
+        for a, b in ev:
+            flush.zero_()
+            a.record()
             fn()
-        b.record()
+            b.record()
         torch.cuda.synchronize()
-        out[name] = a.elapsed_time(b) / reps
+        out[name] = sum(a.elapsed_time(b) for a, b in ev) / reps
     names = list(out)
     vals = max_over_ranks([out[n] for n in names], dev)
     return dict(zip(names, vals))
