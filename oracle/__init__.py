@@ -9,6 +9,7 @@ Arrays of floating-point elements are passed as their raw bit patterns:
 uint16 for bf16 / f16, uint32 for f32.
 """
 import ctypes
+import os
 
 import numpy as np
 
@@ -20,11 +21,16 @@ _BITS = {"bf16": np.uint16, "f16": np.uint16, "f32": np.uint32}
 
 _lib = None
 
+# An already-built oracle library to load instead of oracle/liboracle.so: the
+# mutation tests point it at copies of the oracle with a planted mistake and
+# check that the pins catch each one.
+LIB_ENV = "MXQ_ORACLE_LIB"
+
 
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get(LIB_ENV) or _build.build()
         L = ctypes.CDLL(path)
         d, i, i64, p = ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
         L.orc_e2m1_value.restype = d

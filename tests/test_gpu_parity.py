@@ -372,6 +372,27 @@ def test_nvfp4_dequantize_exact(dtype):
     assert_bits_equal(bits(y), oracle.nvfp4_dequantize(wp, ws, wg, _NAME[dtype]), "dequant")
 
 
+@pytest.mark.parametrize("rule", ["max", "mse"])
+def test_nvfp4_blocks_far_below_the_tensor_max(rule):
+    # block-scale quotients below 2^-9 clamp to the smallest E4M3 scale
+    # (byte 0x01) under the max rule; values of a few 2^-9 g still get codes
+    grid = 2.0**-9 / 2688.0
+    x = torch.zeros(4, 64)
+    x[0, 0] = 1.0
+    x[0, 1:64] = gen.normal_bf16(43, (63,)).float() * 0.25
+    for r in range(1, 4):
+        x[r] = torch.tensor([(0.3 + 0.09 * i) * grid * r * (-1) ** i for i in range(64)])
+    x = x.to(torch.bfloat16).to(DEV)
+    p, s, g = mxq.nvfp4_quantize(x, rule=rule)
+    fn = oracle.nvfp4_quantize if rule == "max" else oracle.nvfp4_quantize_mse
+    wp, ws, wg = fn(bits(x))
+    assert float(g.item()) == wg
+    assert_bits_equal(u8(s), ws, "block scales")
+    assert_bits_equal(u8(p), wp, "packed")
+    if rule == "max":
+        assert int(u8(s)[1].min()) == 0x01
+
+
 def test_nvfp4_zero_and_ragged():
     z = torch.zeros(3, 48, dtype=torch.bfloat16, device=DEV)
     p, s, g = mxq.nvfp4_quantize(z)

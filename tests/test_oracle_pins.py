@@ -541,6 +541,23 @@ def test_nvfp4_matches_float32_reference():
     assert np.array_equal(p, wp)
 
 
+def test_nvfp4_block_far_below_the_tensor_max_takes_the_smallest_scale():
+    # amax_b / (6 g) below 2^-9 clamps to the smallest E4M3 scale 2^-9 (byte
+    # 0x01, the page's clamp [2^-9, 448]); the block's values, between
+    # 0.25 and 6 grid units of 2^-9 g, still get nonzero codes
+    x = torch.zeros(2, 32)
+    x[0, 0] = 1.0
+    x[0, 1:16] = gen.normal_bf16(41, (15,)).float() * 0.25
+    grid = 2.0**-9 / 2688.0
+    x[1] = torch.tensor([(0.3 + 0.17 * i) * grid * (-1) ** i for i in range(32)])
+    x = x.to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    p, s, g = oracle.nvfp4_quantize(bits)
+    wp, ws, wg = nvfp4_reference(oracle.decode(bits, "bf16"))
+    assert g == wg and np.array_equal(s, ws) and np.array_equal(p, wp)
+    assert (s[1] == 0x01).all() and ((p[1] & 0x77) != 0).any()
+
+
 def test_nvfp4_page_facts(facts):
     x = gen.expert_weights(1, 32, 256).view(32, 256).clone()
     x[5, 16:32] = 0.0  # one all-zero block
