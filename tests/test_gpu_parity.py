@@ -393,6 +393,22 @@ def test_nvfp4_blocks_far_below_the_tensor_max(rule):
         assert int(u8(s)[1].min()) == 0x01
 
 
+@pytest.mark.parametrize("rule", ["max", "mse"])
+def test_nvfp4_sign_follows_x_where_the_quotient_underflows(rule):
+    x = torch.zeros(2, 32)
+    x[0, 0] = 1e30
+    x[0, 1:8] = torch.tensor([-1e-20, -1e-20, 1e-20, -3e-25, 2.5e28, -7e27, -1e-30])
+    x[1] = gen.normal_bf16(44, (32,)).float() * 1e-19
+    x = x.to(torch.bfloat16).to(DEV)
+    p, s, g = mxq.nvfp4_quantize(x, rule=rule)
+    fn = oracle.nvfp4_quantize if rule == "max" else oracle.nvfp4_quantize_mse
+    wp, ws, wg = fn(bits(x))
+    assert float(g.item()) == wg
+    assert_bits_equal(u8(s), ws, "block scales")
+    assert_bits_equal(u8(p), wp, "packed")
+    assert (int(u8(p)[0, 0]) >> 4) == 8 and (int(u8(p)[0, 1]) & 15) == 8
+
+
 def test_nvfp4_zero_and_ragged():
     z = torch.zeros(3, 48, dtype=torch.bfloat16, device=DEV)
     p, s, g = mxq.nvfp4_quantize(z)

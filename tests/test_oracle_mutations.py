@@ -21,7 +21,13 @@ from oracle import build as oracle_build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 
-# name -> (text in oracle/mxq_oracle.c, replacement, which occurrence (0-based))
+# name -> (text in oracle/mxq_oracle.c, replacement, which occurrence (0-based)).
+# Left out as equivalent (no input can tell them apart from the oracle):
+# dropping the clamp of the NVFP4 block-scale quotient at 448 (the quotient is
+# at most 448 (1 + 2^-22) and the E4M3 cast saturates at 448); dropping the
+# +0 fix-up of unpacked fp4 zeros (table entry 8 is already +0.0); dropping the
+# zero-weight shortcut of the mse element cast (0 / d, even 0 / 0, casts to
+# code 0, and -0.0 < 0 is false).
 MUTATIONS = {
     # E2M1 element cast
     "tie_rule_flipped": ("(a == E2M1_MIDPOINTS[i]) && (i % 2 == 1)",
@@ -67,8 +73,6 @@ MUTATIONS = {
     # NVFP4 two-level
     "nvfp4_global_scale_without_6": ("f32_div(amax, 6.0 * 448.0)", "f32_div(amax, 448.0)", 0),
     "nvfp4_zero_block_scale_not_one": ("if (q == 0.0) q = 1.0;", "if (q == 0.0) q = 0.0;", 0),
-    # (the upper clamp of the quotient to 448 has no observable effect: the
-    # quotient is at most 448 (1 + 2^-22) and the E4M3 cast saturates at 448)
     "nvfp4_scale_lower_clamp_dropped": ("if (q < ldexp(1.0, -9)) q = ldexp(1.0, -9);",
                                         "if (q < ldexp(1.0, -9)) q = q;", 0),
     "nvfp4_dequant_scale_byte_bias": ("double s = orc_decode_e4m3(block_scales[r * (K / 16) + k / 16]);",
@@ -83,6 +87,25 @@ MUTATIONS = {
     "mse_last_minimum": ("if (err < best_err) {", "if (err <= best_err) {", 0),
     "mse_error_sign": ("double e = fma(q, d, -w[i]);", "double e = fma(q, d, w[i]);", 0),
     "mse_drops_code_126": ("for (int c = 1; c <= 126; ++c) {", "for (int c = 1; c < 126; ++c) {", 0),
+    # element codecs
+    "f16_decode_subnormal_scale": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);", 0),
+    "f16_encode_bias": ("return s | (uint16_t)((e + 15) << 10) | m;",
+                        "return s | (uint16_t)((e + 16) << 10) | m;", 0),
+    "f32_overflow_threshold": ("if (fabs(r) > ldexp(16777215.0, 104)) r = copysign(INFINITY, v);",
+                               "if (fabs(r) > ldexp(16777215.0, 103)) r = copysign(INFINITY, v);", 0),
+    "bf16_overflow_threshold": ("if (fabs(r) > ldexp(255.0, 120)) r = copysign(INFINITY, v);",
+                                "if (fabs(r) > ldexp(255.0, 119)) r = copysign(INFINITY, v);", 0),
+    # cache tail group and zero signs
+    "cache_tail_group_reads_past_the_row": ("int64_t c1 = c0 + B < C ? c0 + B : C;",
+                                            "int64_t c1 = c0 + B;", 0),
+    "cache_zero_block_scale": ("if (amax == 0.0) return lo;", "if (amax == 0.0) return 0;", 0),
+    # mse degenerate cases
+    "mse_zero_tensor_scale": ("int code = g == 0.0 ? 0x38 : orc_nvfp4_mse_code(w, g);",
+                              "int code = g == 0.0 ? 0x01 : orc_nvfp4_mse_code(w, g);", 0),
+    "mse_sign_from_the_quotient": ("nib[h] = (orc_e2m1_code(fabs(f32_div(xi, d))) & 7) | (xi < 0.0 ? 8 : 0);",
+                                   "nib[h] = orc_e2m1_code(f32_div(xi, d));", 0),
+    "nvfp4_sign_from_the_quotient": ("lo = (orc_e2m1_code(fabs(f32_div(x0, d))) & 7) | (x0 < 0.0 ? 8 : 0);",
+                                     "lo = orc_e2m1_code(f32_div(x0, d));", 0),
     # W4A4
     "w4a4_activations_not_quantized": ("for (int64_t k = 0; k < K; ++k) xa[k] = mx_element(qp, qs, K, 0, k);",
                                        "for (int64_t k = 0; k < K; ++k) xa[k] = decode_bf16(x[t * K + k]);", 0),

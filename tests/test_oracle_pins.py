@@ -173,6 +173,27 @@ def test_f16_rounding_matches_numpy():
     assert np.array_equal(oracle.round_to(v, "f16"), want)
 
 
+def _same_values(got, want):
+    nan = np.isnan(want)
+    return (np.array_equal(np.isnan(got), nan) and np.array_equal(got[~nan], want[~nan])
+            and np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan])))
+
+
+def test_every_f16_and_bf16_pattern_decodes_like_the_libraries():
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    assert _same_values(oracle.decode(allb, "f16"), allb.view(np.float16).astype(np.float64))
+    want = torch.from_numpy(allb.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    assert _same_values(oracle.decode(allb, "bf16"), want)
+
+
+def test_f32_patterns_decode_like_numpy():
+    rng = np.random.default_rng(5)
+    u = np.concatenate([rng.integers(0, 2**32, 200000, dtype=np.uint64).astype(np.uint32),
+                        np.array([0, 0x80000000, 1, 0x807FFFFF, 0x7F7FFFFF, 0x7F800000, 0xFF800000,
+                                  0x00800000], dtype=np.uint32)])
+    assert _same_values(oracle.decode(u, "f32"), u.view(np.float32).astype(np.float64))
+
+
 def test_f32_rounding_matches_numpy():
     rng = np.random.default_rng(3)
     v = rng.standard_normal(100000) * 10.0 ** rng.uniform(-45, 38, 100000)
@@ -556,6 +577,17 @@ def test_nvfp4_block_far_below_the_tensor_max_takes_the_smallest_scale():
     wp, ws, wg = nvfp4_reference(oracle.decode(bits, "bf16"))
     assert g == wg and np.array_equal(s, ws) and np.array_equal(p, wp)
     assert (s[1] == 0x01).all() and ((p[1] & 0x77) != 0).any()
+
+
+def test_nvfp4_sign_follows_x_where_the_quotient_underflows():
+    # the code's sign bit is taken from x (reading N4): -1e-20 / d underflows
+    # to -0.0 in binary32 here (d ~ 448 * 1e30 / 2688) and still gets code 8
+    x = torch.zeros(1, 16)
+    x[0, 0], x[0, 1], x[0, 2], x[0, 3] = 1e30, -1e-20, -1e-20, 1e-20  # odd and even columns
+    bits = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for quantize in (oracle.nvfp4_quantize, oracle.nvfp4_quantize_mse):
+        p, s, g = quantize(bits)
+        assert (p[0, 0] >> 4) == 8 and (p[0, 1] & 15) == 8 and (p[0, 1] >> 4) == 0
 
 
 def test_nvfp4_page_facts(facts):
