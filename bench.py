@@ -20,6 +20,7 @@ Multi-GPU (torchrun): every rank runs the same per-GPU workload (weak
 scaling, no data exchange); timings are the max over ranks.
 """
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -338,7 +339,9 @@ def run_gpu(args, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
+        # a short limit: a rank that never arrives ends the others' barrier
+        # or all-reduce with an error instead of a long hang
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(minutes=3))
     step = Step(torch, mxq, gen, dev)
     for _ in range(args.warmup):
         step.run()
