@@ -231,3 +231,41 @@ def test_sizes_beyond_62_bits_are_rejected(L):
     assert L.nvfp4_dequantize(A1, A2, A3, BIG, BIG, A3, 0, NULL) == ESHAPE
     assert L.quantize_cache_packed(A1, 0, BIG, 1 << 30, 0, 32, A2, A3, NULL) == ESHAPE
     assert L.mxfp4_grouped_mm(A1, A2, A3, A3, BIG, 2, 128, BIG, 0, A1, NULL, NULL) == ESHAPE
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mxq.h"
+
+int main(void) {
+  char buf[64];
+  int64_t x[8];
+  /* argument errors come back before anything touches a GPU */
+  int a = mx_quantize(NULL, MXQ_BF16, 4, 64, NULL, NULL, NULL);
+  int b = mx_quantize(x, MXQ_BF16, 4, 48, x, x, NULL);
+  int c = quantize_cache(x, x, MXQ_BF16, 1, 8, MXQ_FMT_NVFP4, 16, NULL);
+  int d = nvfp4_quantize(x, MXQ_F32, 2, 40, x, x, (float*)x, x, NULL);
+  int e = mxfp4_grouped_mm(x, x, x, (const int32_t*)x, 8, 0, 128, 256, 0, x, NULL, NULL);
+  snprintf(buf, sizeof buf, "%s", mxq_status_string(a));
+  printf("%d %d %d %d %d %s %d %d\n", a, b, c, d, e, buf, mxq_version() >= 100,
+         MXQ_NVFP4_WORKSPACE_BYTES);
+  return strcmp(buf, "MXQ_ERR_INVALID_ARG") != 0;
+}
+"""
+
+
+def test_plain_c_program_builds_against_the_header_and_links(tmp_path, L):
+    # the boundary is a C ABI: a C11 program (no C++, no CUDA headers) that
+    # includes include/mxq.h and links libmxq.so sees every status above
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(mxq._abi.lib_path())
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lmxq",
+                           "-Wl,-rpath," + libdir, "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split() == [str(EARG), str(ESHAPE), str(EARG), str(ESHAPE), str(ESHAPE),
+                                  "MXQ_ERR_INVALID_ARG", "1", "16"]
