@@ -159,6 +159,97 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+# A row-wise call on pinned host tensors of at least two chunks streams them
+# through the GPU in row ranges of about this many input bytes: the copy of
+# chunk i+1 in, the kernels of chunk i and the copy of chunk i-1 out run on
+# three streams at once (both copy directions of the bus and the GPU busy
+# together).  The results equal one call on the whole tensor: these
+# operations treat every row on its own.
+HOST_CHUNK_BYTES = 64 << 20
+_HOST_DEPTH = 3  # device buffer sets in rotation
+
+
+def _streamable(inputs, outputs):
+    """Every input a pinned contiguous host tensor, every given output on
+    the host."""
+    return (torch.cuda.is_available()
+            and all(not t.is_cuda and t.is_pinned() and t.is_contiguous() for t in inputs)
+            and all(o is None or not o.is_cuda for o in outputs))
+
+
+def _host_target(t, shape, dtype, name):
+    """Host output of `shape`: the caller's tensor (checked as _out checks a
+    buffer) or a new pinned one."""
+    n = 1
+    for v in shape:
+        n *= v
+    if t is None:
+        return torch.empty(shape, dtype=dtype, pin_memory=True)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, not %s" % (name, dtype, t.dtype))
+    if t.numel() != n or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous tensor of %d elements" % (name, n))
+    return t
+
+
+def _stream_rows(inputs, outputs, rows, launch, what):
+    """Stream a row-wise call through the GPU in row chunks.
+
+    inputs: pinned host tensors, each viewed [rows, -1]; outputs: host
+    tensors to fill, each viewed [rows, -1]; launch(dev_inputs, dev_outputs,
+    n_rows, stream) issues one chunk's kernels and returns the status.
+    Returns False (nothing done) below two chunks."""
+    ins = [t.view(rows, -1) for t in inputs]
+    outs = [t.view(rows, -1) for t in outputs]
+    in_row = sum(t.shape[1] * t.element_size() for t in ins)
+    chunk = max(1, HOST_CHUNK_BYTES // max(1, in_row))
+    n_chunks = (rows + chunk - 1) // chunk
+    if n_chunks < 2:
+        return False
+    dev = torch.device("cuda", torch.cuda.current_device())
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    depth = min(_HOST_DEPTH, n_chunks)
+    d_in = [[torch.empty((chunk, t.shape[1]), dtype=t.dtype, device=dev) for t in ins]
+            for _ in range(depth)]
+    d_out = [[torch.empty((chunk, t.shape[1]), dtype=t.dtype, device=dev) for t in outs]
+             for _ in range(depth)]
+    in_free = [None] * depth   # the kernels that last read input set j are done
+    out_free = [None] * depth  # the copy that last read output set j is done
+    st = ctypes.c_void_p(comp.cuda_stream)
+    try:
+        for i in range(n_chunks):
+            j = i % depth
+            r0, r1 = i * chunk, min(rows, (i + 1) * chunk)
+            n = r1 - r0
+            if in_free[j] is not None:
+                s_in.wait_event(in_free[j])
+            with torch.cuda.stream(s_in):
+                for d, h in zip(d_in[j], ins):
+                    d[:n].copy_(h[r0:r1], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+            comp.wait_event(landed)
+            if out_free[j] is not None:
+                comp.wait_event(out_free[j])
+            _check(launch([d[:n] for d in d_in[j]], [d[:n] for d in d_out[j]], n, st), what)
+            done = torch.cuda.Event()
+            done.record(comp)
+            in_free[j] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                for d, h in zip(d_out[j], outs):
+                    h[r0:r1].copy_(d[:n], non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(s_out)
+            out_free[j] = copied
+    finally:
+        # every copy out follows its kernels, which follow their copy in
+        s_out.synchronize()
+        comp.synchronize()
+    return True
+
+
 def mx_quantize(x, packed=None, scales=None):
     """MXFP4 quantize + pack along the last dim.
 
@@ -168,6 +259,17 @@ def mx_quantize(x, packed=None, scales=None):
     """
     if x.dtype not in _DTYPES:
         raise TypeError("mx_quantize: unsupported dtype %s" % x.dtype)
+    if _streamable([x], [packed, scales]) and x.dim() >= 1 and x.shape[-1] > 0:
+        K = x.shape[-1]
+        rows, lead = x.numel() // K, tuple(x.shape[:-1])
+        hp = _host_target(packed, lead + (K // 2,), torch.uint8, "packed")
+        hs = _host_target(scales, lead + (K // 32,), torch.uint8, "scales")
+        dt = _DTYPES[x.dtype]
+        if _stream_rows([x], [hp, hs], rows,
+                        lambda di, do, n, st: lib().mx_quantize(_ptr(di[0]), dt, n, K,
+                                                                _ptr(do[0]), _ptr(do[1]), st),
+                        "mx_quantize"):
+            return hp, hs
     x, host = _to_device(x)
     x = x.contiguous()
     K = x.shape[-1]
@@ -185,6 +287,17 @@ def mx_dequantize(packed, scales, dtype=torch.bfloat16, out=None):
     """Unpack [..., K/2] E2M1 bytes with [..., K/32] E8M0 scales to dtype [..., K]."""
     if dtype not in _DTYPES:
         raise TypeError("mx_dequantize: unsupported dtype %s" % dtype)
+    if (_streamable([packed, scales], [out]) and packed.dim() >= 1 and packed.shape[-1] > 0
+            and scales.numel() * 16 == packed.numel()):
+        K = 2 * packed.shape[-1]
+        rows = packed.numel() // packed.shape[-1]
+        ho = _host_target(out, tuple(packed.shape[:-1]) + (K,), dtype, "out")
+        dt = _DTYPES[dtype]
+        if _stream_rows([packed, scales], [ho], rows,
+                        lambda di, do, n, st: lib().mx_dequantize(_ptr(di[0]), _ptr(di[1]), n, K,
+                                                                  _ptr(do[0]), dt, st),
+                        "mx_dequantize"):
+            return ho
     packed, host = _to_device(packed)
     scales, _ = _to_device(scales, packed.device)
     packed = packed.contiguous()
@@ -208,6 +321,16 @@ def quantize_cache(values, format, block_size, out=None):
         raise TypeError("quantize_cache: unsupported dtype %s" % values.dtype)
     if format not in _FORMATS:
         raise ValueError("quantize_cache: format must be one of %s" % sorted(_FORMATS))
+    if _streamable([values], [out]) and values.dim() >= 1 and values.shape[-1] > 0:
+        C = values.shape[-1]
+        rows = values.numel() // C
+        ho = _host_target(out, tuple(values.shape), values.dtype, "out")
+        dt, fmt, B = _DTYPES[values.dtype], _FORMATS[format], int(block_size)
+        if _stream_rows([values], [ho], rows,
+                        lambda di, do, n, st: lib().quantize_cache(_ptr(di[0]), _ptr(do[0]), dt, n,
+                                                                   C, fmt, B, st),
+                        "quantize_cache"):
+            return ho
     values, host = _to_device(values)
     values = values.contiguous()
     C = values.shape[-1] if values.dim() else 1

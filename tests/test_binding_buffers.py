@@ -126,3 +126,42 @@ def test_host_outputs_match_the_oracle():
     wp, ws = oracle.mx_quantize(x.view(torch.int16).numpy().view(np.uint16), "bf16")
     assert np.array_equal(packed.numpy(), np.asarray(wp, dtype=np.uint8).reshape(32, 128))
     assert np.array_equal(scales.numpy(), np.asarray(ws, dtype=np.uint8).reshape(32, 8))
+
+
+@pytest.fixture
+def small_chunks():
+    # stream host tensors in many small chunks (ragged last one included)
+    old = _abi.HOST_CHUNK_BYTES
+    _abi.HOST_CHUNK_BYTES = 3000
+    yield
+    _abi.HOST_CHUNK_BYTES = old
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_streamed_host_calls_equal_whole_device_calls(small_chunks, dtype):
+    x = gen.mixed_blocks(37, 256, device=DEV).to(dtype)  # 37 rows: chunks of 5 or 2 rows
+    hx = x.cpu().pin_memory()
+    p, s = mxq.mx_quantize(x)
+    hp, hs = mxq.mx_quantize(hx)
+    assert not hp.is_cuda and torch.equal(hp, p.cpu()) and torch.equal(hs, s.cpu())
+    y = mxq.mx_dequantize(p, s, dtype)
+    hy = mxq.mx_dequantize(hp.pin_memory(), hs.pin_memory(), dtype)
+    assert torch.equal(hy.view(torch.uint8), y.cpu().view(torch.uint8))
+    for fmt, B in (("fp8", 128), ("mxfp4", 32), ("nvfp4", 16)):
+        q = mxq.quantize_cache(x, fmt, B)
+        hq = mxq.quantize_cache(hx, fmt, B)
+        assert torch.equal(hq.view(torch.uint8), q.cpu().view(torch.uint8)), fmt
+
+
+@pytest.mark.gpu
+def test_streamed_host_calls_fill_caller_buffers_and_report_errors(small_chunks):
+    hx = gen.normal_bf16(16, (40, 64)).pin_memory()
+    hp = torch.empty(40, 32, dtype=torch.uint8)                # pageable target
+    hs = torch.empty(40, 2, dtype=torch.uint8, pin_memory=True)
+    rp, rs = mxq.mx_quantize(hx, hp, hs)
+    assert rp is hp and rs is hs
+    wp, ws = mxq.mx_quantize(hx.to(DEV))
+    assert torch.equal(hp, wp.cpu()) and torch.equal(hs, ws.cpu())
+    with pytest.raises(mxq.MxqError):
+        mxq.quantize_cache(hx, "fp8", 0)  # block_size < 1, reported by the first chunk
