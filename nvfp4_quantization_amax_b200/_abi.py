@@ -353,11 +353,23 @@ def quantize_cache_packed(values, format, block_size, codes=None, scales=None):
         raise TypeError("quantize_cache_packed: unsupported dtype %s" % values.dtype)
     if format not in _FORMATS:
         raise ValueError("quantize_cache_packed: format must be one of %s" % sorted(_FORMATS))
+    B = int(block_size)
+    if (_streamable([values], [codes, scales]) and values.dim() >= 1 and values.shape[-1] > 0
+            and B >= 1 and values.shape[-1] % B == 0):
+        C = values.shape[-1]
+        rows, lead = values.numel() // C, tuple(values.shape[:-1])
+        hc = _host_target(codes, lead + (C if format == "fp8" else C // 2,), torch.uint8, "codes")
+        hs = _host_target(scales, lead + (C // B,), torch.uint8, "scales")
+        dt, fmt = _DTYPES[values.dtype], _FORMATS[format]
+        if _stream_rows([values], [hc, hs], rows,
+                        lambda di, do, n, st: lib().quantize_cache_packed(
+                            _ptr(di[0]), dt, n, C, fmt, B, _ptr(do[0]), _ptr(do[1]), st),
+                        "quantize_cache_packed"):
+            return hc, hs
     values, host = _to_device(values)
     values = values.contiguous()
     C = values.shape[-1] if values.dim() else 1
     rows = values.numel() // C if C else 0
-    B = int(block_size)
     lead = tuple(values.shape[:-1])
     dev = values.device
     if B < 1:
@@ -376,10 +388,22 @@ def dequantize_cache_packed(codes, scales, format, block_size, dtype=torch.bfloa
         raise TypeError("dequantize_cache_packed: unsupported dtype %s" % dtype)
     if format not in _FORMATS:
         raise ValueError("dequantize_cache_packed: format must be one of %s" % sorted(_FORMATS))
+    B = int(block_size)
+    if (_streamable([codes, scales], [out]) and scales.dim() >= 1 and scales.shape[-1] > 0
+            and B >= 1):
+        C = scales.shape[-1] * B
+        rows = scales.numel() // scales.shape[-1]
+        if codes.numel() == rows * (C if format == "fp8" else C // 2):
+            ho = _host_target(out, tuple(scales.shape[:-1]) + (C,), dtype, "out")
+            dt, fmt = _DTYPES[dtype], _FORMATS[format]
+            if _stream_rows([codes, scales], [ho], rows,
+                            lambda di, do, n, st: lib().dequantize_cache_packed(
+                                _ptr(di[0]), _ptr(di[1]), n, C, fmt, B, _ptr(do[0]), dt, st),
+                            "dequantize_cache_packed"):
+                return ho
     codes, host = _to_device(codes)
     scales, _ = _to_device(scales, codes.device)
     codes, scales = codes.contiguous(), scales.contiguous()
-    B = int(block_size)
     C = scales.shape[-1] * B
     rows = scales.numel() // scales.shape[-1] if scales.shape[-1] else 0
     if codes.numel() != rows * (C if format == "fp8" else C // 2):
@@ -549,6 +573,19 @@ def nvfp4_dequantize(packed, block_scales, global_scale, dtype=torch.bfloat16, o
     """Unpack NVFP4 storage: E2M1 code * E4M3 block scale * global scale."""
     if dtype not in _DTYPES:
         raise TypeError("nvfp4_dequantize: unsupported dtype %s" % dtype)
+    if (_streamable([packed, block_scales], [out]) and packed.dim() >= 1 and packed.shape[-1] > 0
+            and block_scales.numel() * 8 == packed.numel() and global_scale.numel() >= 1):
+        K = 2 * packed.shape[-1]
+        rows = packed.numel() // packed.shape[-1]
+        ho = _host_target(out, tuple(packed.shape[:-1]) + (K,), dtype, "out")
+        dev = torch.device("cuda", torch.cuda.current_device())
+        gs = global_scale.reshape(-1)[:1].to(device=dev, dtype=torch.float32)
+        dt = _DTYPES[dtype]
+        if _stream_rows([packed, block_scales], [ho], rows,
+                        lambda di, do, n, st: lib().nvfp4_dequantize(
+                            _ptr(di[0]), _ptr(di[1]), _ptr(gs), n, K, _ptr(do[0]), dt, st),
+                        "nvfp4_dequantize"):
+            return ho
     packed, host = _to_device(packed)
     block_scales, _ = _to_device(block_scales, packed.device)
     global_scale, _ = _to_device(global_scale, packed.device)

@@ -165,3 +165,20 @@ def test_streamed_host_calls_fill_caller_buffers_and_report_errors(small_chunks)
     assert torch.equal(hp, wp.cpu()) and torch.equal(hs, ws.cpu())
     with pytest.raises(mxq.MxqError):
         mxq.quantize_cache(hx, "fp8", 0)  # block_size < 1, reported by the first chunk
+
+
+@pytest.mark.gpu
+def test_streamed_packed_cache_and_nvfp4_dequant_equal_device_calls(small_chunks):
+    x = gen.mixed_blocks(29, 256, device=DEV)
+    hx = x.cpu().pin_memory()
+    for fmt, B in (("fp8", 128), ("mxfp4", 32), ("nvfp4", 16)):
+        c, s = mxq.quantize_cache_packed(x, fmt, B)
+        hc, hs = mxq.quantize_cache_packed(hx, fmt, B)
+        assert torch.equal(hc, c.cpu()) and torch.equal(hs, s.cpu()), fmt
+        y = mxq.dequantize_cache_packed(c, s, fmt, B)
+        hy = mxq.dequantize_cache_packed(hc.pin_memory(), hs.pin_memory(), fmt, B)
+        assert torch.equal(hy.view(torch.uint8), y.cpu().view(torch.uint8)), fmt
+    p, s, g = mxq.nvfp4_quantize(x)
+    y = mxq.nvfp4_dequantize(p, s, g, torch.float32)
+    hy = mxq.nvfp4_dequantize(p.cpu().pin_memory(), s.cpu().pin_memory(), g.cpu(), torch.float32)
+    assert not hy.is_cuda and torch.equal(hy.view(torch.uint8), y.cpu().view(torch.uint8))
