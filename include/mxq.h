@@ -48,7 +48,7 @@ typedef enum {
   MXQ_ERR_INVALID_ARG = -1, /* null pointer, bad enum, aliasing in/out    */
   MXQ_ERR_SHAPE = -2,       /* negative size, K % 32 != 0, ...            */
   MXQ_ERR_ALIGNMENT = -3,   /* a pointer the call needs aligned is not    */
-  MXQ_ERR_UNSUPPORTED = -4, /* valid request this build does not handle   */
+  MXQ_ERR_UNSUPPORTED = -4, /* valid request this library does not handle */
   MXQ_ERR_CUDA = -5,        /* launch failed                              */
   MXQ_ERR_BAD_OFFS = -6,    /* device-side: offs not a valid partition    */
   MXQ_ERR_TIMEOUT = -7      /* device-side: a pipeline wait gave up       */
