@@ -48,6 +48,22 @@ int resident_ctas(const void* kernel, int threads, size_t smem) {
   return n;
 }
 
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int>, cudaError_t> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const auto key = std::make_tuple(kernel, dev, bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  const auto it = done.find(key);
+  if (it != done.end()) return it->second;
+  const cudaError_t err =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err != cudaSuccess) (void)cudaGetLastError();  // reported by the return value
+  done[key] = err;
+  return err;
+}
+
 int wave_grid(const void* kernel, int threads, int64_t n_units, int64_t per_cta) {
   int64_t need = (n_units + per_cta - 1) / per_cta;
   const int64_t wave = (int64_t)num_sms() * resident_ctas(kernel, threads, 0);

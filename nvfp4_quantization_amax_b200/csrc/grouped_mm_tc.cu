@@ -34,7 +34,6 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "mxq.h"
 #include "mxq_device.cuh"
@@ -680,12 +679,7 @@ int launch_tc(const void* a, const void* packed, const void* scales, const int32
     }
   }
   auto kernel = grouped_mm_tc_kernel<kDgrad, kPair>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  });
-  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  if (allow_dynamic_smem((const void*)kernel, (int)kSmem) != cudaSuccess) return MXQ_ERR_CUDA;
   // Upper bound on the tile count: every expert may add one ragged tile.
   const int64_t tiles = ((T + kBN - 1) / kBN + E) * (nout / G::kTileM);
   const int64_t slots = num_sms() / G::kCG;

@@ -14,6 +14,10 @@ int num_sms();
 // of dynamic shared memory (occupancy query, cached per kernel and device;
 // 1 if the query fails).
 int resident_ctas(const void* kernel, int threads, size_t smem);
+// Let `kernel` launch with `bytes` of dynamic shared memory on the current
+// device (the attribute belongs to the device's context, so it is set once
+// per kernel and device; the outcome is cached).
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes);
 // Grid of a grid-stride streaming kernel: one CTA per per_cta units, at
 // most one full wave (SMs x resident CTAs), so that no CTA waits for a
 // second wave.

@@ -36,8 +36,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
-#include <mutex>
 #include <type_traits>
 
 #include "mxq.h"
@@ -423,12 +421,7 @@ int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* pac
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return MXQ_ERR_CUDA;
   auto kernel = w4a4_tc_kernel<kNV>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F::kSmem);
-  });
-  if (attr_err != cudaSuccess) return MXQ_ERR_CUDA;
+  if (allow_dynamic_smem((const void*)kernel, (int)F::kSmem) != cudaSuccess) return MXQ_ERR_CUDA;
   const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
   const int64_t sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
