@@ -70,7 +70,12 @@ MUTATIONS = {
     "gemm_dgrad_transposed_weight": ("o[k] += g * w[n * K + k];", "o[k] += g * w[k * N + n];", 0),
     "gemm_expert_rows_off_by_one": ("int64_t lo = e == 0 ? 0 : offs[e - 1], hi = offs[e];",
                                     "int64_t lo = e == 0 ? 0 : offs[e - 1] + 1, hi = offs[e];", 0),
+    "offs_not_checked_for_order": ("if (offs[e] < prev) return ORC_EOFFS;",
+                                   "if (offs[e] < prev && 0) return ORC_EOFFS;", 0),
+    "offs_total_not_checked": ("return prev == T ? ORC_OK : ORC_EOFFS;", "return ORC_OK;", 0),
     # NVFP4 two-level
+    "nvfp4_dequant_rounding_order": ("double v = f32_mul(E2M1_TABLE[nib] * s, (double)global_scale);",
+                                     "double v = E2M1_TABLE[nib] * f32_mul(s, (double)global_scale);", 0),
     "nvfp4_global_scale_without_6": ("f32_div(amax, 6.0 * 448.0)", "f32_div(amax, 448.0)", 0),
     "nvfp4_zero_block_scale_not_one": ("if (q == 0.0) q = 1.0;", "if (q == 0.0) q = 0.0;", 0),
     "nvfp4_scale_lower_clamp_dropped": ("if (q < ldexp(1.0, -9)) q = ldexp(1.0, -9);",
@@ -98,6 +103,10 @@ MUTATIONS = {
     # cache tail group and zero signs
     "cache_tail_group_reads_past_the_row": ("int64_t c1 = c0 + B < C ? c0 + B : C;",
                                             "int64_t c1 = c0 + B;", 0),
+    "cache_fp8_loses_negative_zero": ("if (fmt == ORC_FP8) return ldexp(orc_round_e4m3(v), k);",
+                                      "if (fmt == ORC_FP8) return ldexp(orc_round_e4m3(v), k) + 0.0;", 0),
+    "packed_cache_e8m0_nan_byte": (": sb == 0xFF       ? NAN /* the E8M0 NaN */",
+                                   ": sb == 0xFF       ? 0.0 /* the E8M0 NaN */", 0),
     "cache_zero_block_scale": ("if (amax == 0.0) return lo;", "if (amax == 0.0) return 0;", 0),
     # mse degenerate cases
     "mse_zero_tensor_scale": ("int code = g == 0.0 ? 0x38 : orc_nvfp4_mse_code(w, g);",

@@ -668,6 +668,26 @@ def test_packed_cache_scale_bytes_decode_to_the_power_of_two(fmt):
         assert v == 2.0 ** k, (fmt, k, b)
 
 
+@pytest.mark.parametrize("fmt", ["fp8", "mxfp4"])
+def test_packed_cache_nan_scale_byte_unpacks_to_nan(fmt):
+    # E8M0 byte 0xFF is NaN (reading P2, the E8M0 format): every element of
+    # its group unpacks to NaN; the next group is code x 2^(0x7F - 127)
+    C, B = 64, 32
+    n = C if fmt == "fp8" else C // 2
+    codes = ((np.arange(n) * 37 + 5) % 256).astype(np.uint8).reshape(1, n)
+    if fmt == "fp8":
+        codes[(codes & 0x7F) == 0x7F] = 0x10  # no E4M3 NaN codes
+    scales = np.array([[0xFF, 0x7F]], np.uint8)
+    v = oracle.decode(oracle.dequantize_cache_packed(codes, scales, fmt, B, C, "f32"), "f32")
+    assert np.isnan(v[0, :B]).all()
+    if fmt == "fp8":
+        want = torch.from_numpy(codes[0, B:].copy()).view(torch.float8_e4m3fn).double().numpy()
+    else:
+        tail = codes[0, B // 2:]
+        want = full_table()[np.stack([tail & 15, tail >> 4], axis=-1).reshape(-1)]
+    assert np.array_equal(v[0, B:], want)
+
+
 def test_packed_cache_codes_follow_the_element_casts():
     x = gen.kv_cache((1, 4, 128)).view(4, 128)
     bits = x.view(torch.int16).numpy().view(np.uint16)
