@@ -269,3 +269,10 @@ def test_plain_c_program_builds_against_the_header_and_links(tmp_path, L):
     assert out.returncode == 0, out.stderr
     assert out.stdout.split() == [str(EARG), str(ESHAPE), str(EARG), str(ESHAPE), str(ESHAPE),
                                   "MXQ_ERR_INVALID_ARG", "1", "16"]
+    # the same program as C++ (the header's extern "C" block) links the same symbols
+    exe_cc = tmp_path / "consumer_cc"
+    subprocess.check_call(["g++", "-x", "c++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), str(src), "-x", "none", "-L", libdir,
+                           "-lmxq", "-Wl,-rpath," + libdir, "-o", str(exe_cc)])
+    out_cc = subprocess.run([str(exe_cc)], capture_output=True, text=True, timeout=60)
+    assert out_cc.returncode == 0 and out_cc.stdout == out.stdout
