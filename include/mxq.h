@@ -156,24 +156,29 @@ int dequantize_cache_packed(const void* codes, const void* scales, int64_t rows,
  * ([MX] MXFP4GroupedMM forward and backward).
  *
  *  a        device, bf16 [T, Kin], rows grouped contiguously by expert,
- *           16-byte aligned.
+ *           aligned to 2 bytes (16 for the tensor-core path, below).
  *  packed   device, [E, N, K/2] bytes; scales device, [E, N, K/32] E8M0
  *           bytes: W_e[n][k] = dequantized value, exactly representable in
  *           bf16 for scale bytes <= 252.
- *  offs     device, int32 [E]: inclusive prefix sums of the expert row counts;
- *           expert e owns rows [offs[e-1], offs[e]) with offs[-1] = 0.
+ *  offs     device, int32 [E], 4-byte aligned: inclusive prefix sums of the
+ *           expert row counts; expert e owns rows [offs[e-1], offs[e]) with
+ *           offs[-1] = 0.
  *  transpose_w = 0 (forward):        Kin = K, y bf16 [T, N], y = a . W_e^T
  *  transpose_w = 1 (input gradient): Kin = N, y bf16 [T, K], y = a . W_e
  *  Products accumulate in fp32; y is rounded to bf16 (nearest-even).
- *  dev_status  device int32 (nullable).  If offs is not non-decreasing
+ *  dev_status  device int32 (nullable, 4-byte aligned).  If offs is not
+ *           non-decreasing
  *           with offs[E-1] == T the kernel writes MXQ_ERR_BAD_OFFS there and
  *           leaves y unwritten; if a pipeline wait gives up it writes
  *           MXQ_ERR_TIMEOUT.  The kernel never writes MXQ_OK: clear the word
  *           before the call to read it afterwards.
  *  Errors (host): K % 32 != 0, E < 1, N < 1, T < 0 -> MXQ_ERR_SHAPE; null
- *  pointers -> MXQ_ERR_INVALID_ARG.  The tensor-core path needs N and K
- *  multiples of 128 and 64 and 16-byte aligned a / y; other shapes run a
- *  slower general kernel. */
+ *  pointers -> MXQ_ERR_INVALID_ARG; a or y not on a 2-byte boundary, offs or
+ *  dev_status not on a 4-byte boundary -> MXQ_ERR_ALIGNMENT.  The
+ *  tensor-core path needs the output width (N, or K for the input gradient)
+ *  a multiple of 128, the reduction width a multiple of 64, and a, y and
+ *  packed 16-byte aligned; other valid calls run a slower general kernel
+ *  with the same results up to the order of the fp32 accumulation. */
 int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
                      int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                      int32_t* dev_status, void* stream);
@@ -189,7 +194,7 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
  *  y        device, bf16 [T, N]: y[t, n] = sum_k xq[t, k] W_e[n, k] with xq
  *           the dequantized activation; products are exact, the sum is
  *           accumulated in f32 by the tensor core and rounded once to bf16.
- *  Every pointer 16-byte aligned.
+ *  Every pointer 16-byte aligned, except offs and dev_status (4 bytes).
  *  Errors: K % 32 != 0, E < 1, N < 1, T < 0 -> MXQ_ERR_SHAPE; null ->
  *  MXQ_ERR_INVALID_ARG; misaligned -> MXQ_ERR_ALIGNMENT; K % 256 != 0 or
  *  N % 128 != 0 (shapes this kernel does not tile) -> MXQ_ERR_UNSUPPORTED.
@@ -208,7 +213,8 @@ int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void
  *  packed, block_scales  device, [E, N, K/2] and [E, N, K/16] bytes: each
  *           expert's weight in NVFP4 (e.g. nvfp4_quantize of W_e).
  *  w_global_scales  device, float [E]: each expert's g.
- *  offs, dev_status, y  as mxfp4_w4a4_grouped_mm.
+ *  offs, dev_status, y  as mxfp4_w4a4_grouped_mm; the two global-scale
+ *           pointers 4-byte aligned, every other pointer 16-byte aligned.
  *  y[t, n] = g_x g_w[e] sum_k (code * s_b)_x[t, k] (code * s_b)_w[n, k]: the
  *  tensor core multiplies codes and block scales exactly and accumulates in
  *  f32; the product of the two global scales multiplies the f32 sum, and y is
@@ -292,8 +298,11 @@ int nvfp4_quantize_mse(const void* x, int x_dtype, int64_t rows, int64_t K, void
  * workspace.  The scratch need does not grow with the input (16 bytes for
  * any shape); a build whose need exceeded MXQ_NOALLOC_SCRATCH_BYTES would
  * return MXQ_ERR_UNSUPPORTED.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress, with that device current);
- * make that first call before capturing the stream into a graph.  All calls
+ * array's device address (cudaGetSymbolAddress, with that device current)
+ * and keeps it for the life of the process; make that first call before
+ * capturing the stream into a graph.  Resetting a device (cudaDeviceReset)
+ * after that first call is not supported: the kept address would then be
+ * stale.  All calls
  * share the one array: the call clears it before use, and calls that overlap
  * on the GPU (for instance on two streams) race on it and must be
  * serialized by the caller.  Never allocates: no cudaMalloc, cudaFree or

@@ -76,6 +76,8 @@ static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 static bool elem_aligned(const void* p, int d) {
   return ((uintptr_t)p & (uintptr_t)((d == MXQ_F32 ? 4 : 2) - 1)) == 0;
 }
+// An int32 word (offs, a status word) sits on a 4-byte boundary; null passes.
+static bool word_aligned(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 static bool valid_dtype(int d) { return d == MXQ_BF16 || d == MXQ_F16 || d == MXQ_F32; }
 static int elem_bytes(int d) { return d == MXQ_F32 ? 4 : 2; }
 
@@ -218,6 +220,11 @@ int mxfp4_grouped_mm(const void* a, const void* packed, const void* scales, cons
   if (!a || !y) return MXQ_ERR_INVALID_ARG;
   if (!fits(T, N > K ? N : K) || !fits(E, N) || !fits(E * N, K)) return MXQ_ERR_SHAPE;
   if (E > 65536) return MXQ_ERR_UNSUPPORTED;
+  // bf16 elements on their own size, int32 words on theirs: the general
+  // kernel reads and writes them one element at a time.
+  if (!elem_aligned(a, MXQ_BF16) || !elem_aligned(y, MXQ_BF16) || !word_aligned(offs) ||
+      !word_aligned(dev_status))
+    return MXQ_ERR_ALIGNMENT;
   {
     const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
     if (!no_alias({{y, T * nout * 2}, {dev_status, 4}},
@@ -240,7 +247,7 @@ int mxfp4_w4a4_grouped_mm(const void* x_packed, const void* x_scales, const void
   if (K % 256 != 0 || N % 128 != 0 || T >= ((int64_t)1 << 31) || E * N >= ((int64_t)1 << 31))
     return MXQ_ERR_UNSUPPORTED;
   if (!aligned16(x_packed) || !aligned16(x_scales) || !aligned16(packed) || !aligned16(scales) ||
-      !aligned16(y))
+      !aligned16(y) || !word_aligned(offs) || !word_aligned(dev_status))
     return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{y, T * N * 2}, {dev_status, 4}},
                 {{x_packed, T * K / 2}, {x_scales, T * K / 32}, {packed, E * N * K / 2},
@@ -263,7 +270,8 @@ int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
   if (K % 256 != 0 || N % 128 != 0 || T >= ((int64_t)1 << 31) || E * N >= ((int64_t)1 << 31))
     return MXQ_ERR_UNSUPPORTED;
   if (!aligned16(x_packed) || !aligned16(x_block_scales) || !aligned16(packed) ||
-      !aligned16(block_scales) || !aligned16(y))
+      !aligned16(block_scales) || !aligned16(y) || !word_aligned(offs) ||
+      !word_aligned(dev_status) || !word_aligned(x_global_scale) || !word_aligned(w_global_scales))
     return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{y, T * N * 2}, {dev_status, 4}},
                 {{x_packed, T * K / 2}, {x_block_scales, T * K / 16}, {x_global_scale, 4},

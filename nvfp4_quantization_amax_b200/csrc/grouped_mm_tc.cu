@@ -717,14 +717,15 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                       int32_t* dev_status, cudaStream_t st) {
   const int64_t kin = transpose_w ? N : K, nout = transpose_w ? K : N;
-  // Weight loads by TMA (the input gradient, and the forward in pairs) need
-  // 16-byte aligned packed bytes and row coordinates below 2^31.
+  // Every tensor-core form reads the packed weights in 16-byte units (TMA
+  // tiles, or 16-byte loads in the single-CTA forward) and addresses weight
+  // rows with 32-bit TMA coordinates.
   const bool w_ok = ((uintptr_t)packed & 15) == 0 && E * N < (int64_t)1 << 31;
   const bool pair =
       nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2 && w_ok;
   const bool tc = kin % Geo<false>::kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
                   ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31 &&
-                  (w_ok || !transpose_w);
+                  w_ok;
   if (!tc)
     return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
                                      dev_status, st);

@@ -99,6 +99,13 @@ def test_grouped_mm_validation(L):
     assert f(A1, A2, A2, NULL, 8, 2, 16, 64, 0, A1, NULL, NULL) == EARG  # offs
     assert f(NULL, A2, A2, A2, 8, 2, 16, 64, 0, A1, NULL, NULL) == EARG  # a
     assert f(A1, A2, A2, A2, 0, 2, 16, 64, 0, A1, NULL, NULL) == OK  # T == 0: no-op
+    # bf16 a / y off their 2-byte boundary, int32 offs / status off 4 bytes:
+    # rejected on the host (the general kernel would fault on them)
+    Y, OFFS = ctypes.c_void_p(0x40000), ctypes.c_void_p(0x50000)
+    assert f(BAD, A2, A2, OFFS, 8, 2, 16, 64, 0, Y, NULL, NULL) == EALIGN
+    assert f(A1, A2, A2, OFFS, 8, 2, 16, 64, 1, BAD, NULL, NULL) == EALIGN
+    assert f(A1, A2, A2, ctypes.c_void_p(0x50002), 8, 2, 16, 64, 0, Y, NULL, NULL) == EALIGN
+    assert f(A1, A2, A2, OFFS, 8, 2, 16, 64, 0, Y, ctypes.c_void_p(0x60002), NULL) == EALIGN
 
 
 def test_binding_fails_loudly_without_gpu():
@@ -181,6 +188,8 @@ def test_w4a4_validation(L):
     assert f(A1, A1, A2, A2, A2, 8, 2, 128, 96, A1, NULL, NULL) == EUNSUP  # K % 256
     assert f(A1, A1, A2, A2, A2, 8, 2, 64, 256, A1, NULL, NULL) == EUNSUP  # N % 128
     assert f(BAD, A1, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
+    assert f(A1, A1, A2, A2, ctypes.c_void_p(0x20002), 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
+    assert f(A1, A1, A2, A2, A2, 8, 2, 128, 256, A1, ctypes.c_void_p(0x60001), NULL) == EALIGN
     assert f(A1, A1, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK  # T == 0
 
 
@@ -192,6 +201,10 @@ def test_nvfp4_w4a4_validation(L):
     assert f(A1, A1, NULL, A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EARG  # x scale
     assert f(A1, A1, A2, A2, A2, A2, A2, 8, 2, 128, 96, A1, NULL, NULL) == EUNSUP
     assert f(BAD, A1, A2, A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL, NULL) == EALIGN
+    assert f(A1, A1, ctypes.c_void_p(0x20001), A2, A2, A2, A2, 8, 2, 128, 256, A1, NULL,
+             NULL) == EALIGN  # x global scale
+    assert f(A1, A1, A2, A2, A2, A2, ctypes.c_void_p(0x20006), 8, 2, 128, 256, A1, NULL,
+             NULL) == EALIGN  # offs
     assert f(A1, A1, A2, A2, A2, A2, A2, 0, 2, 128, 256, A1, NULL, NULL) == OK
 
 
