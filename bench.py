@@ -378,14 +378,23 @@ def run_gpu(args, rank, world):
     e2e_dt, h2d, d2h = time_e2e(torch, mxq, step, max(1, min(args.steps, 3)))
     e2e_dt = max_over_ranks([e2e_dt], dev)[0]
     next_ms = time_next_rows(torch, mxq, step, dev)
+    extra = {}
+    if world == 1:
+        # the small-workload latency and the mixed-block sweep, outside the
+        # timed step (the sweep needs ~68 GB, so the step's tensors go first)
+        extra["config1_latency"] = time_config1(torch, mxq, gen, dev)
+        del step
+        torch.cuda.empty_cache()
+        if not args.no_sweep:
+            extra["sweep"] = time_sweep(torch, mxq, gen, dev, args.sweep_max_log2)
 
     if rank == 0:
-        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary(), next_ms)
+        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary(), next_ms, extra)
     if world > 1:
         dist.destroy_process_group()
 
 
-def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=None):
+def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=None, extra=None):
     peaks, peak_src = load_peaks()
     ab = algorithmic_bytes()
     qd_bytes = ab["mx_quantize"] + ab["mx_dequantize"] + 3 * ab["quantize_cache"]
@@ -484,6 +493,8 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
                 "includes": "nvfp4_quantize of the activations (two passes) + the block-scaled GEMM",
                 "workload": "x bf16 [32768,7168], W NVFP4 [32,2048,7168], multinomial counts"}
         line["next_rows"] = rows
+    if extra:
+        line.update(extra)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     print(json.dumps(line), flush=True)
@@ -491,18 +502,50 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
 
 # ------------------------------------------------------ CPU oracle arm
 
+def host_cpu():
+    """Host cores this process may use and the CPU model, read at run time."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return int(cores or 1), model
+
+
+def sampled_rows(offs, per_expert=16, seed=8):
+    """Every expert's first and last row plus `per_expert` seeded rows."""
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    starts = np.concatenate([[0], offs[:-1]])
+    rows = []
+    for lo, hi in zip(starts, offs):
+        if hi > lo:
+            rows += [lo, hi - 1] + list(rng.integers(lo, hi, per_expert))
+    return np.unique(np.array(rows, np.int64))
+
+
 def cpu_baseline(budget_s):
-    """The scalar oracle, as it stands, on a bounded sample of the same
-    workload (single thread).  Returns GB/s over the same algorithmic bytes
-    per element as the GPU metric, plus the oracle's grouped-GEMM GFLOP/s."""
+    """The scalar oracle, as it stands, timed on the host cores on bounded
+    samples of the same workload: single-threaded, and the same source built
+    with OpenMP on every core this process may use.  GB/s over the same
+    algorithmic bytes per element as the GPU metric; the grouped GEMM as
+    GFLOP/s of the exact double sums over every expert's first and last row
+    plus 16 seeded rows (the oracle dequantizes each expert it touches)."""
     import numpy as np
     import torch
 
     import oracle
     import synthetic as gen
 
-    per = max(budget_s / 4.0, 0.5)
-    done = {}
+    cores, model = host_cpu()
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"  # input generation only
+    per = max(budget_s / 8.0, 0.4)
 
     def timed(fn, bytes_per_call):
         n, t0 = 0, time.perf_counter()
@@ -513,61 +556,103 @@ def cpu_baseline(budget_s):
             if dt >= per:
                 return n * bytes_per_call, dt, n
 
-    W = gen.expert_weights(1, 16, 7168).view(16, 7168)
-    wb = W.view(torch.int16).numpy().view(np.uint16)
-    pk, sc = oracle.mx_quantize(wb)
-    kv = gen.kv_cache((1, 64, 512)).view(64, 512).view(torch.int16).numpy().view(np.uint16)
-    e_w = 16 * 7168
-    b1, t1, n1 = timed(lambda: oracle.mx_quantize(wb), e_w * 2 + e_w // 2 + e_w // 32)
-    b2, t2, n2 = timed(lambda: oracle.mx_dequantize(pk, sc), e_w // 2 + e_w // 32 + e_w * 2)
-    e_kv = 64 * 512
+    def bf16_bits(t):
+        return t.cpu().view(torch.int16).numpy().view(np.uint16)
 
-    def qc():
-        for f, b in CACHE_RUNS:
-            oracle.quantize_cache(kv, f, b)
-    b3, t3, n3 = timed(qc, 3 * e_kv * 4)
-    done["gbs"] = (b1 + b2 + b3) / (t1 + t2 + t3) / 1e9
-    # grouped GEMM: 2 rows of one expert, forward (includes dequantizing W_e)
-    Wg = gen.expert_weights(1, 256, 7168, workload=5)
-    pg, sg = oracle.mx_quantize(Wg.view(torch.int16).numpy().view(np.uint16))
-    pg, sg = pg.reshape(1, 256, 3584), sg.reshape(1, 256, 224)
-    a = gen.normal_bf16(3, (8, 7168)).view(torch.int16).numpy().view(np.uint16)
-    offs = np.array([8], np.int32)
+    def quant_dequant_cache(w_rows, kv_rows):
+        W = gen.expert_weights(1, w_rows, 7168).view(w_rows, 7168)
+        wb = bf16_bits(W)
+        pk, sc = oracle.mx_quantize(wb)
+        kv = bf16_bits(gen.kv_cache((1, kv_rows, 512)).view(kv_rows, 512))
+        e_w, e_kv = w_rows * 7168, kv_rows * 512
+        b1, t1, n1 = timed(lambda: oracle.mx_quantize(wb), e_w * 2 + e_w // 2 + e_w // 32)
+        b2, t2, n2 = timed(lambda: oracle.mx_dequantize(pk, sc), e_w // 2 + e_w // 32 + e_w * 2)
+
+        def qc():
+            for f, b in CACHE_RUNS:
+                oracle.quantize_cache(kv, f, b)
+        b3, t3, n3 = timed(qc, 3 * e_kv * 4)
+        return (b1 + b2 + b3) / (t1 + t2 + t3) / 1e9, (n1, n2, n3), t1 + t2 + t3
+
+    gbs1, n_1, t_1 = quant_dequant_cache(16, 64)
+    with oracle.all_cores():
+        gbs_all, n_all, t_all = quant_dequant_cache(max(16, 8 * cores), max(64, 32 * cores))
+
+    # grouped GEMM forward on the benchmark's inputs (W packed by the oracle)
+    counts = gen.expert_counts(T, E).numpy()
+    offs = np.cumsum(counts).astype(np.int32)
+    rows = sampled_rows(offs)
+    W5 = gen.expert_weights(E, N, K, device=gen_dev, workload=5)
+    with oracle.all_cores():
+        p5, s5 = oracle.mx_quantize(bf16_bits(W5.view(E * N, K)))
+    del W5
+    p5, s5 = p5.reshape(E, N, K // 2), s5.reshape(E, N, K // 32)
+    a = bf16_bits(gen.normal_bf16(gen.seed_for(5, 3), (T, K), device=gen_dev))
+    first = rows[rows < offs[0]]  # one expert's rows, single-threaded
     t0 = time.perf_counter()
-    oracle.grouped_mm(a, pg, sg, offs, rows=np.arange(8))
-    gdt = time.perf_counter() - t0
-    done["gemm_gflops"] = 2.0 * 8 * 256 * 7168 / gdt / 1e9
-    return {"value": round(done["gbs"], 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "gemm_gflops": round(done["gemm_gflops"], 4),
-            "sample": ("mx_quantize %dx and mx_dequantize %dx of [16,7168] weight rows, "
-                       "quantize_cache (3 formats) %dx of [64,512] KV rows, ~%.0f s total; "
-                       "GEMM: 8 rows x 256 outputs x 7168" % (n1, n2, n3, t1 + t2 + t3))}
+    oracle.grouped_mm(a, p5, s5, offs, rows=first)
+    g1 = 2.0 * first.size * N * K / (time.perf_counter() - t0) / 1e9
+    with oracle.all_cores():
+        t0 = time.perf_counter()
+        oracle.grouped_mm(a, p5, s5, offs, rows=rows)
+        g_all = 2.0 * rows.size * N * K / (time.perf_counter() - t0) / 1e9
+    return {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "gbs_all_cores": round(gbs_all, 4), "cores_all": cores, "cpu_model": model,
+            "gemm_gflops": round(g1, 4), "gemm_rows": int(first.size),
+            "gemm_gflops_all_cores": round(g_all, 4), "gemm_rows_all_cores": int(rows.size),
+            "sample": ("single thread: mx_quantize %dx and mx_dequantize %dx of [16,7168] weight "
+                       "rows, quantize_cache (3 formats) %dx of [64,512] KV rows, %.1f s; "
+                       "all %d cores (OpenMP build of the same source): %dx/%dx of [%d,7168] and "
+                       "%dx of [%d,512], %.1f s; grouped GEMM forward of the benchmark inputs "
+                       "(T=32768, E=32, N=2048, K=7168): first and last row plus 16 seeded rows "
+                       "per expert (%d rows) on all cores, expert 0's %d of them single-threaded"
+                       % (n_1[0], n_1[1], n_1[2], t_1, cores, n_all[0], n_all[1],
+                          max(16, 8 * cores), n_all[2], max(64, 32 * cores), t_all,
+                          rows.size, first.size))}
 
 
-def run_sweep(args):
+def time_config1(torch, mxq, gen, dev, reps=20):
+    """Latency of the small MXFP4 workload (bf16 [64,256] with its four forced
+    rows): mx_quantize and mx_dequantize, microseconds, median of `reps`
+    calls after 5 warm-up calls, L2 flushed before each call."""
+    x = gen.mx_small(dev)
+    p, s = mxq.mx_quantize(x)
+    y = torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, fn in (("mx_quantize", lambda: mxq.mx_quantize(x, p, s)),
+                     ("mx_dequantize", lambda: mxq.mx_dequantize(p, s, torch.bfloat16, y))):
+        for _ in range(5):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        out[name] = round(statistics.median(ts), 2)
+    return {"unit": "us", "workload": "bf16 [64,256], 4 forced rows",
+            "timing": "median of %d, L2 flushed before each call" % reps, **out}
+
+
+def time_sweep(torch, mxq, gen, dev, max_log2=21):
     """Bandwidth sweep over row counts of the mixed-block workload x bf16
     [R, 7168] (normal, subnormal-range, zero and single-spike 32-blocks):
     mx_quantize, mx_dequantize and quantize_cache in the three formats, device
     time per call (CUDA events, median of 5 after 2 warm-up calls; L2 is
-    flushed before each timed call).  Prints one JSON line."""
-    import torch
-
-    import nvfp4_quantization_amax_b200 as mxq
-    import synthetic as gen
-
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
+    flushed before each timed call).  R = 2^10, 2^12, ..., 2^20, 2^21."""
     C = 7168
-    r_max = 1 << min(args.sweep_max_log2, 21)
+    r_max = 1 << max_log2
     x = gen.mixed_blocks(r_max, C, device=dev)
     out = torch.empty_like(x)
     packed = torch.empty((r_max, C // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((r_max, C // 32), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     rows_out = []
-    logs = list(range(10, min(args.sweep_max_log2, 20) + 1, 2))
-    if args.sweep_max_log2 >= 21:
-        logs.append(21)
+    logs = sorted(set(list(range(10, min(max_log2, 20) + 1, 2)) + [max_log2]))
     for lg in logs:
         R = 1 << lg
         xr, outr, pr, sr = x[:R], out[:R], packed[:R], scales[:R]
@@ -596,15 +681,29 @@ def run_sweep(args):
             ms = sorted(ts)[2]
             row[name] = {"ms": round(ms, 4), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
         rows_out.append(row)
-    print(json.dumps({"sweep": "mixed blocks bf16 [R, 7168]", "peak_hbm_gbs":
-                      load_peaks()[0]["hbm_gbs"], "rows": rows_out}), flush=True)
+    del x, out, packed, scales, flush
+    torch.cuda.empty_cache()
+    return {"workload": "mixed blocks bf16 [R, 7168]", "unit": "GB/s",
+            "timing": "median of 5, L2 flushed before each call", "rows": rows_out}
+
+
+def run_sweep(args):
+    """The mixed-block sweep alone, as one JSON line."""
+    import torch
+
+    import nvfp4_quantization_amax_b200 as mxq
+    import synthetic as gen
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sw = time_sweep(torch, mxq, gen, dev, min(args.sweep_max_log2, 21))
+    sw["peak_hbm_gbs"] = load_peaks()[0]["hbm_gbs"]
+    print(json.dumps(sw), flush=True)
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; the loop keeps the contract's shape
     cb = cpu_baseline(max(4.0, min(30.0, 2.0 * args.steps)))
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -612,7 +711,8 @@ def run_reference(args, rank, world):
             "data": "synthetic",
             "config": {"workload": WORKLOAD,
                        "sample": "each step times the scalar CPU oracle on a bounded sample of "
-                                 "this workload (rows of the same tensors), single thread"},
+                                 "this workload (rows of the same tensors), single thread; "
+                                 "cpu_baseline also gives the all-core figures"},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -629,7 +729,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the step: the mixed-block bandwidth sweep over row counts")
-    ap.add_argument("--sweep-max-log2", type=int, default=20)
+    ap.add_argument("--sweep-max-log2", type=int, default=21, choices=range(10, 22))
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave the mixed-block sweep out of the default run")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

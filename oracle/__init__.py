@@ -8,6 +8,7 @@ this module only moves numpy arrays in and out of it.
 Arrays of floating-point elements are passed as their raw bit patterns:
 uint16 for bf16 / f16, uint32 for f32.
 """
+import contextlib
 import ctypes
 import os
 
@@ -19,7 +20,8 @@ DTYPES = {"bf16": 0, "f16": 1, "f32": 2}
 FORMATS = {"fp8": 0, "mxfp4": 1, "nvfp4": 2}
 _BITS = {"bf16": np.uint16, "f16": np.uint16, "f32": np.uint32}
 
-_lib = None
+_libs = {}
+_all_cores = False
 
 # An already-built oracle library to load instead of oracle/liboracle.so: the
 # mutation tests point it at copies of the oracle with a planted mistake and
@@ -27,10 +29,21 @@ _lib = None
 LIB_ENV = "MXQ_ORACLE_LIB"
 
 
+@contextlib.contextmanager
+def all_cores():
+    """Within the block, calls use the OpenMP build of the same oracle
+    source, whose row loops run on all host cores (identical results)."""
+    global _all_cores
+    prev, _all_cores = _all_cores, True
+    try:
+        yield
+    finally:
+        _all_cores = prev
+
+
 def lib():
-    global _lib
-    if _lib is None:
-        path = os.environ.get(LIB_ENV) or _build.build()
+    path = os.environ.get(LIB_ENV) or _build.build(openmp=_all_cores)
+    if path not in _libs:
         L = ctypes.CDLL(path)
         d, i, i64, p = ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
         L.orc_e2m1_value.restype = d
@@ -90,8 +103,8 @@ def lib():
         L.orc_nvfp4_w4a4_grouped_mm.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, i64, p]
         L.orc_grouped_mm.restype = i
         L.orc_grouped_mm.argtypes = [p, p, p, p, i64, i64, i64, i64, i, p, i64, p]
-        _lib = L
-    return _lib
+        _libs[path] = L
+    return _libs[path]
 
 
 def _ptr(a):

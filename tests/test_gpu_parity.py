@@ -258,8 +258,9 @@ def test_grouped_mm_ragged_experts(transpose_w):
 
 
 @pytest.mark.parametrize("transpose_w", [False, True])
-def test_grouped_mm_scales_across_decoder_paths(transpose_w):
-    # scale bytes 136..150 straddle the two weight-decoding paths (<= 142 and above)
+def test_grouped_mm_scales_above_the_benchmark_range(transpose_w):
+    # scale bytes 136..150: larger weights than the benchmark's (the whole
+    # 0..252 range is covered per expert in test_gpu_gemm_edges.py)
     check_gemm([129, 64, 300], N=256, K=256, transpose_w=transpose_w, scale_lo=136,
                scale_hi=150)
 
