@@ -266,7 +266,103 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
         out[name] = sum(a.elapsed_time(b) for a, b in ev) / reps
     names = list(out)
     vals = max_over_ranks([out[n] for n in names], dev)
-    return dict(zip(names, vals))
+    times = dict(zip(names, vals))
+    # work of the mse sweep: evaluations of expert 0's blocks under the
+    # tensor's g (the same i.i.d. weights in every expert)
+    blocks0 = W_SHAPE[1] * W_SHAPE[2] // 16
+    times["_mse_evals_per_block"] = mse_evaluations(torch, step.W[0], float(g2.item())) / blocks0
+    return times
+
+
+E4M3_POS_CODES = 126  # positive finite E4M3 bytes 0x01 .. 0x7E
+
+
+def mse_evaluations(torch, w, g, lanes=4):
+    """(candidate, weight) evaluations the mse-rule kernel performs on the
+    16-blocks of w (bf16 [rows, K]) under the global scale g, replaying its
+    pruning (the measurement's work unit, not a result): each block's codes
+    are visited from the top (the first code whose quotient amax / d_c is at
+    most 0.25, by binary search, else 126) downwards, `lanes` interleaved
+    slots each stopping at the first code whose d underflows to 0 or whose
+    clipping error (amax - 6 d)^2 alone exceeds the slot's best sum so far.
+    Each visit evaluates 16 weights.  Error sums are formed in float64 from
+    float32 quotients as in the kernel; a sum that differs from the kernel's
+    in its last bits can move a stop by one code, so the count is exact up to
+    such margins."""
+    f32, f64 = torch.float32, torch.float64
+    dev = w.device
+    x = w.reshape(-1, 16).to(f32)
+    ax = x.abs()
+    amax = ax.amax(1)
+    codes = torch.arange(E4M3_POS_CODES + 1, device=dev)
+    # E4M3 value of each code byte: exponent field (bits 3-6), mantissa bits 0-2
+    e, m = (codes >> 3) & 15, codes & 7
+    s_c = torch.where(e == 0, m.to(f32) * 2.0 ** -9, (1.0 + m.to(f32) / 8.0) * torch.pow(
+        torch.tensor(2.0, device=dev), (e - 7).to(f32)))
+    d_c = (s_c * torch.tensor(g, dtype=f32, device=dev)).to(f32)
+
+    def all_zero(c):
+        dc = d_c[c]
+        return (dc != 0) & ((amax / dc) <= 0.25)
+    # c_top: binary search for the first all-zero code where code 126 is all-zero
+    lo = torch.ones_like(amax, dtype=torch.int64)
+    hi = torch.full_like(lo, E4M3_POS_CODES)
+    top_zero = all_zero(hi)
+    for _ in range(8):
+        mid = (lo + hi) >> 1
+        z = all_zero(mid)
+        hi = torch.where(z & (lo < hi), mid, hi)
+        lo = torch.where(~z & (lo < hi), mid + 1, lo)
+    c_top = torch.where(top_zero, lo, torch.full_like(lo, E4M3_POS_CODES))
+    mids = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=f32, device=dev)
+    table = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=f64, device=dev)
+    amax64, ax64 = amax.to(f64), ax.to(f64)
+    total = 0
+    for slot in range(lanes):
+        best = torch.full_like(amax64, float("inf"))
+        alive = torch.ones_like(amax, dtype=torch.bool)
+        for k in range(E4M3_POS_CODES):
+            c = c_top - slot - lanes * k
+            alive &= c >= 1
+            if not bool(alive.any()):
+                break
+            cc = c.clamp(min=1)
+            d = d_c[cc]
+            alive &= d != 0
+            t = amax64 - 6.0 * d.to(f64)
+            alive &= ~((t > 0) & (t * t * (1.0 - 2.0 ** -40) > best))
+            total += int(alive.sum()) * 16
+            v = ax / d[:, None]
+            idx = torch.bucketize(v, mids)
+            idx += ((v == 0.75) | (v == 1.75) | (v == 3.5)).to(idx.dtype)
+            err = ((table[idx] * d.to(f64)[:, None] - ax64) ** 2).sum(1)
+            better = alive & (err <= best)
+            best = torch.where(better, err, best)
+    return total
+
+
+def mse_roofline(evals_s, clocks):
+    """Issue-rate roofline of the mse sweep.  Unit: one (candidate, weight)
+    evaluation.  The kernel's thread instructions per evaluation come from
+    an ncu count (profiles/mse_issue.json: smsp__thread_inst_executed.sum of
+    one launch over the evaluations the replay counts for that launch); the
+    peak is every SM sub-partition issuing one full warp instruction per
+    clock: 148 x 4 x 32 thread instructions per cycle at the SM clock
+    sampled during the benchmark."""
+    path = os.path.join(ROOT, "profiles", "mse_issue.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        prof = json.load(f)
+    if prof.get("source_sha") != source_hash("nvfp4_mse.cu"):
+        return None
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    per_eval = prof["thread_inst_per_eval"]
+    peak = 148 * 4 * 32 * mhz * 1e6 / per_eval
+    return {"bound": "issue", "unit": "G evaluations/s", "achieved": round(evals_s / 1e9, 2),
+            "peak": round(peak / 1e9, 2), "frac": round(evals_s / peak, 4),
+            "thread_inst_per_eval": per_eval, "sm_mhz": mhz,
+            "peak_source": "148 SMs x 4 schedulers x 32 lanes per clock"}
 
 
 def next_row_bytes():
@@ -462,6 +558,7 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         "clocks": clocks,
     }
     if next_ms:
+        evals_per_block = next_ms.pop("_mse_evals_per_block", None)
         nb = next_row_bytes()
         w = W_SHAPE[0] * W_SHAPE[1] * W_SHAPE[2]
         rows = {}
@@ -473,10 +570,16 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
                        "frac": round(gbs / peaks["hbm_gbs"], 4),
                        "workload": ("bf16 [64,2048,7168] expert weights" if n.startswith("nvfp4")
                                     else "bf16 [4,8192,512] KV cache")}
-        # the sweep is arithmetic: 126 candidate scales x 16 weights per block
-        rows["nvfp4_quantize_mse"]["bound"] = "alu"
-        rows["nvfp4_quantize_mse"]["g_candidates_per_s"] = round(
-            126 * w / (next_ms["nvfp4_quantize_mse"] * 1e-3) / 1e9, 1)
+        # the sweep is arithmetic: at most 126 candidate scales x 16 weights
+        # per block, of which the kernel evaluates only those that can win
+        mse = rows["nvfp4_quantize_mse"]
+        mse["bound"] = "issue"
+        mse["g_candidates_per_s"] = round(126 * w / (next_ms["nvfp4_quantize_mse"] * 1e-3) / 1e9, 1)
+        if evals_per_block is not None:
+            evals_s = evals_per_block * (w // 16) / (next_ms["nvfp4_quantize_mse"] * 1e-3)
+            mse["evaluations_per_block"] = round(evals_per_block, 3)
+            mse["g_evaluations_per_s"] = round(evals_s / 1e9, 2)
+            mse["roofline"] = mse_roofline(evals_s, clocks)
         if w4 is not None:
             # fp4 peak: the measured bf16 burst x the nominal fp4 / bf16 ratio (9 / 2.25)
             tf = gemm_flops() / (w4 * 1e-3) / 1e12

@@ -317,6 +317,27 @@ int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, 
  * to launches made after the call.  Returns the previous limit. */
 uint64_t mxq_set_wait_limit_ns(uint64_t ns);
 
+/* Debug variant of the library (libmxq_debug.so, the same sources built
+ * with MXQ_DEBUG_CHECKS; no counterpart on the source pages).  There every
+ * kernel tests the element index of each global-memory access (and each
+ * indexed shared-memory store of the GEMM epilogues and weight decode)
+ * against the extent the launch was given; a failed test records the check
+ * id, the index and the extent, and the access is skipped, so nothing traps
+ * and no out-of-range address is touched.
+ *
+ * mxq_debug_checks: record (host, int64_t[3]) = {check id, index, extent} of
+ *   the first failed check since the previous call, or zeros; the record is
+ *   then cleared.  Synchronizes with the device (it copies the records
+ *   back).  Returns MXQ_OK in the debug variant, MXQ_ERR_UNSUPPORTED (record
+ *   zeroed) in the normal library; null record -> MXQ_ERR_INVALID_ARG.
+ * mxq_debug_selftest: launches one checked store one element past the
+ *   extent it declares into dev_words (device, two int32, 4-byte aligned;
+ *   the store would land in the second word, which the check must leave
+ *   untouched), so that the next mxq_debug_checks returns {99, 1, 1}.
+ *   MXQ_ERR_UNSUPPORTED (no launch) in the normal library. */
+int mxq_debug_checks(int64_t* record);
+int mxq_debug_selftest(int32_t* dev_words, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* mxq_status_string(int status);
 

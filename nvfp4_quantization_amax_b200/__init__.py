@@ -14,6 +14,8 @@ results are copied back to host memory before the call returns.
 from ._abi import (  # noqa: F401
     CacheQuantization,
     MxqError,
+    debug_checks,
+    debug_selftest,
     lib,
     lib_path,
     mx_dequantize,

@@ -19,18 +19,25 @@ class MxqError(RuntimeError):
         self.status = status
 
 
+# Load another build of the library instead of libmxq.so (the debug variant,
+# libmxq_debug.so, built with `python -m nvfp4_quantization_amax_b200.build
+# --debug`).
+LIB_ENV = "MXQ_LIBRARY"
+
+
 def lib_path():
-    return _LIB_PATH
+    return os.environ.get(LIB_ENV) or _LIB_PATH
 
 
 def lib():
     """Load libmxq.so (built in-tree by nvfp4_quantization_amax_b200.build)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(_LIB_PATH):
-            raise RuntimeError("libmxq.so not found at %s; build it with "
-                               "`python -m nvfp4_quantization_amax_b200.build`" % _LIB_PATH)
-        L = ctypes.CDLL(_LIB_PATH)
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError("%s not found; build it with "
+                               "`python -m nvfp4_quantization_amax_b200.build`" % path)
+        L = ctypes.CDLL(path)
         i, i32, i64, p = ctypes.c_int, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
         L.mx_quantize.restype = i
         L.mx_quantize.argtypes = [p, i, i64, i64, p, p, p]
@@ -44,6 +51,10 @@ def lib():
         L.mxq_status_string.argtypes = [i]
         L.mxq_version.restype = i
         L.mxq_version.argtypes = []
+        L.mxq_debug_checks.restype = i
+        L.mxq_debug_checks.argtypes = [p]
+        L.mxq_debug_selftest.restype = i
+        L.mxq_debug_selftest.argtypes = [p, p]
         L.nvfp4_quantize.restype = i
         L.nvfp4_quantize.argtypes = [p, i, i64, i64, p, p, p, p, p]
         L.nvfp4_quantize_mse.restype = i
@@ -68,6 +79,22 @@ def lib():
 
 def status_string(status):
     return lib().mxq_status_string(int(status)).decode()
+
+
+def debug_checks():
+    """(check id, index, extent) of the first failed index check since the
+    previous call, or None; only the debug variant of the library has checks
+    (the normal one raises MxqError with MXQ_ERR_UNSUPPORTED)."""
+    rec = (ctypes.c_int64 * 3)()
+    _check(lib().mxq_debug_checks(ctypes.cast(rec, ctypes.c_void_p)), "mxq_debug_checks")
+    return None if rec[0] == 0 else (int(rec[0]), int(rec[1]), int(rec[2]))
+
+
+def debug_selftest(words):
+    """Launch the debug variant's self-test into `words` (device int32 [2])."""
+    if not (words.is_cuda and words.dtype == torch.int32 and words.numel() >= 2):
+        raise ValueError("debug_selftest needs a device int32 tensor of 2 words")
+    _check(lib().mxq_debug_selftest(_ptr(words), _stream(words.device)), "mxq_debug_selftest")
 
 
 def set_wait_limit_ns(ns):

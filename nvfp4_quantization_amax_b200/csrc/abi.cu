@@ -10,9 +10,19 @@
 #include <tuple>
 
 #include "mxq.h"
+#include "mxq_device.cuh"
 #include "mxq_launch.h"
 
 namespace mxq {
+
+// Debug variant: a checked store one element past the extent it was given
+// (the caller's buffer holds two words, so even an unchecked store would
+// stay inside it).  The check records (kChkSelfTest, 1, 1) and skips it.
+__global__ void debug_selftest_kernel(int32_t* words) {
+  if (MXQ_IN_RANGE(kChkSelfTest, 1, 1)) words[1] = 1;
+}
+
+MXQ_DEFINE_CHECK_READER(check_record_abi)
 
 int num_sms() {
   static std::mutex mu;
@@ -362,6 +372,41 @@ const char* mxq_status_string(int status) {
     case MXQ_ERR_TIMEOUT: return "MXQ_ERR_TIMEOUT";
     default: return "MXQ_ERR_UNKNOWN";
   }
+}
+
+int mxq_debug_checks(int64_t* record) {
+  if (!record) return MXQ_ERR_INVALID_ARG;
+  record[0] = record[1] = record[2] = 0;
+#ifdef MXQ_DEBUG_CHECKS
+  using Reader = int (*)(unsigned long long*);
+  const Reader readers[] = {check_record_abi,         check_record_elementwise,
+                            check_record_cache_packed, check_record_nvfp4,
+                            check_record_nvfp4_mse,    check_record_grouped_mm_general,
+                            check_record_grouped_mm_tc, check_record_w4a4};
+  int status = MXQ_OK;
+  for (Reader rd : readers) {
+    unsigned long long r[3];
+    const int rc = rd(r);
+    if (rc != MXQ_OK) status = rc;
+    else if (r[0] != 0 && record[0] == 0)
+      for (int i = 0; i < 3; ++i) record[i] = (int64_t)r[i];
+  }
+  return status;
+#else
+  return MXQ_ERR_UNSUPPORTED;
+#endif
+}
+
+int mxq_debug_selftest(int32_t* dev_words, void* stream) {
+  if (!dev_words) return MXQ_ERR_INVALID_ARG;
+  if (((uintptr_t)dev_words & 3) != 0) return MXQ_ERR_ALIGNMENT;
+#ifdef MXQ_DEBUG_CHECKS
+  debug_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(dev_words);
+  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+#else
+  (void)stream;
+  return MXQ_ERR_UNSUPPORTED;
+#endif
 }
 
 uint64_t mxq_set_wait_limit_ns(uint64_t ns) { return set_wait_limit_ns(ns); }

@@ -149,7 +149,7 @@ pack_cache_kernel(const void* __restrict__ in, void* __restrict__ codes,
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
-      if (item < n_items) load8<DT>(in, item, bits[u]);
+      if (item < n_items && MXQ_IN_RANGE(kChkPackIn, item, n_items)) load8<DT>(in, item, bits[u]);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -167,8 +167,10 @@ pack_cache_kernel(const void* __restrict__ in, void* __restrict__ codes,
       float x[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) x[j] = elem_to_f32<DT>(bits[u][j]);
-      store_codes<FMT>(codes, item, encode8<FMT>(x, exp2i(-k)));
-      if ((lane & (LPB - 1)) == 0) scales[item / LPB] = (uint8_t)scale_byte<FMT>(k);
+      if (MXQ_IN_RANGE(kChkPackOut, item, n_items))
+        store_codes<FMT>(codes, item, encode8<FMT>(x, exp2i(-k)));
+      if ((lane & (LPB - 1)) == 0 && MXQ_IN_RANGE(kChkPackScale, item / LPB, n_items / LPB))
+        scales[item / LPB] = (uint8_t)scale_byte<FMT>(k);
     }
   }
 }
@@ -186,8 +188,11 @@ unpack_cache_kernel(const void* __restrict__ codes, const uint8_t* __restrict__ 
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t item = base + u * stride;
       if (item < n_items) {
-        c[u] = load_codes<FMT>(codes, item);
-        sb[u] = __ldg(scales + item / LPB);
+        c[u] = MXQ_IN_RANGE(kChkUnpackIn, item, n_items) ? load_codes<FMT>(codes, item)
+                                                         : make_uint2(0u, 0u);
+        sb[u] = MXQ_IN_RANGE(kChkUnpackScale, item / LPB, n_items / LPB)
+                    ? (uint32_t)__ldg(scales + item / LPB)
+                    : 0u;
       }
     }
 #pragma unroll
@@ -196,7 +201,7 @@ unpack_cache_kernel(const void* __restrict__ codes, const uint8_t* __restrict__ 
       if (item >= n_items) continue;
       float v[8];
       decode8<FMT>(c[u], scale_value<FMT>(sb[u]), v);
-      store8<DT>(out, item, v);
+      if (MXQ_IN_RANGE(kChkUnpackOut, item, n_items)) store8<DT>(out, item, v);
     }
   }
 }
@@ -222,20 +227,26 @@ pack_cache_general_kernel(const void* __restrict__ in, uint8_t* __restrict__ cod
   for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < n_groups;
        g += (int64_t)gridDim.x * kThreads) {
     const int64_t c0 = g * B;  // groups never straddle rows (channels % B == 0)
+    [[maybe_unused]] const int64_t n_el = n_groups * B;
+    auto elem = [&](int64_t i) {
+      return MXQ_IN_RANGE(kChkPackIn, i, n_el) ? elem_bits_at<DT>(in, i) : 0u;
+    };
     uint32_t m = 0;
-    for (int c = 0; c < B; ++c) m = max(m, mag_as_f32_bits<DT>(elem_bits_at<DT>(in, c0 + c)));
+    for (int c = 0; c < B; ++c) m = max(m, mag_as_f32_bits<DT>(elem(c0 + c)));
     const int k = group_scale_exp<FMT>(m);
     const float inv = exp2i(-k);
-    scales[g] = (uint8_t)scale_byte<FMT>(k);
+    if (MXQ_IN_RANGE(kChkPackScale, g, n_groups)) scales[g] = (uint8_t)scale_byte<FMT>(k);
     for (int c = 0; c < B; c += 2) {
-      const float a = elem_to_f32<DT>(elem_bits_at<DT>(in, c0 + c));
-      const float b = c + 1 < B ? elem_to_f32<DT>(elem_bits_at<DT>(in, c0 + c + 1)) : 0.0f;
+      const float a = elem_to_f32<DT>(elem(c0 + c));
+      const float b = c + 1 < B ? elem_to_f32<DT>(elem(c0 + c + 1)) : 0.0f;
       if constexpr (FMT == MXQ_FMT_FP8) {
         const uint32_t two = e4m3x2(a * inv, b * inv);
-        codes[c0 + c] = (uint8_t)two;
-        if (c + 1 < B) codes[c0 + c + 1] = (uint8_t)(two >> 8);
+        if (MXQ_IN_RANGE(kChkPackOut, c0 + c, n_el)) codes[c0 + c] = (uint8_t)two;
+        if (c + 1 < B && MXQ_IN_RANGE(kChkPackOut, c0 + c + 1, n_el))
+          codes[c0 + c + 1] = (uint8_t)(two >> 8);
       } else {
-        codes[(c0 + c) / 2] = (uint8_t)e2m1x2(fmaf(a, inv, 0.0f), fmaf(b, inv, 0.0f));
+        if (MXQ_IN_RANGE(kChkPackOut, (c0 + c) / 2, n_el / 2))
+          codes[(c0 + c) / 2] = (uint8_t)e2m1x2(fmaf(a, inv, 0.0f), fmaf(b, inv, 0.0f));
       }
     }
   }
@@ -248,17 +259,20 @@ unpack_cache_general_kernel(const uint8_t* __restrict__ codes, const uint8_t* __
   for (int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x; g < n_groups;
        g += (int64_t)gridDim.x * kThreads) {
     const int64_t c0 = g * B;
-    const float s = scale_value<FMT>(scales[g]);
+    [[maybe_unused]] const int64_t n_el = n_groups * B;
+    const float s = scale_value<FMT>(MXQ_IN_RANGE(kChkUnpackScale, g, n_groups) ? scales[g] : 0u);
     for (int c = 0; c < B; ++c) {
       float v;
       if constexpr (FMT == MXQ_FMT_FP8) {
-        v = f16lo(e4m3x2_to_f16x2(codes[c0 + c])) * s;
+        v = f16lo(e4m3x2_to_f16x2(MXQ_IN_RANGE(kChkUnpackIn, c0 + c, n_el) ? codes[c0 + c] : 0u)) *
+            s;
       } else {
-        const uint32_t byte = codes[(c0 + c) / 2];
+        const uint32_t byte =
+            MXQ_IN_RANGE(kChkUnpackIn, (c0 + c) / 2, n_el / 2) ? codes[(c0 + c) / 2] : 0u;
         const uint32_t h2 = e2m1x2_to_f16x2(((c0 + c) & 1) ? (byte >> 4) : (byte & 15u));
         v = fmaf(f16lo(h2), s, 0.0f);
       }
-      store_one<DT>(out, c0 + c, v);
+      if (MXQ_IN_RANGE(kChkUnpackOut, c0 + c, n_el)) store_one<DT>(out, c0 + c, v);
     }
   }
 }
@@ -344,5 +358,7 @@ int launch_dequantize_cache_packed(const void* codes, const void* scales, int64_
   return launch_packed(nullptr, const_cast<void*>(codes), (uint8_t*)const_cast<void*>(scales),
                        out, false, dt, rows, C, fmt, B, fast, st);
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_cache_packed)
 
 }  // namespace mxq

@@ -94,7 +94,8 @@ mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
-      if (item < n_items) raw[u] = load_raw8<DT>(x, item);
+      if (item < n_items && MXQ_IN_RANGE(kChkMxQuantIn, item, n_items))
+        raw[u] = load_raw8<DT>(x, item);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -113,8 +114,9 @@ mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
       // keeps its sign, so the code's sign bit is set iff x < 0.
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = fmaf(elem_to_f32<DT>(raw_elem<DT>(raw[u], j)), inv, 0.0f);
-      packed[item] = e2m1x8(v);
-      if ((lane & 3) == 0) scales[item >> 2] = (uint8_t)(e + 127);
+      if (MXQ_IN_RANGE(kChkMxQuantOut, item, n_items)) packed[item] = e2m1x8(v);
+      if ((lane & 3) == 0 && MXQ_IN_RANGE(kChkMxQuantScale, item >> 2, n_items / 4))
+        scales[item >> 2] = (uint8_t)(e + 127);
     }
   }
 }
@@ -134,14 +136,16 @@ mx_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __restr
     for (int u = 0; u < kUnroll; ++u) {
       int64_t item = base + u * stride + lane;
       if (item < n_items) {
-        p[u] = ld_stream_u32(packed + item);
-        s[u] = ld_stream_u8(scales + (item >> 2));
+        p[u] = MXQ_IN_RANGE(kChkMxDeqIn, item, n_items) ? ld_stream_u32(packed + item) : 0u;
+        s[u] = MXQ_IN_RANGE(kChkMxDeqScale, item >> 2, n_items / 4)
+                   ? ld_stream_u8(scales + (item >> 2))
+                   : 0u;
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       int64_t item = base + u * stride + lane;
-      if (item >= n_items) continue;
+      if (item >= n_items || !MXQ_IN_RANGE(kChkMxDeqOut, item, n_items)) continue;
       if (s[u] == 0xFFu) {  // E8M0 NaN
         store8_bits<DT>(out, item, ElemTraits<DT>::kNaN);
         continue;
@@ -228,7 +232,8 @@ quantize_cache_kernel(const void* __restrict__ in, void* __restrict__ out, int64
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
-      if (item < n_items) raw[u] = load_raw8<DT>(in, item);
+      if (item < n_items && MXQ_IN_RANGE(kChkCacheIn, item, n_items))
+        raw[u] = load_raw8<DT>(in, item);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -244,7 +249,7 @@ quantize_cache_kernel(const void* __restrict__ in, void* __restrict__ out, int64
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = elem_to_f32<DT>(raw_elem<DT>(raw[u], j)) * inv;  // exact
       fake_quant8<FMT>(v, s);
-      store8<DT>(out, item, v);
+      if (MXQ_IN_RANGE(kChkCacheOut, item, n_items)) store8<DT>(out, item, v);
     }
   }
 }
@@ -279,7 +284,9 @@ quantize_cache_general_kernel(const void* __restrict__ in, void* __restrict__ ou
     int64_t c0 = (g % groups_per_row) * B;
     int64_t c1 = c0 + B < C ? c0 + B : C;
     uint32_t m = 0;
-    for (int64_t c = c0; c < c1; ++c) m = max(m, mag_as_f32_bits<DT>(load_elem_bits<DT>(in, r * C + c)));
+    for (int64_t c = c0; c < c1; ++c)
+      if (MXQ_IN_RANGE(kChkCacheGenIn, r * C + c, rows * C))
+        m = max(m, mag_as_f32_bits<DT>(load_elem_bits<DT>(in, r * C + c)));
     int k = cache_scale_exp<FMT>(m);
     float inv = exp2i(-k), s = exp2i(k);
     for (int64_t c = c0; c < c1; c += 8) {
@@ -287,11 +294,14 @@ quantize_cache_general_kernel(const void* __restrict__ in, void* __restrict__ ou
       int n = (int)(c1 - c < 8 ? c1 - c : 8);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        v[j] = j < n ? elem_to_f32<DT>(load_elem_bits<DT>(in, r * C + c + j)) * inv : 0.0f;
+        v[j] = j < n && MXQ_IN_RANGE(kChkCacheGenIn, r * C + c + j, rows * C)
+                   ? elem_to_f32<DT>(load_elem_bits<DT>(in, r * C + c + j)) * inv
+                   : 0.0f;
       fake_quant8<FMT>(v, s);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j < n) store_elem<DT>(out, r * C + c + j, v[j]);
+        if (j < n && MXQ_IN_RANGE(kChkCacheGenOut, r * C + c + j, rows * C))
+          store_elem<DT>(out, r * C + c + j, v[j]);
     }
   }
 }
@@ -398,5 +408,7 @@ int launch_quantize_cache(const void* in, void* out, int dt, int64_t rows, int64
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_elementwise)
 
 }  // namespace mxq

@@ -21,7 +21,8 @@ __constant__ float kE2M1Value[16] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6
                                      0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f};
 
 __device__ __forceinline__ float weight_at(const uint8_t* packed, const uint8_t* scales,
-                                           int64_t K, int64_t n, int64_t k) {
+                                           int64_t K, int64_t n, int64_t k, int64_t N) {
+  if (!MXQ_IN_RANGE(kChkGemmGenW, n * K + k, N * K)) return 0.0f;
   uint32_t byte = packed[n * (K / 2) + k / 2];
   uint32_t nib = (k & 1) ? (byte >> 4) : (byte & 15u);
   uint32_t s = scales[n * (K / 32) + k / 32];
@@ -55,14 +56,16 @@ grouped_mm_general_kernel(const __nv_bfloat16* __restrict__ a, const uint8_t* __
       for (int i = tid; i < kTM * kTK; i += kGThreads) {
         int t = i / kTK, kk = i % kTK;
         int64_t row = row0 + t, r = r0 + kk;
-        As[kk][t] = (row < row_end && r < kin) ? __bfloat162float(a[row * kin + r]) : 0.0f;
+        As[kk][t] = (row < row_end && r < kin && MXQ_IN_RANGE(kChkGemmGenIn, row * kin + r, T * kin))
+                        ? __bfloat162float(a[row * kin + r])
+                        : 0.0f;
       }
       for (int i = tid; i < kTN * kTK; i += kGThreads) {
         int o = i / kTK, kk = i % kTK;
         int64_t oc = o0 + o, r = r0 + kk;
         float w = 0.0f;
         if (oc < nout && r < kin)
-          w = transpose_w ? weight_at(pe, se, K, r, oc) : weight_at(pe, se, K, oc, r);
+          w = transpose_w ? weight_at(pe, se, K, r, oc, N) : weight_at(pe, se, K, oc, r, N);
         Ws[kk][o] = w;
       }
       __syncthreads();
@@ -87,7 +90,8 @@ grouped_mm_general_kernel(const __nv_bfloat16* __restrict__ a, const uint8_t* __
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         int64_t oc = o0 + tx * 4 + j;
-        if (oc < nout) y[row * nout + oc] = __float2bfloat16_rn(acc[i][j]);
+        if (oc < nout && MXQ_IN_RANGE(kChkGemmGenOut, row * nout + oc, T * nout))
+          y[row * nout + oc] = __float2bfloat16_rn(acc[i][j]);
       }
     }
   }
@@ -108,5 +112,7 @@ int launch_grouped_mm_general(const void* a, const void* packed, const void* sca
       transpose_w, (__nv_bfloat16*)y, dev_status);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_grouped_mm_general)
 
 }  // namespace mxq

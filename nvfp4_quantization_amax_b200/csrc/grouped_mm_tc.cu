@@ -69,7 +69,6 @@ constexpr int kMaxSmemExperts = 4096;               // offs cached in smem up to
 constexpr int kMaxSmemExpertsW = 256;               // (when smem also holds weight slots)
 constexpr int kWStages = 3;                         // packed-weight slots staged by TMA
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
-constexpr uint64_t kAbortSettleNs = 50000ull;
 
 template <bool kPair>
 struct Geo {
@@ -112,17 +111,13 @@ struct Shared {
   uint64_t wempty[kWStages];  // the dequantization warps are done with a slot
   uint64_t d_full, d_empty, drain;
   uint32_t tmem_base;
+  uint32_t peer_issued;  // activation stages the odd CTA of a pair loaded (written into the even CTA)
   int abort;
 };
 
-// Two E2M1 codes (one byte) -> two bf16 values times the block scale
-// 2^(s-127): exact E2M1 -> f16 (cvt), exact f32 products, one rounding to
-// bf16 that is exact whenever the weight is a normal bf16 value.
-__device__ __forceinline__ float scale_f32(uint32_t s) { return exp2i((int)s - 127); }
-
+__device__ __forceinline__ float scale_f32(uint32_t s) { return mx_block_scale(s); }
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t byte, float scale) {
-  const uint32_t h2 = e2m1x2_to_f16x2(byte);
-  return pack2<kBF16>(f16lo(h2) * scale, f16hi(h2) * scale);
+  return mx_dequant_pair(byte, scale);
 }
 
 __device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
@@ -231,6 +226,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
     mbar_init(&sh->d_full, 1);
     mbar_init(&sh->d_empty, kEpiWarps * G::kCG);
     mbar_init(&sh->drain, 1);
+    sh->peer_issued = 0;
     sh->abort = 0;
     fence_barrier_init();
   }
@@ -257,6 +253,7 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
   constexpr int kBK = G::kBK;
   const int nk = (int)(kin / kBK);
   const int64_t col_tiles = nout / G::kTileM;
+  uint32_t b_issued = 0;  // activation stages this CTA loaded (TMA lane 0)
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------ TMA producer (B)
@@ -286,9 +283,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           }
         }
       }
-      // Loads still in flight land before the CTA may exit (the even CTA's
-      // barrier counts both CTAs' bytes).
-      if (rank == 0) {
+      b_issued = it;
+      // Loads still in flight land before the CTA may exit.  (In pairs both
+      // CTAs' loads count on the even CTA's barriers: see the teardown.)
+      if constexpr (!kPair) {
         int abort_local = 0;
         for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
           bwait<kPair>(&sh->full_b[j % S], (j / S) & 1, &abort_local, kDrainLimitNs);
@@ -377,6 +375,11 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
       else mma_commit(&sh->drain);
       int abort_local = 0;
       mbar_wait(&sh->drain, 0, &abort_local, kDrainLimitNs);
+    } else if (kPair && lane == 0) {
+      // the leader's last commit (multicast) also lands here before this
+      // CTA may exit
+      int abort_local = 0;
+      mbar_wait(&sh->drain, 0, &abort_local, kDrainLimitNs);
     }
     __syncwarp();
   } else if (warp >= kEpiWarps) {
@@ -416,8 +419,11 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           uint32_t sb4;
           if (scales_by_tma)
             sb4 = *reinterpret_cast<const uint32_t*>(sS + ws * G::kSBytes + row * 16 + ((4 * ks) & 15));
-          else
+          else if (MXQ_IN_RANGE(kChkGemmTcScale, (e * N + m0 + row) * (K / 32) + 4 * ks + 3,
+                                E * N * (K / 32)))
             sb4 = *reinterpret_cast<const uint32_t*>(srow + 4 * ks);
+          else
+            sb4 = 0u;
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh->wempty[ws]);
           const int s = wi % S;
@@ -466,8 +472,11 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           if (j < nk) {
 #pragma unroll
             for (int c = 0; c < kV; ++c) {
-              pb[j][c] = ldg16(prow + (kBK / 2) * j + 16 * c);
-              sb[j][c] = srow[(kBK / 32) * j + c];
+              const bool in = MXQ_IN_RANGE(
+                  kChkGemmTcW, (e * N + n) * (K / 2) + (kBK / 4) * h + (kBK / 2) * j + 16 * c + 15,
+                  E * N * (K / 2));
+              pb[j][c] = in ? ldg16(prow + (kBK / 2) * j + 16 * c) : make_uint4(0u, 0u, 0u, 0u);
+              sb[j][c] = in ? srow[(kBK / 32) * j + c] : 0u;
             }
           }
         for (int ks0 = 0; ks0 < nk && ok; ks0 += 4) {
@@ -542,9 +551,14 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
               const int row = 32 * sub_i + 8 * j + rsub;  // n within the stage
               wd[sub_i][j] = *reinterpret_cast<const uint32_t*>(
                   wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
-              const uint32_t sb = scales_by_tma
-                                      ? (uint32_t)sst[row * 16 + soff]
-                                      : (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)];
+              [[maybe_unused]] const int64_t gi = e * N * (K / 32) + (m0 + 32 * q) / 32 +
+                                 ((int64_t)ks * kBK + row) * (K / 32);
+              const uint32_t sb =
+                  scales_by_tma
+                      ? (uint32_t)sst[row * 16 + soff]
+                      : (MXQ_IN_RANGE(kChkGemmTcScale, gi, E * N * (K / 32))
+                             ? (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)]
+                             : 0u);
               sc[sub_i][j] = scale_f32(sb);
             }
           __syncwarp();
@@ -600,8 +614,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-          sY[(32 * c + j) * kBM + col] = (uint16_t)(pr & 0xFFFFu);
-          sY[(32 * c + j + 1) * kBM + col] = (uint16_t)(pr >> 16);
+          if (MXQ_IN_RANGE(kChkGemmTcSmem, (32 * c + j + 1) * kBM + col, kBN * kBM)) {
+            sY[(32 * c + j) * kBM + col] = (uint16_t)(pr & 0xFFFFu);
+            sY[(32 * c + j + 1) * kBM + col] = (uint16_t)(pr >> 16);
+          }
         }
       }
       tc_fence_before();
@@ -612,7 +628,9 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
       // two rows of 128 outputs (256 bytes each) per warp instruction
       for (int r = 2 * warp + (lane >> 4); r < rows; r += 2 * kEpiWarps) {
         const uint4 val = *reinterpret_cast<const uint4*>(sY + r * kBM + 8 * (lane & 15));
-        *reinterpret_cast<uint4*>(yt + (int64_t)r * nout + 8 * (lane & 15)) = val;
+        const int64_t col0 = walk.col_tile * G::kTileM + rank * kBM + 8 * (lane & 15);
+        if (MXQ_IN_RANGE(kChkGemmTcOut, (row0 + r) * nout + col0 + 7, T * nout))
+          *reinterpret_cast<uint4*>(yt + (int64_t)r * nout + 8 * (lane & 15)) = val;
       }
     }
   }
@@ -620,14 +638,28 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) {
-    // After an abort the odd CTA may still have a TMA load in flight that
-    // counts on the even CTA's barrier; give it time to land (bounded).
-    if (*abort) {
-      const uint64_t t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < kAbortSettleNs) {
+    // After an abort the two CTAs may have loaded different numbers of
+    // activation stages, and the odd CTA's loads count on the even CTA's
+    // barriers.  The odd CTA reports its count; the even CTA settles the
+    // stages only one of them loaded (completing the transaction bytes that
+    // will never come, or expecting the ones that will) and waits, bounded,
+    // until every load of either CTA has landed.  Without an abort both
+    // counts are equal and every stage has long completed.
+    if (rank == 1 && warp == kTmaWarp && lane == 0)
+      st_shared_cluster_u32(mapa_shared(smem_addr(&sh->peer_issued), 0), b_issued);
+    cluster_sync();
+    if (rank == 0 && warp == kTmaWarp && lane == 0) {
+      const uint32_t mine = b_issued, peer = sh->peer_issued;
+      const uint32_t lo = mine < peer ? mine : peer, hi = mine < peer ? peer : mine;
+      for (uint32_t j = lo; j < hi; ++j) {
+        if (j < mine) mbar_complete_tx(&sh->full_b[j % S], G::kStageBytes);
+        else mbar_arrive_expect_tx(&sh->full_b[j % S], G::kStageBytes);
       }
+      int abort_local = 0;
+      for (uint32_t j = hi > (uint32_t)S ? hi - S : 0; j < hi; ++j)
+        mbar_wait(&sh->full_b[j % S], (j / S) & 1, &abort_local, kDrainLimitNs);
     }
-    cluster_sync();  // no peer still uses this CTA's TMEM or barriers
+    cluster_sync();  // no peer still uses this CTA's TMEM, barriers or shared memory
   }
   if (warp == kMmaWarp) {
     tc_fence_after();
@@ -721,19 +753,20 @@ int launch_grouped_mm(const void* a, const void* packed, const void* scales, con
   // tiles, or 16-byte loads in the single-CTA forward) and addresses weight
   // rows with 32-bit TMA coordinates.
   const bool w_ok = ((uintptr_t)packed & 15) == 0 && E * N < (int64_t)1 << 31;
-  const bool pair =
-      nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2 && w_ok;
   const bool tc = kin % Geo<false>::kBK == 0 && nout % kBM == 0 && ((uintptr_t)a & 15) == 0 &&
                   ((uintptr_t)y & 15) == 0 && T < (int64_t)1 << 31 && kin < (int64_t)1 << 31 &&
                   w_ok;
   if (!tc)
     return launch_grouped_mm_general(a, packed, scales, offs, T, E, N, K, transpose_w, y,
                                      dev_status, st);
+  const bool pair = nout % (2 * kBM) == 0 && kin % Geo<true>::kBK == 0 && num_sms() >= 2 && w_ok;
   if (transpose_w)
     return pair ? launch_tc<true, true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
                 : launch_tc<true, false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
   return pair ? launch_tc<false, true>(a, packed, scales, offs, T, E, N, K, y, dev_status, st)
               : launch_tc<false, false>(a, packed, scales, offs, T, E, N, K, y, dev_status, st);
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_grouped_mm_tc)
 
 }  // namespace mxq

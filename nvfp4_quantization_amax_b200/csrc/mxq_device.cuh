@@ -26,6 +26,60 @@ constexpr int kBF16 = MXQ_BF16;
 constexpr int kF16 = MXQ_F16;
 constexpr int kF32 = MXQ_F32;
 
+// ---------------------------------------------------- debug index checks
+//
+// The library's debug variant is built with -DMXQ_DEBUG_CHECKS.  There every
+// checked global-memory access first tests its element index against the
+// extent the kernel was launched for; a failed test records (check id,
+// index, extent) in this translation unit's record (the first failure
+// wins; a host reader per unit returns and clears it) and the access is
+// skipped, so nothing traps and no out-of-range address is touched.  In the
+// normal build a check is the constant true and compiles away.
+enum MxqCheckId {
+  kChkMxQuantIn = 1, kChkMxQuantOut, kChkMxQuantScale,
+  kChkMxDeqIn, kChkMxDeqScale, kChkMxDeqOut,
+  kChkCacheIn, kChkCacheOut, kChkCacheGenIn, kChkCacheGenOut,
+  kChkNvAmaxIn, kChkNvQuantIn, kChkNvQuantOut, kChkNvQuantScale,
+  kChkNvDeqIn, kChkNvDeqScale, kChkNvDeqOut,
+  kChkMseIn, kChkMseOut, kChkMseScale,
+  kChkPackIn, kChkPackOut, kChkPackScale, kChkUnpackIn, kChkUnpackScale, kChkUnpackOut,
+  kChkGemmGenIn, kChkGemmGenW, kChkGemmGenOut,
+  kChkGemmTcOut, kChkGemmTcScale, kChkGemmTcSmem, kChkGemmTcTmem,
+  kChkW4Out, kChkW4Scale, kChkW4Smem, kChkGemmTcW,
+  kChkSelfTest = 99
+};
+
+#ifdef MXQ_DEBUG_CHECKS
+static __device__ unsigned long long g_mxq_check_record[3];
+__device__ __forceinline__ bool mxq_in_range(int id, int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  if (atomicCAS(&g_mxq_check_record[0], 0ull, (unsigned long long)id) == 0ull) {
+    g_mxq_check_record[1] = (unsigned long long)i;
+    g_mxq_check_record[2] = (unsigned long long)n;
+  }
+  return false;
+}
+#define MXQ_IN_RANGE(id, i, n) ::mxq::mxq_in_range((id), (int64_t)(i), (int64_t)(n))
+// Host reader of this unit's record: copies it to out[3], then clears it.
+#define MXQ_DEFINE_CHECK_READER(fn)                                                    \
+  int fn(unsigned long long* out) {                                                    \
+    if (cudaMemcpyFromSymbol(out, g_mxq_check_record, 3 * sizeof(unsigned long long)) != \
+        cudaSuccess)                                                                   \
+      return MXQ_ERR_CUDA;                                                             \
+    const unsigned long long zero[3] = {0ull, 0ull, 0ull};                             \
+    return cudaMemcpyToSymbol(g_mxq_check_record, zero, sizeof(zero)) == cudaSuccess   \
+               ? MXQ_OK                                                                \
+               : MXQ_ERR_CUDA;                                                         \
+  }
+#else
+#define MXQ_IN_RANGE(id, i, n) true
+#define MXQ_DEFINE_CHECK_READER(fn) \
+  int fn(unsigned long long* out) { \
+    out[0] = out[1] = out[2] = 0ull; \
+    return MXQ_ERR_UNSUPPORTED;      \
+  }
+#endif
+
 // ---------------------------------------------------------------- memory
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {

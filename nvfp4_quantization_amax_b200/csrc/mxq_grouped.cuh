@@ -7,7 +7,20 @@
 
 #include <cstdint>
 
+#include "mxq_device.cuh"
+
 namespace mxq {
+
+// Weight decode of the tensor-core kernels: two E2M1 codes (one byte, low
+// nibble first) -> two bf16 values times the block scale 2^(s-127): exact
+// E2M1 -> f16 (cvt), exact f32 products, one rounding to bf16 that is exact
+// whenever the weight is a bf16 value (every scale byte up to 252).
+__device__ __forceinline__ float mx_block_scale(uint32_t s) { return exp2i((int)s - 127); }
+
+__device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) {
+  const uint32_t h2 = e2m1x2_to_f16x2(byte);
+  return pack2<kBF16>(f16lo(h2) * scale, f16hi(h2) * scale);
+}
 
 // True iff offs is non-negative, non-decreasing and ends at T.  Called by
 // every thread of a CTA (contains __syncthreads); block-uniform result.

@@ -58,6 +58,15 @@ int launch_nvfp4_w4a4_grouped_mm(const void* xq, const void* xs, const float* xg
 int launch_w4a4_grouped_mm(const void* xq, const void* xs, const void* packed, const void* scales,
                            const int32_t* offs, int64_t T, int64_t E, int64_t N, int64_t K,
                            void* y, int32_t* dev_status, uint64_t wait_limit_ns, cudaStream_t st);
+// Readers of each translation unit's debug check record (copy to out[3]
+// and clear; MXQ_ERR_UNSUPPORTED in the normal build).
+int check_record_elementwise(unsigned long long* out);
+int check_record_cache_packed(unsigned long long* out);
+int check_record_nvfp4(unsigned long long* out);
+int check_record_nvfp4_mse(unsigned long long* out);
+int check_record_grouped_mm_general(unsigned long long* out);
+int check_record_grouped_mm_tc(unsigned long long* out);
+int check_record_w4a4(unsigned long long* out);
 int launch_grouped_mm(const void* a, const void* packed, const void* scales, const int32_t* offs,
                       int64_t T, int64_t E, int64_t N, int64_t K, int transpose_w, void* y,
                       int32_t* dev_status, cudaStream_t st);

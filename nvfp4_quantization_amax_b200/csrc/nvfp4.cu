@@ -70,7 +70,10 @@ nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restr
     uint4 a[kNvUnroll], b[kNvUnroll];
 #pragma unroll
     for (int u = 0; u < kNvUnroll; ++u)
-      if (base + u * stride < n_items) load_vec8<DT>(x, base + u * stride, a[u], b[u]);
+      if (base + u * stride < n_items && MXQ_IN_RANGE(kChkNvAmaxIn, base + u * stride, n_items))
+        load_vec8<DT>(x, base + u * stride, a[u], b[u]);
+      else
+        a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int u = 0; u < kNvUnroll; ++u)
       if (base + u * stride < n_items) m = max(m, amax8<DT>(a[u], b[u]));
@@ -85,6 +88,27 @@ nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restr
   }
 }
 
+// E2M1 codes of the eight binary32 quotients w_j / d, with -0.0 giving the
+// code of +0.0 (no sign bit) and a nonzero weight whose quotient underflows
+// keeping its sign.  r = fl32(1 / d) for d in the bracket's range, else 0:
+// then the IEEE divisions decide.  Bracket (see e2m1x8_quot): the products
+// are fma(w, r(1 -+ 2^-19), +0), which round exactly like w r(1 -+ 2^-19)
+// except that a zero product is +0.
+__device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, float d, float r) {
+  if (r != 0.0f) {
+    const float r_lo = r * (1.0f - 0x1p-19f), r_hi = r * (1.0f + 0x1p-19f);
+    uint32_t a = 0, b = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a |= e2m1x2(fmaf(w[2 * j], r_lo, 0.0f), fmaf(w[2 * j + 1], r_lo, 0.0f)) << (8 * j);
+      b |= e2m1x2(fmaf(w[2 * j], r_hi, 0.0f), fmaf(w[2 * j + 1], r_hi, 0.0f)) << (8 * j);
+    }
+    if (a == b) return a;
+  }
+  return e2m1x8_div(w[0] + 0.0f, w[1] + 0.0f, w[2] + 0.0f, w[3] + 0.0f, w[4] + 0.0f, w[5] + 0.0f,
+                    w[6] + 0.0f, w[7] + 0.0f, d);
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
@@ -96,7 +120,10 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const float t = __fmul_rn(6.0f, g);
   if (blockIdx.x == 0 && threadIdx.x == 0) *global_scale = g;
   const int lane = threadIdx.x & 31;
-  const uint32_t negzero = (DT == kF32) ? 0x80000000u : 0x8000u;
+  // The two lanes of a 16-block (lanes 2i, 2i+1) share its scale; of the
+  // four unroll slots, lane parity p derives the scales of slots 2p and
+  // 2p + 1 and the pair swaps them by shuffle.
+  const int p = lane & 1;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
   for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kNvUnroll) {
@@ -104,39 +131,67 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
 #pragma unroll
     for (int u = 0; u < kNvUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
-      if (item < n_items) load_vec8<DT>(x, item, va[u], vb[u]);
+      if (item < n_items && MXQ_IN_RANGE(kChkNvQuantIn, item, n_items))
+        load_vec8<DT>(x, item, va[u], vb[u]);
+    }
+    uint32_t m[kNvUnroll];
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      m[u] = item < n_items ? amax8<DT>(va[u], vb[u]) : 0u;
+      m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], 1));  // the block's two lanes
+    }
+    // both lanes of a block are in range or out of range together (the
+    // item count is even and pairs are aligned)
+    if (zero) {
+#pragma unroll
+      for (int u = 0; u < kNvUnroll; ++u) {
+        const int64_t item = base + u * stride + lane;
+        if (item >= n_items) continue;
+        if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items)) packed[item] = 0u;
+        if (p == 0 && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
+          block_scales[item >> 1] = 0x38u;  // E4M3 1.0
+      }
+      continue;
+    }
+    float dm[2], rm[2];
+    uint32_t sm[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t mk = p ? m[2 + k] : m[k];
+      float q = __fdiv_rn(__uint_as_float(mk), t);
+      if (q == 0.0f) q = 1.0f;
+      q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
+      sm[k] = e4m3x2(q, 0.0f) & 0xFFu;
+      const float s = f16lo(e4m3x2_to_f16x2(sm[k]));
+      dm[k] = __fmul_rn(s, g);
+      rm[k] = quot_fast_ok(dm[k]) ? __frcp_rn(dm[k]) : 0.0f;
+    }
+    float d4[kNvUnroll], r4[kNvUnroll];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float dk = __shfl_xor_sync(0xffffffffu, dm[k], 1);
+      const float rk = __shfl_xor_sync(0xffffffffu, rm[k], 1);
+      d4[k] = p ? dk : dm[k];
+      r4[k] = p ? rk : rm[k];
+      d4[2 + k] = p ? dm[k] : dk;
+      r4[2 + k] = p ? rm[k] : rk;
     }
 #pragma unroll
     for (int u = 0; u < kNvUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
-      const bool valid = item < n_items;
-      uint32_t m = valid ? amax8<DT>(va[u], vb[u]) : 0u;
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));  // the two lanes of a 16-block
-      if (!valid) continue;
-      uint32_t sbyte;
-      uint32_t codes = 0;
-      if (zero) {
-        sbyte = 0x38u;  // E4M3 1.0
-      } else {
-        float q = __fdiv_rn(__uint_as_float(m), t);
-        if (q == 0.0f) q = 1.0f;
-        q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
-        sbyte = e4m3x2(q, 0.0f) & 0xFFu;
-        const float s = f16lo(e4m3x2_to_f16x2(sbyte));
-        const float d = __fmul_rn(s, g);
-        float w[8];
+      if (item >= n_items) continue;
+      float w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t bits = elem_bits<DT>(va[u], vb[u], j);
-          if (bits == negzero) bits = 0u;  // -0.0 carries no sign into the code
-          w[j] = elem_to_f32<DT>(bits);
-        }
-        // E2M1 of the binary32 quotients w / d (the sign is kept on underflow)
-        codes = quot_fast_ok(d) ? e2m1x8_quot(w, d)
-                                : e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
-      }
-      packed[item] = codes;
-      if ((lane & 1) == 0) block_scales[item >> 1] = (uint8_t)sbyte;
+      for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(va[u], vb[u], j));
+      if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items))
+        packed[item] = e2m1x8_quot_unsigned_zero(w, d4[u], r4[u]);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t item = base + (2 * p + k) * stride + lane;
+      if (item < n_items && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
+        block_scales[item >> 1] = (uint8_t)sm[k];
     }
   }
 }
@@ -156,8 +211,10 @@ nvfp4_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __re
     for (int u = 0; u < kNvUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
       if (item < n_items) {
-        p[u] = ld_stream_u32(packed + item);
-        sb[u] = ld_stream_u8(block_scales + (item >> 1));
+        p[u] = MXQ_IN_RANGE(kChkNvDeqIn, item, n_items) ? ld_stream_u32(packed + item) : 0u;
+        sb[u] = MXQ_IN_RANGE(kChkNvDeqScale, item >> 1, n_items / 2)
+                    ? ld_stream_u8(block_scales + (item >> 1))
+                    : 0u;
       }
     }
 #pragma unroll
@@ -174,7 +231,7 @@ nvfp4_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __re
         v[2 * j] = fmaf(f16lo(h2) * s, g, 0.0f);
         v[2 * j + 1] = fmaf(f16hi(h2) * s, g, 0.0f);
       }
-      store8<DT>(out, item, v);
+      if (MXQ_IN_RANGE(kChkNvDeqOut, item, n_items)) store8<DT>(out, item, v);
     }
   }
 }
@@ -278,5 +335,7 @@ int launch_nvfp4_dequantize(const void* packed, const void* block_scales, const 
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_nvfp4)
 
 }  // namespace mxq

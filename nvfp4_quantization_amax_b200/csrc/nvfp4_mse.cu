@@ -71,7 +71,9 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
   const bool valid = blk < n_blocks;
 
   float w[16];
-  if (valid) load_block16<DT>(x, blk, w);
+  if (valid && MXQ_IN_RANGE(kChkMseIn, blk, n_blocks)) load_block16<DT>(x, blk, w);
+  else
+    for (int i = 0; i < 16; ++i) w[i] = 0.0f;
 
   int best_c = 0x38;
   if (!zero) {
@@ -177,8 +179,8 @@ nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
       codes = make_uint2(e2m1x8(v), e2m1x8(v + 8));
     }
   }
-  packed[blk] = codes;
-  block_scales[blk] = (uint8_t)best_c;
+  if (MXQ_IN_RANGE(kChkMseOut, blk, n_blocks)) packed[blk] = codes;
+  if (MXQ_IN_RANGE(kChkMseScale, blk, n_blocks)) block_scales[blk] = (uint8_t)best_c;
 }
 
 int mse_grid(int64_t n_blocks) {
@@ -214,5 +216,7 @@ int launch_nvfp4_quantize_mse(const void* x, int dt, int64_t rows, int64_t K, vo
   }
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_nvfp4_mse)
 
 }  // namespace mxq

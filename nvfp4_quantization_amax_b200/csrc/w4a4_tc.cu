@@ -234,11 +234,19 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       const uint8_t* xsc = x_scales + pwalk.row0 * srow + kSPR * pks;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        wv[i] = __ldg(reinterpret_cast<const SV*>(wsc + (lane + 32 * i) * srow));
+        wv[i] = MXQ_IN_RANGE(kChkW4Scale,
+                             (pwalk.expert * N + pwalk.col_tile * kM + lane + 32 * i) * srow +
+                                 kSPR * pks + kSPR - 1,
+                             E * N * srow)
+                    ? __ldg(reinterpret_cast<const SV*>(wsc + (lane + 32 * i) * srow))
+                    : SV{};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = lane + 32 * i;
-        xv[i] = r < rows ? __ldg(reinterpret_cast<const SV*>(xsc + r * srow)) : SV{};
+        xv[i] = r < rows && MXQ_IN_RANGE(kChkW4Scale, (pwalk.row0 + r) * srow + kSPR * pks + kSPR - 1,
+                                         T * srow)
+                    ? __ldg(reinterpret_cast<const SV*>(xsc + r * srow))
+                    : SV{};
       }
       if (++pks == nk) {
         pks = 0;
@@ -383,8 +391,10 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-          sY[(32 * c + j) * kM + col] = (uint16_t)(pr & 0xFFFFu);
-          sY[(32 * c + j + 1) * kM + col] = (uint16_t)(pr >> 16);
+          if (MXQ_IN_RANGE(kChkW4Smem, (32 * c + j + 1) * kM + col, kN * kM)) {
+            sY[(32 * c + j) * kM + col] = (uint16_t)(pr & 0xFFFFu);
+            sY[(32 * c + j + 1) * kM + col] = (uint16_t)(pr >> 16);
+          }
         }
       }
       tc_fence_before();
@@ -394,7 +404,9 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       __nv_bfloat16* yt = y + row0 * N + walk.col_tile * kM;
       for (int r = 2 * warp + (lane >> 4); r < rows; r += 2 * kEpiWarps) {
         const uint4 val = *reinterpret_cast<const uint4*>(sY + r * kM + 8 * (lane & 15));
-        *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+        if (MXQ_IN_RANGE(kChkW4Out, (row0 + r) * N + walk.col_tile * kM + 8 * (lane & 15) + 7,
+                         T * N))
+          *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
       }
     }
   }
@@ -448,5 +460,7 @@ int launch_nvfp4_w4a4_grouped_mm(const void* xq, const void* xs, const float* xg
   return launch_w4a4<true>(xq, xs, xg, packed, scales, wg, offs, T, E, N, K, y, dev_status,
                            wait_limit_ns, st);
 }
+
+MXQ_DEFINE_CHECK_READER(check_record_w4a4)
 
 }  // namespace mxq

@@ -116,6 +116,15 @@ def test_binding_fails_loudly_without_gpu():
         mxq.quantize_cache(torch.zeros(4, 32, dtype=torch.bfloat16), "fp8", 32)
 
 
+def test_debug_entry_points_are_unsupported_in_the_normal_library(L):
+    rec = (ctypes.c_int64 * 3)(7, 7, 7)
+    assert L.mxq_debug_checks(ctypes.cast(rec, ctypes.c_void_p)) == EUNSUP
+    assert list(rec) == [0, 0, 0]
+    assert L.mxq_debug_checks(NULL) == EARG
+    assert L.mxq_debug_selftest(A1, NULL) == EUNSUP  # nothing launched
+    assert L.mxq_debug_selftest(BAD, NULL) == EALIGN
+
+
 def test_wait_limit_setter_round_trips(L):
     prev = mxq.set_wait_limit_ns(123)
     assert mxq.set_wait_limit_ns(prev) == 123

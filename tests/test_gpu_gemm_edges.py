@@ -98,11 +98,10 @@ def assert_per_expert(y, ref, owner, what):
         rms = np.sqrt(np.mean(r ** 2))
         bound = REL * np.maximum(np.abs(r), 1e-2 * rms) + ABS
         excess = np.abs(y[m] - r) / bound
-        i = int(np.argmax(excess))
-        assert excess[i] <= 1.0, "%s: expert %d output %d: got %r want %r (rms %r)" % (
-            what, e, i, y[m].reshape(-1)[i] if y[m].ndim == 1 else y[m].flat[i],
-            r.flat[i], rms)
-        worst = max(worst, float(excess[i]))
+        i = int(np.argmax(excess))  # index into the flattened outputs
+        assert excess.flat[i] <= 1.0, "%s: expert %d output %d: got %r want %r (rms %r)" % (
+            what, e, i, y[m].flat[i], r.flat[i], rms)
+        worst = max(worst, float(excess.flat[i]))
     return worst
 
 

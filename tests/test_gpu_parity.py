@@ -335,6 +335,26 @@ def test_grouped_mm_wait_timeout_reports_status():
     check_gemm([700, 300, 50], N=128, K=512, transpose_w=False)
 
 
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_wait_timeout_pair_shape(transpose_w):
+    # The same on the CTA-pair kernel (output width a multiple of 256): after
+    # the abort both CTAs' activation loads are settled and drained before
+    # either CTA exits, and the context stays usable.
+    counts = [700, 300, 50]
+    x, g, packed, scales, offs = moe_case(counts, N=256, K=512)
+    a = g if transpose_w else x
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    prev = mxq.set_wait_limit_ns(0)
+    try:
+        mxq.mxfp4_grouped_mm(a.to(DEV), packed.to(DEV), scales.to(DEV), offs.to(DEV),
+                             transpose_w=transpose_w, status=status)
+        torch.cuda.synchronize()
+    finally:
+        mxq.set_wait_limit_ns(prev)
+    assert int(status.item()) == -7
+    check_gemm(counts, N=256, K=512, transpose_w=transpose_w)
+
+
 # ------------------------------------------------------- NVFP4 two-level
 
 def nv_inputs(dtype):
