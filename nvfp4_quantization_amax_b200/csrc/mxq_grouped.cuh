@@ -22,6 +22,26 @@ __device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) 
   return pack2<kBF16>(f16lo(h2) * scale, f16hi(h2) * scale);
 }
 
+// The same result with fewer instructions for scale bytes s <= 142 (the
+// caller checks).  The f16 pattern of an E2M1 value, its exponent and
+// mantissa shifted down by 3 bits into bf16's layout and its sign kept, is
+// the bf16 pattern of the value times 2^-112 (a normal number, or zero); one
+// bf16 multiply by 2^(s - 15) then gives value * 2^(s - 127), which is
+// exactly representable in bf16 (subnormals included), so the multiply is
+// exact, as the f32 path is.
+constexpr uint32_t kMxFastScaleMax = 142;  // 2^(s - 15) is then a bf16 value
+__device__ __forceinline__ uint32_t mx_fast_factor(uint32_t s) {
+  const uint32_t e = (s + 112u) << 7;  // bf16 exponent field of 2^(s - 15)
+  return e | (e << 16);
+}
+__device__ __forceinline__ uint32_t mx_dequant_pair_fast(uint32_t byte, uint32_t factor) {
+  const uint32_t h2 = e2m1x2_to_f16x2(byte);
+  const uint32_t t = ((h2 >> 3) & 0x0FFF0FFFu) | (h2 & 0x80008000u);
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(factor));
+  return r;
+}
+
 // True iff offs is non-negative, non-decreasing and ends at T.  Called by
 // every thread of a CTA (contains __syncthreads); block-uniform result.
 __device__ __forceinline__ bool offs_valid(const int32_t* offs, int64_t E, int64_t T) {
