@@ -15,7 +15,11 @@ namespace mxq {
 // nibble first) -> two bf16 values times the block scale 2^(s-127): exact
 // E2M1 -> f16 (cvt), exact f32 products, one rounding to bf16 that is exact
 // whenever the weight is a bf16 value (every scale byte up to 252).
-__device__ __forceinline__ float mx_block_scale(uint32_t s) { return exp2i((int)s - 127); }
+// 2^(s - 127) as f32: the exponent field s for s >= 1 (255 gives +inf, as
+// exp2i(128) does), the subnormal 2^-127 for s = 0.
+__device__ __forceinline__ float mx_block_scale(uint32_t s) {
+  return __uint_as_float(s != 0u ? s << 23 : 0x00400000u);
+}
 
 __device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) {
   const uint32_t h2 = e2m1x2_to_f16x2(byte);
