@@ -428,10 +428,6 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           if (lane == 0) mbar_arrive(&sh->wempty[ws]);
           const int s = wi % S;
           bool waited = false;
-          // the bf16-multiply decode when every scale byte the warp meets allows it
-          const bool fast = __all_sync(
-              0xffffffffu, (sb4 & 0xFFu) <= kMxFastScaleMax && ((sb4 >> 8) & 0xFFu) <= kMxFastScaleMax &&
-                               ((sb4 >> 16) & 0xFFu) <= kMxFastScaleMax && (sb4 >> 24) <= kMxFastScaleMax);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t v[32];
@@ -440,17 +436,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
               const uint4 dd = d[2 * hh + c];
               const uint32_t w[4] = {dd.x, dd.y, dd.z, dd.w};
               const uint32_t sbyte = (sb4 >> (8 * (2 * hh + c))) & 0xFFu;
-              if (fast) {
-                const uint32_t f = mx_fast_factor(sbyte);
+              const uint32_t flo = mx_split_factor_lo(sbyte), fhi = mx_split_factor_hi(sbyte);
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  v[16 * c + i] = mx_dequant_pair_fast((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, f);
-              } else {
-                const float sc = scale_f32(sbyte);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
-              }
+              for (int i = 0; i < 16; ++i)
+                v[16 * c + i] = mx_dequant_pair_split((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, flo, fhi);
             }
             if (!waited) {
               if (!(ok = warp_wait<kPair>(&sh->empty[s], ((wi / S) & 1) ^ 1, abort, wait_limit_ns)))
