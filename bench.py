@@ -73,9 +73,16 @@ def load_peaks():
 
 
 def source_hash(name):
-    p = os.path.join(ROOT, "nvfp4_quantization_amax_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel's translation unit and every header beside it (the
+    device helpers it includes), so that a profile taken before a change to
+    either no longer counts."""
+    csrc = os.path.join(ROOT, "nvfp4_quantization_amax_b200", "csrc")
+    h = hashlib.sha256()
+    headers = sorted(f for f in os.listdir(csrc) if f.endswith((".cuh", ".h")))
+    for f in [name] + headers:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel_key, src):
