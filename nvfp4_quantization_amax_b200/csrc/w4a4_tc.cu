@@ -20,12 +20,16 @@
 // tokens of the expert and k the reduction index, 256 per pipeline stage
 // (128 bytes of codes per row: one 128-byte-swizzled TMA row).
 //   * warp 4 (one lane) TMA-loads both code tiles of a stage;
-//   * warp 5 gathers the stage's scale bytes (8 or 16 per row: 128 weight
-//     rows and 256 token rows) from the row-major [rows, K/32 or K/16] scale
-//     arrays and writes them into the tensor core's scale layout in shared
-//     memory: blocks of 128 rows x 4 scales, row r at byte 16 (r % 32) +
-//     4 (r / 32) + the scale's index;
-//   * warp 6 (one lane) copies those blocks into TMEM (tcgen05.cp, 32 lanes
+//   * warps 5 and 6 gather the stage's scale bytes (8 or 16 per row: 128
+//     weight rows and 256 token rows, half of them each) from the row-major
+//     [rows, K/32 or K/16] scale arrays and write them into the tensor
+//     core's scale layout in shared memory: blocks of 128 rows x 4 scales,
+//     row r at byte 16 (r % 32) + 4 (r / 32) + the scale's index.  Where the
+//     rows allow it they load a row's scales of several stages at once (32
+//     bytes: one L2 sector when the row is sector-aligned), since one
+//     sector per row and stage is as many bytes into the SM as a quarter
+//     of the stage's codes;
+//   * warp 7 (one lane) copies those blocks into TMEM (tcgen05.cp, 32 lanes
 //     x 128 bits, replicated to the four lane quarters) and issues four
 //     K=64 MMAs per stage, each selecting its scales by block and byte id;
 //   * warps 0-3 drain D, round to bf16, stage the tile in shared memory and
@@ -87,9 +91,10 @@ struct W4Fmt {
 };
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
-constexpr int kSfWarp = 5;
-constexpr int kMmaWarp = 6;
-constexpr int kThreads = 7 * 32;
+constexpr int kSfWarp = 5;   // warps 5 and 6
+constexpr int kSfWarps = 2;
+constexpr int kMmaWarp = 7;
+constexpr int kThreads = 8 * 32;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 
@@ -128,7 +133,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // core's scale layout (s in 0..3).
 __device__ __forceinline__ uint32_t sf_offset(int r) { return 16 * (r & 31) + 4 * ((r >> 5) & 3); }
 
-template <bool kNV>
+// kWide: each scale load covers kG stages (32 bytes per row); otherwise one
+// stage (8 or 16 bytes per row).
+template <bool kNV, bool kWide>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const uint8_t* __restrict__ x_scales, const uint8_t* __restrict__ w_scales,
@@ -162,7 +169,7 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh->full[s], 2);  // TMA expect_tx arrive + scale warp arrive
+      mbar_init(&sh->full[s], 1 + kSfWarps);  // TMA expect_tx arrive + scale warp arrives
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->d_full, 1);
@@ -213,103 +220,136 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         mbar_wait(&sh->full[j % kStages], (j / kStages) & 1, &abort_local, kDrainLimitNs);
     }
     __syncwarp();
-  } else if (warp == kSfWarp) {
-    // ------------------------------------------- scale-factor producer
-    // Stage ks needs scales 8ks .. 8ks+7 of every row: weight rows n0 + m
-    // (m = lane + 32i) and token rows row0 + r (r = lane + 32i, zero past
-    // the expert's rows).  Scales 0-3 go to block 0, 4-7 to block 1 (of
-    // each 128-row group).  The global loads run two stages ahead of the
-    // stores (a cursor of its own walks the same (tile, stage) sequence),
-    // so their latency overlaps the tensor core's work.
-    using SV = typename std::conditional<kNV, uint4, uint2>::type;  // a row's scales of a stage
+  } else if (warp >= kSfWarp && warp < kSfWarp + kSfWarps) {
+    // ------------------------------------------- scale-factor producers
+    // Stage ks needs scales kSPR ks .. kSPR ks + kSPR - 1 of every row:
+    // weight rows n0 + m and token rows row0 + r (zero past the expert's
+    // rows).  Scale warp u takes m = lane + 32 (kRowsW u + i) and
+    // r = lane + 32 (kRowsX u + i).  Scales 0-3 go to block 0, 4-7 to
+    // block 1, ... (of each 128-row group).  A load brings a row's scales of
+    // kG consecutive stages (a group); the loads run one group ahead of the
+    // stores (a cursor of its own walks the same (tile, group) sequence), so
+    // their latency overlaps the tensor core's work.
     constexpr int kSPR = F::kScalesPerRow;
+    constexpr int kG = kWide ? 32 / kSPR : 1;      // stages per load
+    constexpr int kW = kG * kSPR / 4;              // 32-bit words per row and load
+    constexpr int kRowsW = 4 / kSfWarps, kRowsX = 8 / kSfWarps;
+    const int u = warp - kSfWarp;
+    using Buf = uint32_t[kRowsW + kRowsX][kW];
     TileWalker pwalk(t_offs, E, kN, col_tiles);
     int64_t ptile = blockIdx.x;
     bool phave = pwalk.seek(ptile);
-    int pks = 0;
-    auto issue = [&](SV (&wv)[4], SV (&xv)[8]) {
+    int pg = 0;  // group within the cursor's tile
+    auto load_row = [&](uint32_t (&w)[kW], const uint8_t* p) {
+      if constexpr (kW == 2) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        w[0] = v.x; w[1] = v.y;
+      } else {
+#pragma unroll
+        for (int h = 0; h < kW / 4; ++h) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + h);
+          w[4 * h] = v.x; w[4 * h + 1] = v.y; w[4 * h + 2] = v.z; w[4 * h + 3] = v.w;
+        }
+      }
+    };
+    auto issue = [&](Buf& buf) {
       if (!phave) return;
       const int64_t rows = pwalk.row_end - pwalk.row0 < kN ? pwalk.row_end - pwalk.row0 : kN;
-      const uint8_t* wsc = w_scales + (pwalk.expert * N + pwalk.col_tile * kM) * srow + kSPR * pks;
-      const uint8_t* xsc = x_scales + pwalk.row0 * srow + kSPR * pks;
+      const int64_t wrow0 = pwalk.expert * N + pwalk.col_tile * kM;
+      const int64_t col = (int64_t)4 * kW * pg;  // first scale byte of the group
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        wv[i] = MXQ_IN_RANGE(kChkW4Scale,
-                             (pwalk.expert * N + pwalk.col_tile * kM + lane + 32 * i) * srow +
-                                 kSPR * pks + kSPR - 1,
-                             E * N * srow)
-                    ? __ldg(reinterpret_cast<const SV*>(wsc + (lane + 32 * i) * srow))
-                    : SV{};
+      for (int i = 0; i < kRowsW; ++i) {
+        const int64_t row = wrow0 + lane + 32 * (kRowsW * u + i);
+        if (MXQ_IN_RANGE(kChkW4Scale, row * srow + col + 4 * kW - 1, E * N * srow))
+          load_row(buf[i], w_scales + row * srow + col);
+        else
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = lane + 32 * i;
-        xv[i] = r < rows && MXQ_IN_RANGE(kChkW4Scale, (pwalk.row0 + r) * srow + kSPR * pks + kSPR - 1,
-                                         T * srow)
-                    ? __ldg(reinterpret_cast<const SV*>(xsc + r * srow))
-                    : SV{};
+          for (int k = 0; k < kW; ++k) buf[i][k] = 0u;
       }
-      if (++pks == nk) {
-        pks = 0;
+#pragma unroll
+      for (int i = 0; i < kRowsX; ++i) {
+        const int r = lane + 32 * (kRowsX * u + i);
+        const int64_t row = pwalk.row0 + r;
+        if (r < rows && MXQ_IN_RANGE(kChkW4Scale, row * srow + col + 4 * kW - 1, T * srow))
+          load_row(buf[kRowsW + i], x_scales + row * srow + col);
+        else
+#pragma unroll
+          for (int k = 0; k < kW; ++k) buf[kRowsW + i][k] = 0u;
+      }
+      if (++pg * kG == nk) {
+        pg = 0;
         ptile += gridDim.x;
         phave = pwalk.seek(ptile);
       }
     };
-    // word b of a row's scales (scales 4b..4b+3) goes to block b; B blocks
-    // are ordered (group 0, block b), (group 1, block b) for b = 0, 1, ...
-    auto words = [](const SV& v, uint32_t (&w)[F::kBlocks]) {
-      if constexpr (kNV) {
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-      } else {
-        w[0] = v.x; w[1] = v.y;
-      }
-    };
-    auto store = [&](int s, const SV (&wv)[4], const SV (&xv)[8]) {
+    // Stage q of the group in buf: word q kBlocks + b of a row (its scales
+    // 4b..4b+3 of the stage) goes to block b; B blocks are ordered
+    // (group 0, block b), (group 1, block b) for b = 0, 1, ...
+    auto store = [&](int s, const Buf& buf, auto qc) {
+      constexpr int q = decltype(qc)::value;
       uint8_t* fa = sSfa(s);
       uint8_t* fb = sSfb(s);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t o = sf_offset(lane + 32 * i);
-        uint32_t w[F::kBlocks];
-        words(wv[i], w);
+      for (int i = 0; i < kRowsW; ++i) {
+        const uint32_t o = sf_offset(lane + 32 * (kRowsW * u + i));
 #pragma unroll
         for (int b = 0; b < F::kBlocks; ++b)
-          *reinterpret_cast<uint32_t*>(fa + b * kSfBlock + o) = w[b];
+          *reinterpret_cast<uint32_t*>(fa + b * kSfBlock + o) = buf[i][q * F::kBlocks + b];
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = lane + 32 * i;
+      for (int i = 0; i < kRowsX; ++i) {
+        const int r = lane + 32 * (kRowsX * u + i);
         const uint32_t o = sf_offset(r);
         const int g = r >> 7;  // 128-row group
-        uint32_t w[F::kBlocks];
-        words(xv[i], w);
 #pragma unroll
         for (int b = 0; b < F::kBlocks; ++b)
-          *reinterpret_cast<uint32_t*>(fb + (2 * b + g) * kSfBlock + o) = w[b];
+          *reinterpret_cast<uint32_t*>(fb + (2 * b + g) * kSfBlock + o) =
+              buf[kRowsW + i][q * F::kBlocks + b];
       }
       fence_proxy_async_smem();  // visible to tcgen05.cp
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->full[s]);
     };
-    SV wa[4], xa[8], wb[4], xb[8];
-    issue(wa, xa);
-    issue(wb, xb);
+    // Stage q (runtime) of the group in buf, dispatched to a constant index.
+    auto store_q = [&](int s, const Buf& buf, int q) {
+      if constexpr (kG == 1) {
+        store(s, buf, std::integral_constant<int, 0>{});
+      } else if constexpr (kG == 2) {
+        if (q == 0) store(s, buf, std::integral_constant<int, 0>{});
+        else store(s, buf, std::integral_constant<int, 1>{});
+      } else {
+        static_assert(kG == 4, "stages per scale load");
+        switch (q) {
+          case 0: store(s, buf, std::integral_constant<int, 0>{}); break;
+          case 1: store(s, buf, std::integral_constant<int, 1>{}); break;
+          case 2: store(s, buf, std::integral_constant<int, 2>{}); break;
+          default: store(s, buf, std::integral_constant<int, 3>{}); break;
+        }
+      }
+    };
+    Buf ba, bb;
+    issue(ba);
+    issue(bb);
     TileWalker walk(t_offs, E, kN, col_tiles);
-    uint32_t it = 0;
+    uint32_t it = 0, grp = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x) {
       for (int ks = 0; ks < nk && ok; ++ks, ++it) {
         const int s = it % kStages;
         if (!(ok = warp_wait(&sh->empty[s], ((it / kStages) & 1) ^ 1, abort, wait_limit_ns)))
           break;
-        // item `it` was loaded into buffer it % 2; refill that buffer with
-        // item it + 2
-        if ((it & 1) == 0) {
-          store(s, wa, xa);
-          issue(wa, xa);
+        // group `grp` was loaded into buffer grp % 2; once its last stage
+        // is stored, refill that buffer with group grp + 2
+        const int q = ks % kG;
+        const bool last = q == kG - 1;
+        if ((grp & 1) == 0) {
+          store_q(s, ba, q);
+          if (last) issue(ba);
         } else {
-          store(s, wb, xb);
-          issue(wb, xb);
+          store_q(s, bb, q);
+          if (last) issue(bb);
         }
+        if (last) ++grp;
       }
     }
   } else if (warp == kMmaWarp) {
@@ -432,7 +472,13 @@ int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* pac
       !make_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, E * N, K / 2, K / 2, kKB, kM,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return MXQ_ERR_CUDA;
-  auto kernel = w4a4_tc_kernel<kNV>;
+  // Scale loads of 32 bytes per row (several stages) when every row's
+  // scales start on a 16-byte boundary and the stages split into whole
+  // groups; 8 or 16 bytes per stage otherwise.
+  const int64_t srow = K / (kNV ? 16 : 32);
+  const int64_t group = kNV ? 2 : 4;
+  const bool wide = srow % 16 == 0 && (K / 256) % group == 0;
+  auto kernel = wide ? w4a4_tc_kernel<kNV, true> : w4a4_tc_kernel<kNV, false>;
   if (allow_dynamic_smem((const void*)kernel, (int)F::kSmem) != cudaSuccess) return MXQ_ERR_CUDA;
   const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
   const int64_t sms = num_sms();
