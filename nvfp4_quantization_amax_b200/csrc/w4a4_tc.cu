@@ -62,7 +62,6 @@ constexpr int kMaxStages = 3;
 constexpr uint32_t kABytes = kM * kKB;            // 16 KB
 constexpr uint32_t kBBytes = kN * kKB;            // 32 KB
 constexpr uint32_t kSfBlock = 512;                // 128 rows x 4 scales
-constexpr uint32_t kStagingBytes = kN * kM * 2;   // 64 KB of bf16 output
 constexpr int kMaxSmemExperts = 256;
 constexpr int kTmemCols = 512;
 constexpr int kDCol = 0;                // accumulator: columns [0, 256)
@@ -79,10 +78,13 @@ struct W4Fmt {
   static constexpr uint32_t kSfaBytes = kBlocks * kSfBlock;
   static constexpr uint32_t kSfbBytes = 2 * kBlocks * kSfBlock;  // two 128-row groups
   static constexpr int kSfbCol = kSfaCol + 4 * kBlocks;
-  // NVFP4 stages are larger (twice the scale bytes): two fit beside the
-  // output staging, which the operand feed of this kernel tolerates.
-  static constexpr int kStages = kNV ? 2 : 3;
+  static constexpr int kStages = 3;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  // Output tokens staged in shared memory at a time (bf16, 128 features
+  // each): the whole tile, or, for NVFP4, whose stages are larger (twice
+  // the scale bytes), half of it, so that three stages fit.
+  static constexpr int kYRows = kNV ? kN / 2 : kN;
+  static constexpr uint32_t kStagingBytes = kYRows * kM * 2;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
@@ -150,7 +152,7 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint16_t* sY = (uint16_t*)(smem + kStages * kStageBytes);
-  Shared* sh = (Shared*)((uint8_t*)sY + kStagingBytes);
+  Shared* sh = (Shared*)((uint8_t*)sY + F::kStagingBytes);
   int32_t* s_offs = (int32_t*)((uint8_t*)sh + 256);
   auto sA = [&](int s) { return smem + s * kStageBytes; };
   auto sB = [&](int s) { return smem + s * kStageBytes + kABytes; };
@@ -419,34 +421,46 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       const int col = 32 * warp + lane;  // output feature within the tile's 128
       // NV: the product of the two per-tensor scales, applied in f32
       const float gg = kNV ? __fmul_rn(x_global[0], w_global[walk.expert]) : 1.0f;
+      constexpr int kYRows = F::kYRows;
+      const int nc = (int)((rows + 31) / 32);  // 32-token chunks of D
+      __nv_bfloat16* yt = y + row0 * N + walk.col_tile * kM;
+      if (rows <= 0 && lane == 0) mbar_arrive(&sh->d_empty);
+      // tokens p0 .. p0 + kYRows - 1 per pass: staged, then stored
+      for (int p0 = 0; p0 < rows; p0 += kYRows) {
+        if (p0 > 0) epi_bar();  // the previous pass's rows are stored
+        const int c_end = nc < (p0 + kYRows) / 32 ? nc : (p0 + kYRows) / 32;
 #pragma unroll 1
-      for (int c = 0; c < (int)((rows + 31) / 32); ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
-        tmem_wait_ld();
-        if constexpr (kNV) {
+        for (int c = p0 / 32; c < c_end; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
+          tmem_wait_ld();
+          if constexpr (kNV) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gg);
-        }
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gg);
+          }
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-          if (MXQ_IN_RANGE(kChkW4Smem, (32 * c + j + 1) * kM + col, kN * kM)) {
-            sY[(32 * c + j) * kM + col] = (uint16_t)(pr & 0xFFFFu);
-            sY[(32 * c + j + 1) * kM + col] = (uint16_t)(pr >> 16);
+          for (int j = 0; j < 32; j += 2) {
+            const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            const int t = 32 * c + j - p0;  // token within the pass
+            if (MXQ_IN_RANGE(kChkW4Smem, (t + 1) * kM + col, kYRows * kM)) {
+              sY[t * kM + col] = (uint16_t)(pr & 0xFFFFu);
+              sY[(t + 1) * kM + col] = (uint16_t)(pr >> 16);
+            }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->d_empty);
-      epi_bar();  // the whole tile is staged
-      __nv_bfloat16* yt = y + row0 * N + walk.col_tile * kM;
-      for (int r = 2 * warp + (lane >> 4); r < rows; r += 2 * kEpiWarps) {
-        const uint4 val = *reinterpret_cast<const uint4*>(sY + r * kM + 8 * (lane & 15));
-        if (MXQ_IN_RANGE(kChkW4Out, (row0 + r) * N + walk.col_tile * kM + 8 * (lane & 15) + 7,
-                         T * N))
-          *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+        if (p0 + kYRows >= rows) {  // every chunk of D is read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->d_empty);
+        }
+        epi_bar();  // the pass is staged
+        const int r_end = rows < p0 + kYRows ? (int)rows : p0 + kYRows;
+        for (int r = p0 + 2 * warp + (lane >> 4); r < r_end; r += 2 * kEpiWarps) {
+          const uint4 val = *reinterpret_cast<const uint4*>(sY + (r - p0) * kM + 8 * (lane & 15));
+          if (MXQ_IN_RANGE(kChkW4Out, (row0 + r) * N + walk.col_tile * kM + 8 * (lane & 15) + 7,
+                           T * N))
+            *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+        }
       }
     }
   }
