@@ -37,12 +37,21 @@ __device__ __forceinline__ uint32_t elem_bits(const uint4& a, const uint4& b, in
   }
 }
 
+// f32 bit pattern of max |x| over the eight elements.  For 16-bit formats
+// the magnitudes are compared pairwise as unsigned halves (monotone in |x|
+// for finite values).
 template <int DT>
 __device__ __forceinline__ uint32_t amax8(const uint4& a, const uint4& b) {
-  uint32_t m = 0;
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    const uint32_t M = 0x7FFF7FFFu;
+    const uint32_t m2 = __vmaxu2(__vmaxu2(a.x & M, a.y & M), __vmaxu2(a.z & M, a.w & M));
+    return mag_as_f32_bits<DT>(max(m2 & 0xFFFFu, m2 >> 16));
+  } else {
+    uint32_t m = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(elem_bits<DT>(a, b, j)));
-  return m;
+    for (int j = 0; j < 8; ++j) m = max(m, mag_as_f32_bits<DT>(elem_bits<DT>(a, b, j)));
+    return m;
+  }
 }
 
 template <int DT>
@@ -97,13 +106,14 @@ nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restr
 __device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, float d, float r) {
   if (r != 0.0f) {
     const float r_lo = r * (1.0f - 0x1p-19f), r_hi = r * (1.0f + 0x1p-19f);
-    uint32_t a = 0, b = 0;
+    float lo[8], hi[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a |= e2m1x2(fmaf(w[2 * j], r_lo, 0.0f), fmaf(w[2 * j + 1], r_lo, 0.0f)) << (8 * j);
-      b |= e2m1x2(fmaf(w[2 * j], r_hi, 0.0f), fmaf(w[2 * j + 1], r_hi, 0.0f)) << (8 * j);
+    for (int j = 0; j < 8; ++j) {
+      lo[j] = fmaf(w[j], r_lo, 0.0f);
+      hi[j] = fmaf(w[j], r_hi, 0.0f);
     }
-    if (a == b) return a;
+    const uint32_t a = e2m1x8(lo);
+    if (a == e2m1x8(hi)) return a;
   }
   return e2m1x8_div(w[0] + 0.0f, w[1] + 0.0f, w[2] + 0.0f, w[3] + 0.0f, w[4] + 0.0f, w[5] + 0.0f,
                     w[6] + 0.0f, w[7] + 0.0f, d);
