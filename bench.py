@@ -253,6 +253,12 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
     del nvq
     calls["nvfp4_w4a4_grouped_mm"] = lambda: mxq.nvfp4_w4a4_grouped_mm(
         step.x, nvp, nvs, nvg, step.offs, step.y, step.status)
+    # the block-scaled GEMMs alone, on activations quantized beforehand
+    calls["_w4a4_gemm"] = lambda: mxq.w4a4_grouped_mm(None, step.P5, step.S5, step.offs, step.y,
+                                                      step.status, x_quantized=(xq, xs))
+    nx = mxq.nvfp4_quantize(step.x)
+    calls["_nvfp4_w4a4_gemm"] = lambda: mxq.nvfp4_w4a4_grouped_mm(
+        None, nvp, nvs, nvg, step.offs, step.y, step.status, x_quantized=nx)
     # Before each timed call a 256 MB write flushes L2 (126 MB) and keeps the
     # GPU busy while the host queues the call, so each event pair holds the
     # call's own kernels on cold inputs and no host launch overhead.
@@ -571,6 +577,15 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
         rows = {}
         w4 = next_ms.pop("w4a4_grouped_mm", None)
         nv4 = next_ms.pop("nvfp4_w4a4_grouped_mm", None)
+        w4g = next_ms.pop("_w4a4_gemm", None)
+        nv4g = next_ms.pop("_nvfp4_w4a4_gemm", None)
+        fp4_peak = 4.0 * peaks["bf16_tflops"]
+
+        def gemm_alone(ms):
+            tf = gemm_flops() / (ms * 1e-3) / 1e12
+            return {"ms": round(ms, 4), "tflops": round(tf, 1),
+                    "frac_of_fp4_peak": round(tf / fp4_peak, 4),
+                    "includes": "the block-scaled GEMM on activations quantized beforehand"}
         for n, ms in next_ms.items():
             gbs = nb[n] / (ms * 1e-3) / 1e9
             rows[n] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
@@ -595,6 +610,8 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
                 "frac_of_fp4_peak": round(tf / (4.0 * peaks["bf16_tflops"]), 4),
                 "includes": "mx_quantize of the activations + the block-scaled GEMM",
                 "workload": "x bf16 [32768,7168], W MXFP4 [32,2048,7168], multinomial counts"}
+            if w4g is not None:
+                rows["w4a4_grouped_mm"]["gemm"] = gemm_alone(w4g)
         if nv4 is not None:
             tf = gemm_flops() / (nv4 * 1e-3) / 1e12
             rows["nvfp4_w4a4_grouped_mm"] = {
@@ -602,6 +619,8 @@ def report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clocks, next_ms=Non
                 "frac_of_fp4_peak": round(tf / (4.0 * peaks["bf16_tflops"]), 4),
                 "includes": "nvfp4_quantize of the activations (two passes) + the block-scaled GEMM",
                 "workload": "x bf16 [32768,7168], W NVFP4 [32,2048,7168], multinomial counts"}
+            if nv4g is not None:
+                rows["nvfp4_w4a4_grouped_mm"]["gemm"] = gemm_alone(nv4g)
         line["next_rows"] = rows
     if extra:
         line.update(extra)

@@ -489,77 +489,130 @@ def mxfp4_grouped_mm(a, packed, scales, offs, transpose_w=False, out=None, statu
     return _result(out, ho, host)
 
 
+def _quantized_operand(t, shape, dtype, name, what):
+    """A quantized activation operand passed by the caller: a contiguous
+    device tensor of the given dtype and shape (checked before any launch)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s: %s must be a CUDA tensor" % (what, name))
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError("%s: %s must be a contiguous %s tensor of shape %s"
+                         % (what, name, dtype, list(shape)))
+    return t
+
+
 def w4a4_grouped_mm(x, packed, scales, offs, out=None, status=None, x_packed=None,
-                    x_scales=None):
+                    x_scales=None, x_quantized=None):
     """W4A4 grouped GEMM: the bf16 activations x [T, K] are quantized to
     MXFP4 (mx_quantize) and multiplied with the MXFP4 expert weights on the
     block-scaled tensor cores.  Returns bf16 [T, N] (forward only).
     x_packed / x_scales: optional preallocated [T, K/2] / [T, K/32] buffers
-    for the quantized activations."""
-    if x.dtype != torch.bfloat16:
-        raise TypeError("w4a4_grouped_mm: activations must be bf16")
-    x, host = _to_device(x)
-    packed, _ = _to_device(packed, x.device)
-    scales, _ = _to_device(scales, x.device)
-    offs, _ = _to_device(offs, x.device)
-    x, packed, scales = x.contiguous(), packed.contiguous(), scales.contiguous()
+    for the quantized activations.
+    x_quantized: optional (x_packed, x_scales) device tensors that already
+    hold the activations as mx_quantize writes them; then x is not used (it
+    may be None) and no quantization runs: the call is the block-scaled GEMM
+    alone (the C entry point mxfp4_w4a4_grouped_mm)."""
+    if x_quantized is None:
+        if x.dtype != torch.bfloat16:
+            raise TypeError("w4a4_grouped_mm: activations must be bf16")
+        x, host = _to_device(x)
+        dev = x.device
+    else:
+        host = False
+        dev = x_quantized[0].device if isinstance(x_quantized[0], torch.Tensor) else None
+        if dev is None or dev.type != "cuda":
+            raise ValueError("w4a4_grouped_mm: x_quantized must hold CUDA tensors")
+    packed, _ = _to_device(packed, dev)
+    scales, _ = _to_device(scales, dev)
+    offs, _ = _to_device(offs, dev)
+    packed, scales = packed.contiguous(), scales.contiguous()
     offs = offs.to(torch.int32).contiguous()
     E, N, Kh = packed.shape
     K = 2 * Kh
-    T = x.shape[0]
-    if x.shape[1] != K:
-        raise ValueError("w4a4_grouped_mm: x must be [T, %d]" % K)
     if tuple(scales.shape) != (E, N, K // 32) or offs.numel() != E:
         raise ValueError("w4a4_grouped_mm: scales [E, N, K/32] and offs [E] expected")
-    for t, name in ((x_packed, "x_packed"), (x_scales, "x_scales")):
-        if t is not None and not (t.is_cuda and t.device == x.device):
-            raise ValueError("w4a4_grouped_mm: %s must be a tensor on %s" % (name, x.device))
-    xq, xs = mx_quantize(x, x_packed, x_scales)
-    out, ho = _out(out, (T, N), torch.bfloat16, x.device, "out")
-    st = _device_word(status, torch.int32, 1, x.device, "status")
+    if x_quantized is None:
+        x = x.contiguous()
+        T = x.shape[0]
+        if x.shape[1] != K:
+            raise ValueError("w4a4_grouped_mm: x must be [T, %d]" % K)
+        for t, name in ((x_packed, "x_packed"), (x_scales, "x_scales")):
+            if t is not None and not (t.is_cuda and t.device == dev):
+                raise ValueError("w4a4_grouped_mm: %s must be a tensor on %s" % (name, dev))
+        xq, xs = mx_quantize(x, x_packed, x_scales)
+    else:
+        xq, xs = x_quantized
+        T = int(xq.shape[0]) if isinstance(xq, torch.Tensor) and xq.dim() == 2 else -1
+        xq = _quantized_operand(xq, (T, K // 2), torch.uint8, "x_quantized[0]", "w4a4_grouped_mm")
+        xs = _quantized_operand(xs, (T, K // 32), torch.uint8, "x_quantized[1]",
+                                "w4a4_grouped_mm")
+        if xs.device != dev:
+            raise ValueError("w4a4_grouped_mm: x_quantized tensors must share a device")
+    out, ho = _out(out, (T, N), torch.bfloat16, dev, "out")
+    st = _device_word(status, torch.int32, 1, dev, "status")
     rc = lib().mxfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(packed), _ptr(scales), _ptr(offs),
-                                     T, E, N, K, _ptr(out), st, _stream(x.device))
+                                     T, E, N, K, _ptr(out), st, _stream(dev))
     _check(rc, "mxfp4_w4a4_grouped_mm")
     return _result(out, ho, host)
 
 
 def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=None,
-                          status=None):
+                          status=None, x_quantized=None):
     """W4A4 grouped GEMM in NVFP4: the bf16 activations x [T, K] are
     quantized to NVFP4 as one tensor (nvfp4_quantize) and multiplied with the
     NVFP4 expert weights (packed [E, N, K/2], E4M3 block scales [E, N, K/16],
     float32 global scales [E]) on the block-scaled tensor cores.  Returns
-    bf16 [T, N]."""
-    if x.dtype != torch.bfloat16:
-        raise TypeError("nvfp4_w4a4_grouped_mm: activations must be bf16")
-    x, host = _to_device(x)
-    packed, _ = _to_device(packed, x.device)
-    block_scales, _ = _to_device(block_scales, x.device)
-    w_global_scales, _ = _to_device(w_global_scales, x.device)
-    offs, _ = _to_device(offs, x.device)
-    x, packed, block_scales = x.contiguous(), packed.contiguous(), block_scales.contiguous()
+    bf16 [T, N].
+    x_quantized: optional (x_packed [T, K/2] uint8, x_block_scales [T, K/16]
+    uint8, x_global_scale float32 [1]) device tensors that already hold the
+    activations as nvfp4_quantize writes them; then x is not used (it may be
+    None) and the call is the block-scaled GEMM alone."""
+    if x_quantized is None:
+        if x.dtype != torch.bfloat16:
+            raise TypeError("nvfp4_w4a4_grouped_mm: activations must be bf16")
+        x, host = _to_device(x)
+        dev = x.device
+    else:
+        host = False
+        dev = x_quantized[0].device if isinstance(x_quantized[0], torch.Tensor) else None
+        if dev is None or dev.type != "cuda":
+            raise ValueError("nvfp4_w4a4_grouped_mm: x_quantized must hold CUDA tensors")
+    packed, _ = _to_device(packed, dev)
+    block_scales, _ = _to_device(block_scales, dev)
+    w_global_scales, _ = _to_device(w_global_scales, dev)
+    offs, _ = _to_device(offs, dev)
+    packed, block_scales = packed.contiguous(), block_scales.contiguous()
     w_global_scales = w_global_scales.to(torch.float32).contiguous()
     offs = offs.to(torch.int32).contiguous()
     E, N, Kh = packed.shape
     K = 2 * Kh
-    T = x.shape[0]
-    if x.shape[1] != K:
-        raise ValueError("nvfp4_w4a4_grouped_mm: x must be [T, %d]" % K)
     if (tuple(block_scales.shape) != (E, N, K // 16) or offs.numel() != E or
             w_global_scales.numel() != E):
         raise ValueError("nvfp4_w4a4_grouped_mm: block_scales [E, N, K/16], global scales [E] "
                          "and offs [E] expected")
-    xq, xs, xg = nvfp4_quantize(x)
-    out, ho = _out(out, (T, N), torch.bfloat16, x.device, "out")
-    st = _device_word(status, torch.int32, 1, x.device, "status")
+    if x_quantized is None:
+        x = x.contiguous()
+        T = x.shape[0]
+        if x.shape[1] != K:
+            raise ValueError("nvfp4_w4a4_grouped_mm: x must be [T, %d]" % K)
+        xq, xs, xg = nvfp4_quantize(x)
+    else:
+        xq, xs, xg = x_quantized
+        T = int(xq.shape[0]) if isinstance(xq, torch.Tensor) and xq.dim() == 2 else -1
+        what = "nvfp4_w4a4_grouped_mm"
+        xq = _quantized_operand(xq, (T, K // 2), torch.uint8, "x_quantized[0]", what)
+        xs = _quantized_operand(xs, (T, K // 16), torch.uint8, "x_quantized[1]", what)
+        if isinstance(xg, torch.Tensor) and xg.numel() == 1:
+            xg = xg.reshape(1)
+        xg = _quantized_operand(xg, (1,), torch.float32, "x_quantized[2]", what)
+        if xs.device != dev or xg.device != dev:
+            raise ValueError("%s: x_quantized tensors must share a device" % what)
+    out, ho = _out(out, (T, N), torch.bfloat16, dev, "out")
+    st = _device_word(status, torch.int32, 1, dev, "status")
     rc = lib().nvfp4_w4a4_grouped_mm(_ptr(xq), _ptr(xs), _ptr(xg), _ptr(packed),
                                      _ptr(block_scales), _ptr(w_global_scales), _ptr(offs),
-                                     T, E, N, K, _ptr(out), st, _stream(x.device))
+                                     T, E, N, K, _ptr(out), st, _stream(dev))
     _check(rc, "nvfp4_w4a4_grouped_mm")
     return _result(out, ho, host)
-
-
-NVFP4_WORKSPACE_BYTES = 16
 
 
 def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspace=None,

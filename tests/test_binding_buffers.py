@@ -182,3 +182,20 @@ def test_streamed_packed_cache_and_nvfp4_dequant_equal_device_calls(small_chunks
     y = mxq.nvfp4_dequantize(p, s, g, torch.float32)
     hy = mxq.nvfp4_dequantize(p.cpu().pin_memory(), s.cpu().pin_memory(), g.cpu(), torch.float32)
     assert not hy.is_cuda and torch.equal(hy.view(torch.uint8), y.cpu().view(torch.uint8))
+
+
+def test_prequantized_w4a4_operands_must_be_cuda_tensors():
+    # refused on the host, before any library call
+    p = torch.zeros(2, 128, 128, dtype=torch.uint8)
+    s = torch.zeros(2, 128, 8, dtype=torch.uint8)
+    offs = torch.tensor([32, 64], dtype=torch.int32)
+    xq = torch.zeros(64, 128, dtype=torch.uint8)
+    xs = torch.zeros(64, 8, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        mxq.w4a4_grouped_mm(None, p, s, offs, x_quantized=(xq, xs))
+    with pytest.raises(ValueError, match="CUDA"):
+        mxq.nvfp4_w4a4_grouped_mm(None, p, torch.zeros(2, 128, 16, dtype=torch.uint8),
+                                  torch.ones(2), offs,
+                                  x_quantized=(xq, torch.zeros(64, 16, dtype=torch.uint8),
+                                               torch.ones(1)))
+

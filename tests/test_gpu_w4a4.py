@@ -155,3 +155,29 @@ def test_nvfp4_w4a4_full_size_sampled():
     counts = gen.expert_counts(T, E).numpy()
     rows = [0, 1, 255, 256, int(np.cumsum(counts)[0]), 20000, T - 1]
     nv_check(list(counts), N, K, rows=rows)
+
+
+def test_prequantized_activations_give_the_same_bits():
+    # x_quantized: the block-scaled GEMM alone on activations quantized beforehand
+    counts = [200, 0, 37, 275]
+    x, packed, scales, offs = case(counts, 256, 512)
+    xd, pd, sd, od = x.to(DEV), packed.to(DEV), scales.to(DEV), offs.to(DEV)
+    want = mxq.w4a4_grouped_mm(xd, pd, sd, od)
+    xq, xs = mxq.mx_quantize(xd)
+    got = mxq.w4a4_grouped_mm(None, pd, sd, od, x_quantized=(xq, xs))
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    wn = gen.expert_weights(len(counts), 256, 512).view(torch.int16).numpy().view(np.uint16)
+    qs = [oracle.nvfp4_quantize(wn[e]) for e in range(len(counts))]
+    nvp = torch.from_numpy(np.stack([q[0] for q in qs])).to(DEV)
+    nvs = torch.from_numpy(np.stack([q[1] for q in qs])).to(DEV)
+    nvg = torch.tensor([q[2] for q in qs], dtype=torch.float32, device=DEV)
+    want = mxq.nvfp4_w4a4_grouped_mm(xd, nvp, nvs, nvg, od)
+    got = mxq.nvfp4_w4a4_grouped_mm(None, nvp, nvs, nvg, od,
+                                    x_quantized=mxq.nvfp4_quantize(xd))
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    # wrong operand shapes are refused before a launch
+    with pytest.raises(ValueError, match="x_quantized"):
+        mxq.w4a4_grouped_mm(None, pd, sd, od, x_quantized=(xq[:, :-1], xs))
+    with pytest.raises(ValueError, match="x_quantized"):
+        mxq.w4a4_grouped_mm(None, pd, sd, od, x_quantized=(xq, xs[:-1]))
+
