@@ -615,6 +615,9 @@ def nvfp4_w4a4_grouped_mm(x, packed, block_scales, w_global_scales, offs, out=No
     return _result(out, ho, host)
 
 
+NVFP4_WORKSPACE_BYTES = 16
+
+
 def nvfp4_quantize(x, packed=None, block_scales=None, global_scale=None, workspace=None,
                    rule="max"):
     """NVFP4 two-level quantize + pack along the last dim (K % 16 == 0).
