@@ -18,6 +18,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------- dependent launches
+
+// With programmatic stream serialization a kernel may start before the
+// previous kernel on its stream has finished; this waits until that kernel
+// has completed and its memory operations are visible.  Without the launch
+// attribute it returns at once.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -160,15 +160,8 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   auto sSfb = [&](int s) { return smem + s * kStageBytes + kABytes + kBBytes + kSfaBytes; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (!offs_valid(offs, E, T)) {
-    if (blockIdx.x == 0 && threadIdx.x == 0 && dev_status) *dev_status = MXQ_ERR_BAD_OFFS;
-    return;
-  }
-  const int32_t* t_offs = offs;
-  if (E <= kMaxSmemExperts) {
-    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) s_offs[e] = offs[e];
-    t_offs = s_offs;
-  }
+  // Set-up that reads nothing the previous kernel on the stream may still be
+  // writing (the launch lets this CTA start while that kernel finishes).
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh->full[s], 1 + kSfWarps);  // TMA expect_tx arrive + scale warp arrives
@@ -187,6 +180,22 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   if (warp == kTmaWarp && lane == 0) {
     prefetch_tmap(&tmap_x);
     prefetch_tmap(&tmap_w);
+  }
+  griddep_wait();  // the previous kernel's results (e.g. the activations) are complete
+  if (!offs_valid(offs, E, T)) {  // (contains __syncthreads)
+    if (blockIdx.x == 0 && threadIdx.x == 0 && dev_status) *dev_status = MXQ_ERR_BAD_OFFS;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(sh->tmem_base, kTmemCols);
+    }
+    return;
+  }
+  const int32_t* t_offs = offs;
+  if (E <= kMaxSmemExperts) {
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) s_offs[e] = offs[e];
+    t_offs = s_offs;
   }
   tc_fence_before();
   __syncthreads();
@@ -497,10 +506,23 @@ int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* pac
   const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
   const int64_t sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
-  kernel<<<grid, kThreads, F::kSmem, st>>>(xmap, wmap, (const uint8_t*)xs, (const uint8_t*)scales,
-                                           xg, wg, offs, T, E, N, K, (__nv_bfloat16*)y,
-                                           dev_status, wait_limit_ns);
-  return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+  // Programmatic stream serialization: the CTAs may start their set-up while
+  // the previous kernel on the stream (typically the activation quantizer)
+  // finishes; they wait for its results before reading any input.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = F::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err =
+      cudaLaunchKernelEx(&cfg, kernel, xmap, wmap, (const uint8_t*)xs, (const uint8_t*)scales, xg,
+                         wg, offs, T, E, N, K, (__nv_bfloat16*)y, dev_status, wait_limit_ns);
+  return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 }  // namespace
