@@ -119,6 +119,87 @@ __device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, fl
                     w[6] + 0.0f, w[7] + 0.0f, d);
 }
 
+// One iteration of the quantize pass over the warp's kNvUnroll items
+// base + u stride + lane.  kFull: all of them exist (no bounds tests).
+template <int DT, bool kFull>
+__device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
+                                                     uint32_t* __restrict__ packed,
+                                                     uint8_t* __restrict__ block_scales,
+                                                     int64_t n_items, int64_t base, int64_t stride,
+                                                     int lane, float g, float t, bool zero) {
+  const int p = lane & 1;
+  auto in_range = [&](int64_t item) { return kFull || item < n_items; };
+  uint4 va[kNvUnroll], vb[kNvUnroll];
+#pragma unroll
+  for (int u = 0; u < kNvUnroll; ++u) {
+    const int64_t item = base + u * stride + lane;
+    if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantIn, item, n_items))
+      load_vec8<DT>(x, item, va[u], vb[u]);
+  }
+  uint32_t m[kNvUnroll];
+#pragma unroll
+  for (int u = 0; u < kNvUnroll; ++u) {
+    const int64_t item = base + u * stride + lane;
+    m[u] = in_range(item) ? amax8<DT>(va[u], vb[u]) : 0u;
+    m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], 1));  // the block's two lanes
+  }
+  // both lanes of a block are in range or out of range together (the
+  // item count is even and pairs are aligned)
+  if (zero) {
+#pragma unroll
+    for (int u = 0; u < kNvUnroll; ++u) {
+      const int64_t item = base + u * stride + lane;
+      if (!in_range(item)) continue;
+      if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items)) packed[item] = 0u;
+      if (p == 0 && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
+        block_scales[item >> 1] = 0x38u;  // E4M3 1.0
+    }
+    return;
+  }
+  // The two lanes of a 16-block (lanes 2i, 2i+1) share its scale; of the
+  // four unroll slots, lane parity p derives the scales of slots 2p and
+  // 2p + 1 and the pair swaps them by shuffle.
+  float dm[2], rm[2];
+  uint32_t sm[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t mk = p ? m[2 + k] : m[k];
+    float q = __fdiv_rn(__uint_as_float(mk), t);
+    if (q == 0.0f) q = 1.0f;
+    q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
+    sm[k] = e4m3x2(q, 0.0f) & 0xFFu;
+    const float s = f16lo(e4m3x2_to_f16x2(sm[k]));
+    dm[k] = __fmul_rn(s, g);
+    rm[k] = quot_fast_ok(dm[k]) ? __frcp_rn(dm[k]) : 0.0f;
+  }
+  float d4[kNvUnroll], r4[kNvUnroll];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float dk = __shfl_xor_sync(0xffffffffu, dm[k], 1);
+    const float rk = __shfl_xor_sync(0xffffffffu, rm[k], 1);
+    d4[k] = p ? dk : dm[k];
+    r4[k] = p ? rk : rm[k];
+    d4[2 + k] = p ? dm[k] : dk;
+    r4[2 + k] = p ? rm[k] : rk;
+  }
+#pragma unroll
+  for (int u = 0; u < kNvUnroll; ++u) {
+    const int64_t item = base + u * stride + lane;
+    if (!in_range(item)) continue;
+    float w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(va[u], vb[u], j));
+    if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items))
+      packed[item] = e2m1x8_quot_unsigned_zero(w, d4[u], r4[u]);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int64_t item = base + (2 * p + k) * stride + lane;
+    if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
+      block_scales[item >> 1] = (uint8_t)sm[k];
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
@@ -130,79 +211,17 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const float t = __fmul_rn(6.0f, g);
   if (blockIdx.x == 0 && threadIdx.x == 0) *global_scale = g;
   const int lane = threadIdx.x & 31;
-  // The two lanes of a 16-block (lanes 2i, 2i+1) share its scale; of the
-  // four unroll slots, lane parity p derives the scales of slots 2p and
-  // 2p + 1 and the pair swaps them by shuffle.
-  const int p = lane & 1;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
   for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kNvUnroll) {
-    uint4 va[kNvUnroll], vb[kNvUnroll];
-#pragma unroll
-    for (int u = 0; u < kNvUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      if (item < n_items && MXQ_IN_RANGE(kChkNvQuantIn, item, n_items))
-        load_vec8<DT>(x, item, va[u], vb[u]);
-    }
-    uint32_t m[kNvUnroll];
-#pragma unroll
-    for (int u = 0; u < kNvUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      m[u] = item < n_items ? amax8<DT>(va[u], vb[u]) : 0u;
-      m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], 1));  // the block's two lanes
-    }
-    // both lanes of a block are in range or out of range together (the
-    // item count is even and pairs are aligned)
-    if (zero) {
-#pragma unroll
-      for (int u = 0; u < kNvUnroll; ++u) {
-        const int64_t item = base + u * stride + lane;
-        if (item >= n_items) continue;
-        if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items)) packed[item] = 0u;
-        if (p == 0 && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
-          block_scales[item >> 1] = 0x38u;  // E4M3 1.0
-      }
-      continue;
-    }
-    float dm[2], rm[2];
-    uint32_t sm[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint32_t mk = p ? m[2 + k] : m[k];
-      float q = __fdiv_rn(__uint_as_float(mk), t);
-      if (q == 0.0f) q = 1.0f;
-      q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
-      sm[k] = e4m3x2(q, 0.0f) & 0xFFu;
-      const float s = f16lo(e4m3x2_to_f16x2(sm[k]));
-      dm[k] = __fmul_rn(s, g);
-      rm[k] = quot_fast_ok(dm[k]) ? __frcp_rn(dm[k]) : 0.0f;
-    }
-    float d4[kNvUnroll], r4[kNvUnroll];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const float dk = __shfl_xor_sync(0xffffffffu, dm[k], 1);
-      const float rk = __shfl_xor_sync(0xffffffffu, rm[k], 1);
-      d4[k] = p ? dk : dm[k];
-      r4[k] = p ? rk : rm[k];
-      d4[2 + k] = p ? dm[k] : dk;
-      r4[2 + k] = p ? rm[k] : rk;
-    }
-#pragma unroll
-    for (int u = 0; u < kNvUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      if (item >= n_items) continue;
-      float w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(va[u], vb[u], j));
-      if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items))
-        packed[item] = e2m1x8_quot_unsigned_zero(w, d4[u], r4[u]);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t item = base + (2 * p + k) * stride + lane;
-      if (item < n_items && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
-        block_scales[item >> 1] = (uint8_t)sm[k];
-    }
+    // every item of this iteration exists (warp-uniform: base is the
+    // warp's first item)
+    if (base + (kNvUnroll - 1) * stride + 32 <= n_items)
+      nvfp4_quantize_items<DT, true>(x, packed, block_scales, n_items, base, stride, lane, g, t,
+                                     zero);
+    else
+      nvfp4_quantize_items<DT, false>(x, packed, block_scales, n_items, base, stride, lane, g, t,
+                                      zero);
   }
 }
 
