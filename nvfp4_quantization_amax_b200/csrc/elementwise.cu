@@ -82,6 +82,44 @@ __device__ __forceinline__ int mx_scale_exp(uint32_t amax_f32bits) {
   return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
+// One iteration of the pack over the warp's kUnroll items base + u stride
+// + lane.  kFull: all of them exist (no bounds tests).
+template <int DT, bool kFull>
+__device__ __forceinline__ void mx_quantize_items(const void* __restrict__ x,
+                                                  uint32_t* __restrict__ packed,
+                                                  uint8_t* __restrict__ scales, int64_t n_items,
+                                                  int64_t base, int64_t stride, int lane) {
+  auto in_range = [&](int64_t item) { return kFull || item < n_items; };
+  Raw8<DT> raw[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int64_t item = base + u * stride + lane;
+    if (in_range(item) && MXQ_IN_RANGE(kChkMxQuantIn, item, n_items))
+      raw[u] = load_raw8<DT>(x, item);
+  }
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const int64_t item = base + u * stride + lane;
+    const bool valid = in_range(item);
+    // Block amax over the four lanes that hold one 32-element block.
+    uint32_t m = valid ? raw_amax<DT>(raw[u]) : 0u;
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    if (!valid) continue;
+    const int e = mx_scale_exp(m);
+    const float inv = exp2i(-e);  // exact power of two
+    float v[8];
+    // x * 2^-e is exact; adding +0 in the same rounding turns -0.0 into
+    // +0.0 (no sign bit for it) while a negative value that underflows
+    // keeps its sign, so the code's sign bit is set iff x < 0.
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = fmaf(elem_to_f32<DT>(raw_elem<DT>(raw[u], j)), inv, 0.0f);
+    if (MXQ_IN_RANGE(kChkMxQuantOut, item, n_items)) packed[item] = e2m1x8(v);
+    if ((lane & 3) == 0 && MXQ_IN_RANGE(kChkMxQuantScale, item >> 2, n_items / 4))
+      scales[item >> 2] = (uint8_t)(e + 127);
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads)
 mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
@@ -90,38 +128,55 @@ mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kUnroll) {
-    Raw8<DT> raw[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      if (item < n_items && MXQ_IN_RANGE(kChkMxQuantIn, item, n_items))
-        raw[u] = load_raw8<DT>(x, item);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      const bool valid = item < n_items;
-      // Block amax over the four lanes that hold one 32-element block.
-      uint32_t m = valid ? raw_amax<DT>(raw[u]) : 0u;
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      if (!valid) continue;
-      const int e = mx_scale_exp(m);
-      const float inv = exp2i(-e);  // exact power of two
-      float v[8];
-      // x * 2^-e is exact; adding +0 in the same rounding turns -0.0 into
-      // +0.0 (no sign bit for it) while a negative value that underflows
-      // keeps its sign, so the code's sign bit is set iff x < 0.
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = fmaf(elem_to_f32<DT>(raw_elem<DT>(raw[u], j)), inv, 0.0f);
-      if (MXQ_IN_RANGE(kChkMxQuantOut, item, n_items)) packed[item] = e2m1x8(v);
-      if ((lane & 3) == 0 && MXQ_IN_RANGE(kChkMxQuantScale, item >> 2, n_items / 4))
-        scales[item >> 2] = (uint8_t)(e + 127);
-    }
+    // warp-uniform: base is the warp's first item
+    if (base + (kUnroll - 1) * stride + 32 <= n_items)
+      mx_quantize_items<DT, true>(x, packed, scales, n_items, base, stride, lane);
+    else
+      mx_quantize_items<DT, false>(x, packed, scales, n_items, base, stride, lane);
   }
 }
 
 // -------------------------------------------------------- mx_dequantize
+
+// One iteration of the unpack over the warp's kUnroll items.  kFull: all
+// of them exist (no bounds tests).
+template <int DT, bool kFull>
+__device__ __forceinline__ void mx_dequantize_items(const uint32_t* __restrict__ packed,
+                                                    const uint8_t* __restrict__ scales,
+                                                    void* __restrict__ out, int64_t n_items,
+                                                    int64_t base, int64_t stride, int lane) {
+  auto in_range = [&](int64_t item) { return kFull || item < n_items; };
+  uint32_t p[kUnroll], s[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    int64_t item = base + u * stride + lane;
+    if (in_range(item)) {
+      p[u] = MXQ_IN_RANGE(kChkMxDeqIn, item, n_items) ? ld_stream_u32(packed + item) : 0u;
+      s[u] = MXQ_IN_RANGE(kChkMxDeqScale, item >> 2, n_items / 4)
+                 ? ld_stream_u8(scales + (item >> 2))
+                 : 0u;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    int64_t item = base + u * stride + lane;
+    if (!in_range(item) || !MXQ_IN_RANGE(kChkMxDeqOut, item, n_items)) continue;
+    if (s[u] == 0xFFu) {  // E8M0 NaN
+      store8_bits<DT>(out, item, ElemTraits<DT>::kNaN);
+      continue;
+    }
+    float scale = exp2i((int)s[u] - 127);  // 2^-127 .. 2^127, exact
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
+      // value * scale is exact; adding +0 turns the -0 of nibble 8 into +0
+      v[2 * j] = fmaf(f16lo(h2), scale, 0.0f);
+      v[2 * j + 1] = fmaf(f16hi(h2), scale, 0.0f);
+    }
+    store8<DT>(out, item, v);
+  }
+}
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads)
@@ -131,36 +186,10 @@ mx_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __restr
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
        base += stride * kUnroll) {
-    uint32_t p[kUnroll], s[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      if (item < n_items) {
-        p[u] = MXQ_IN_RANGE(kChkMxDeqIn, item, n_items) ? ld_stream_u32(packed + item) : 0u;
-        s[u] = MXQ_IN_RANGE(kChkMxDeqScale, item >> 2, n_items / 4)
-                   ? ld_stream_u8(scales + (item >> 2))
-                   : 0u;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t item = base + u * stride + lane;
-      if (item >= n_items || !MXQ_IN_RANGE(kChkMxDeqOut, item, n_items)) continue;
-      if (s[u] == 0xFFu) {  // E8M0 NaN
-        store8_bits<DT>(out, item, ElemTraits<DT>::kNaN);
-        continue;
-      }
-      float scale = exp2i((int)s[u] - 127);  // 2^-127 .. 2^127, exact
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
-        // value * scale is exact; adding +0 turns the -0 of nibble 8 into +0
-        v[2 * j] = fmaf(f16lo(h2), scale, 0.0f);
-        v[2 * j + 1] = fmaf(f16hi(h2), scale, 0.0f);
-      }
-      store8<DT>(out, item, v);
-    }
+    if (base + (kUnroll - 1) * stride + 32 <= n_items)
+      mx_dequantize_items<DT, true>(packed, scales, out, n_items, base, stride, lane);
+    else
+      mx_dequantize_items<DT, false>(packed, scales, out, n_items, base, stride, lane);
   }
 }
 
