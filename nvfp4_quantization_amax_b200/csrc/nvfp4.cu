@@ -200,8 +200,10 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
   }
 }
 
+// Four CTAs per SM for 16-bit inputs (64 registers; the extra warps hide
+// more of the pass's latency than the few spilled values cost).
 template <int DT>
-__global__ void __launch_bounds__(kNvThreads)
+__global__ void __launch_bounds__(kNvThreads, ElemTraits<DT>::kBytes == 2 ? 4 : 1)
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
                       uint8_t* __restrict__ block_scales, float* __restrict__ global_scale,
                       const uint32_t* __restrict__ amax_word, int64_t n_items) {
