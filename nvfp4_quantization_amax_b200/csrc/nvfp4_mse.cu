@@ -48,8 +48,11 @@ __device__ __forceinline__ void load_block16(const void* x, int64_t blk, float* 
   for (int i = 0; i < 16; ++i) w[i] = elem_to_f32<DT>(bits[i]);
 }
 
+// Four CTAs per SM (64 registers, a few values spilled): the sweep is
+// issue-bound with lanes of a warp searching different numbers of codes,
+// and the extra warps fill more issue slots.
 template <int DT>
-__global__ void __launch_bounds__(kMseThreads)
+__global__ void __launch_bounds__(kMseThreads, 4)
 nvfp4_mse_kernel(const void* __restrict__ x, uint2* __restrict__ packed,
                  uint8_t* __restrict__ block_scales, float* __restrict__ global_scale,
                  const uint32_t* __restrict__ amax_word, int64_t n_blocks) {
