@@ -767,12 +767,13 @@ def time_config1(torch, mxq, gen, dev, reps=20):
             "timing": "median of %d, L2 flushed before each call" % reps, **out}
 
 
-def time_sweep(torch, mxq, gen, dev, max_log2=21):
+def time_sweep(torch, mxq, gen, dev, max_log2=21, min_log2=10):
     """Bandwidth sweep over row counts of the mixed-block workload x bf16
     [R, 7168] (normal, subnormal-range, zero and single-spike 32-blocks):
     mx_quantize, mx_dequantize and quantize_cache in the three formats, device
     time per call (CUDA events, median of 5 after 2 warm-up calls; L2 is
-    flushed before each timed call).  R = 2^10, 2^12, ..., 2^20, 2^21."""
+    flushed before each timed call).  R = 2^10, 2^12, ..., 2^20, 2^21 (those
+    from 2^min_log2 to 2^max_log2)."""
     C = 7168
     r_max = 1 << max_log2
     x = gen.mixed_blocks(r_max, C, device=dev)
@@ -782,6 +783,7 @@ def time_sweep(torch, mxq, gen, dev, max_log2=21):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     rows_out = []
     logs = sorted(set(list(range(10, min(max_log2, 20) + 1, 2)) + [max_log2]))
+    logs = [lg for lg in logs if lg >= min_log2] or [max_log2]
     for lg in logs:
         R = 1 << lg
         xr, outr, pr, sr = x[:R], out[:R], packed[:R], scales[:R]
@@ -825,7 +827,7 @@ def run_sweep(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    sw = time_sweep(torch, mxq, gen, dev, min(args.sweep_max_log2, 21))
+    sw = time_sweep(torch, mxq, gen, dev, min(args.sweep_max_log2, 21), args.sweep_min_log2)
     sw["peak_hbm_gbs"] = load_peaks()[0]["hbm_gbs"]
     print(json.dumps(sw), flush=True)
 
@@ -859,6 +861,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the step: the mixed-block bandwidth sweep over row counts")
     ap.add_argument("--sweep-max-log2", type=int, default=21, choices=range(10, 22))
+    ap.add_argument("--sweep-min-log2", type=int, default=10, choices=range(10, 22),
+                    help="with --sweep: leave out the row counts below 2^N")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave the mixed-block sweep out of the default run")
     args = ap.parse_args()

@@ -22,6 +22,7 @@ import numpy as np
 import pytest
 import torch
 
+import full_size_gemm
 import nvfp4_quantization_amax_b200 as mxq
 import oracle
 import synthetic as gen
@@ -168,9 +169,7 @@ def test_grouped_mm_full_size_eighteen_rows_per_expert(transpose_w):
     counts = gen.expert_counts(T, E).numpy()
     offs = np.cumsum(counts).astype(np.int32)
     rows = sampled_rows(offs)
-    W = gen.expert_weights(E, N, K, device=DEV, workload=5)
-    packed, scales = mxq.mx_quantize(W)
-    del W
+    hp, hs, packed, scales = full_size_gemm.packed_weights(DEV)  # packed by the oracle
     a = gen.normal_bf16(gen.seed_for(5, 4 if transpose_w else 3), (T, N if transpose_w else K),
                         device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -240,13 +239,11 @@ def test_w4a4_full_size_eighteen_rows_per_expert():
     counts = gen.expert_counts(T, E).numpy()
     offs = np.cumsum(counts).astype(np.int32)
     rows = sampled_rows(offs)
-    W = gen.expert_weights(E, N, K, device=DEV, workload=5)
-    P, S = mxq.mx_quantize(W)
-    del W
+    hp, hs, P, S = full_size_gemm.packed_weights(DEV)  # packed by the oracle
     x = gen.normal_bf16(gen.seed_for(5, 3), (T, K), device=DEV)
     y = mxq.w4a4_grouped_mm(x, P, S, torch.from_numpy(offs).to(DEV))
     torch.cuda.synchronize()
-    ref = oracle.w4a4_grouped_mm(bits(x), P.cpu().numpy(), S.cpu().numpy(), offs, rows)
+    ref = oracle.w4a4_grouped_mm(bits(x), hp, hs, offs, rows)
     yv = oracle.decode(bits(y[torch.from_numpy(rows).to(DEV)]), "bf16")
     assert_per_expert(yv, ref, owners(offs, rows), "w4a4 full size")
 
@@ -276,3 +273,67 @@ def test_nvfp4_w4a4_global_scales_far_apart():
     ref = oracle.nvfp4_w4a4_grouped_mm(bits(x), packed.numpy(), bs.numpy(), gw.numpy(), offs,
                                        rows)
     assert_per_expert(oracle.decode(bits(y), "bf16"), ref, owners(offs, rows), "nvfp4 w4a4")
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_reduced_benchmark_case_all_outputs(transpose_w):
+    # the benchmark workload's recipe at T=4096, E=8, N=256, K=512: every
+    # output against the oracle's exact sum, weights packed by the oracle
+    T, E, N, K = 4096, 8, 256, 512
+    offs = np.cumsum(gen.expert_counts(T, E).numpy()).astype(np.int32)
+    W = gen.expert_weights(E, N, K, workload=5)
+    packed, scales = oracle.mx_quantize(bits(W).reshape(E * N, K), "bf16")
+    packed, scales = packed.reshape(E, N, K // 2), scales.reshape(E, N, K // 32)
+    a = gen.normal_bf16(gen.seed_for(5, 4 if transpose_w else 3), (T, N if transpose_w else K))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = mxq.mxfp4_grouped_mm(a.to(DEV), torch.from_numpy(packed).to(DEV),
+                             torch.from_numpy(scales).to(DEV), torch.from_numpy(offs).to(DEV),
+                             transpose_w=transpose_w, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    with oracle.all_cores():
+        ref = oracle.grouped_mm(bits(a), packed, scales, offs, transpose_w=transpose_w)
+    rows = np.arange(T)
+    assert_per_expert(oracle.decode(bits(y), "bf16"), ref, owners(offs, rows), "reduced case")
+
+
+@pytest.mark.parametrize("transpose_w", [False, True])
+def test_grouped_mm_full_size_all_outputs_against_fp32_matmul(transpose_w):
+    # A secondary check, beside the oracle's sampled rows: every output of
+    # the benchmark GEMM against an fp32 matrix product (torch, TF32 off)
+    # per expert, of the weights the oracle dequantizes.  The product's own
+    # error (fp32 accumulation over <= 7168 terms) is far inside the bar.
+    T, E, N, K = full_size_gemm.T, full_size_gemm.E, full_size_gemm.N, full_size_gemm.K
+    hp, hs, packed, scales = full_size_gemm.packed_weights(DEV)
+    offs = full_size_gemm.offsets()
+    a = gen.normal_bf16(gen.seed_for(5, 4 if transpose_w else 3), (T, N if transpose_w else K),
+                        device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = mxq.mxfp4_grouped_mm(a, packed, scales, torch.from_numpy(offs).to(DEV),
+                             transpose_w=transpose_w, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    with oracle.all_cores():
+        wbits = oracle.mx_dequantize(hp, hs, "bf16")  # [E, N, K] bf16 bits
+    W = torch.from_numpy(wbits.view(np.int16)).to(DEV).view(torch.bfloat16)
+    del wbits
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        worst = 0.0
+        lo = 0
+        for e in range(E):
+            hi = int(offs[e])
+            if hi == lo:
+                continue
+            We = W[e].float()
+            ref = a[lo:hi].float() @ (We if transpose_w else We.t())
+            got = y[lo:hi].float()
+            rms = ref.pow(2).mean().sqrt()
+            bound = REL * torch.maximum(ref.abs(), 1e-2 * rms) + ABS
+            excess = float(((got - ref).abs() / bound).max())
+            assert excess <= 1.0, "expert %d: %r" % (e, excess)
+            worst = max(worst, excess)
+            lo = hi
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev

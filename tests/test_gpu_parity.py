@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import full_size_gemm
 import nvfp4_quantization_amax_b200 as mxq
 import oracle
 import synthetic as gen
@@ -302,9 +303,7 @@ def test_grouped_mm_full_size_sampled(transpose_w):
         if hi > lo:
             rows += [lo, hi - 1] + list(rng.integers(lo, hi, 2))
     rows = np.unique(np.array(rows, np.int64))
-    W = gen.expert_weights(E, N, K, device=DEV, workload=5)
-    packed, scales = mxq.mx_quantize(W)
-    del W
+    hp, hs, packed, scales = full_size_gemm.packed_weights(DEV)  # packed by the oracle
     a = gen.normal_bf16(gen.seed_for(5, 4 if transpose_w else 3), (T, N if transpose_w else K),
                         device=DEV)
     offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
@@ -312,7 +311,7 @@ def test_grouped_mm_full_size_sampled(transpose_w):
     y = mxq.mxfp4_grouped_mm(a, packed, scales, offs_d, transpose_w=transpose_w, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    ref = oracle.grouped_mm(bits(a), u8(packed), u8(scales), offs.astype(np.int32),
+    ref = oracle.grouped_mm(bits(a), hp, hs, offs.astype(np.int32),
                             transpose_w=transpose_w, rows=rows)
     yv = oracle.decode(bits(y[torch.tensor(rows, device=DEV)]), "bf16")
     assert gemm_error(yv, ref) <= GEMM_TOL

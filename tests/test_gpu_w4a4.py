@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import full_size_gemm
 import nvfp4_quantization_amax_b200 as mxq
 import oracle
 import synthetic as gen
@@ -70,16 +71,14 @@ def test_w4a4_full_size_sampled():
     T, E, N, K = 32768, 32, 2048, 7168
     counts = gen.expert_counts(T, E).numpy()
     offs = torch.tensor(np.cumsum(counts), dtype=torch.int32)
-    W = gen.expert_weights(E, N, K, device=DEV, workload=5)
-    P, S = mxq.mx_quantize(W)
-    del W
+    hp, hs, P, S = full_size_gemm.packed_weights(DEV)  # packed by the oracle
     x = gen.normal_bf16(gen.seed_for(5, 3), (T, K), device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     y = mxq.w4a4_grouped_mm(x, P, S, offs.to(DEV), status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     rows = np.array([0, 1, 255, 256, int(offs[0]) - 1, int(offs[0]), 12345, 20000, T - 1])
-    ref = oracle.w4a4_grouped_mm(bits(x), P.cpu().numpy(), S.cpu().numpy(), offs.numpy(), rows)
+    ref = oracle.w4a4_grouped_mm(bits(x), hp, hs, offs.numpy(), rows)
     assert error(oracle.decode(bits(y)[rows], "bf16"), ref) <= TOL
 
 
