@@ -14,7 +14,7 @@
 // rounds the f32 accumulation; y is rounded once to bf16 (NVFP4: after the
 // f32 product with g_x g_w[e]).
 //
-// Mapping (persistent, one CTA per SM, seven warps):
+// Mapping (persistent, one CTA per SM, eight warps):
 //   D[m, j] (f32, TMEM) += A[m, k] (weights, smem) * B[j, k] (tokens, smem)
 // with m one of the CTA's 128 weight rows (TMEM lanes), j one of up to 256
 // tokens of the expert and k the reduction index, 256 per pipeline stage
@@ -32,10 +32,14 @@
 //   * warp 7 (one lane) copies those blocks into TMEM (tcgen05.cp, 32 lanes
 //     x 128 bits, replicated to the four lane quarters) and issues four
 //     K=64 MMAs per stage, each selecting its scales by block and byte id;
-//   * warps 0-3 drain D, round to bf16, stage the tile in shared memory and
-//     store the expert's rows.
-// Every mbarrier wait is bounded: on a time-out the CTA stops all roles,
-// drains what it issued, frees TMEM and reports MXQ_ERR_TIMEOUT.
+//   * warps 0-3 drain D, round to bf16, stage the tile in shared memory
+//     (NVFP4: in two passes of 128 tokens, which leaves room for a third
+//     stage) and store the expert's rows.
+// The launch allows the CTAs to start while the previous kernel on the
+// stream finishes (programmatic stream serialization): they set up their
+// barriers and TMEM, then wait for that kernel's results before reading any
+// input.  Every mbarrier wait is bounded: on a time-out the CTA stops all
+// roles, drains what it issued, frees TMEM and reports MXQ_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
