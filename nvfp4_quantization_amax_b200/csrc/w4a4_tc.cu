@@ -59,35 +59,42 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kM = 128;                 // weight rows per tile (TMEM lanes)
-constexpr int kN = 256;                 // tokens per tile (MMA N)
+constexpr int kM = 128;                 // weight rows per MMA (TMEM lanes)
 constexpr int kKB = 128;                // bytes of codes per row per stage (256 K)
 constexpr int kMaxStages = 3;
-constexpr uint32_t kABytes = kM * kKB;            // 16 KB
-constexpr uint32_t kBBytes = kN * kKB;            // 32 KB
 constexpr uint32_t kSfBlock = 512;                // 128 rows x 4 scales
 constexpr int kMaxSmemExperts = 256;
 constexpr int kTmemCols = 512;
-constexpr int kDCol = 0;                // accumulator: columns [0, 256)
-constexpr int kSfaCol = 256;            // A scales: 4 columns per block
 
 // The two block-scaled formats: MXFP4 (one E8M0 scale per 32 K; a stage's
 // 8 scales per row fill 2 blocks, each MMA uses half a TMEM word) and NVFP4
 // (one UE4M3 scale per 16 K; 16 scales per row, 4 blocks, each MMA uses a
-// whole word).
-template <bool kNV>
+// whole word), and two tile shapes: 128 weight rows x 256 tokens, or
+// (kBig, when N is a multiple of 256) 256 weight rows x 192 tokens, two
+// M=128 MMAs sharing each token tile: 22 % fewer operand bytes and 11 %
+// fewer scale copies per product.
+template <bool kNV, bool kBig>
 struct W4Fmt {
   static constexpr int kScalesPerRow = kNV ? 16 : 8;       // per stage (256 K)
   static constexpr int kBlocks = kScalesPerRow / 4;         // per 128-row group
-  static constexpr uint32_t kSfaBytes = kBlocks * kSfBlock;
+  static constexpr int kMG = kBig ? 2 : 1;                  // 128-row weight groups per tile
+  static constexpr int kTileM = kM * kMG;                   // weight rows per tile
+  static constexpr int kTileN = kBig ? 192 : 256;           // tokens per tile (MMA N)
+  static constexpr uint32_t kABytes = kTileM * kKB;
+  static constexpr uint32_t kBBytes = kTileN * kKB;
+  static constexpr uint32_t kSfaBytes = kMG * kBlocks * kSfBlock;
   static constexpr uint32_t kSfbBytes = 2 * kBlocks * kSfBlock;  // two 128-row groups
-  static constexpr int kSfbCol = kSfaCol + 4 * kBlocks;
+  // TMEM: the kMG accumulators (kTileN columns each), then the A scales
+  // (4 columns per block, group-major), then the B scales (8 per block).
+  static constexpr int kSfaCol = kMG * kTileN;
+  static constexpr int kSfbCol = kSfaCol + 4 * kMG * kBlocks;
   static constexpr int kStages = 3;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   // Output tokens staged in shared memory at a time (bf16, 128 features
-  // each): the whole tile, or, for NVFP4, whose stages are larger (twice
-  // the scale bytes), half of it, so that three stages fit.
-  static constexpr int kYRows = kNV ? kN / 2 : kN;
+  // each): 128 x 256 tiles stage all 256 (MXFP4) or 128 (NVFP4, whose
+  // stages carry twice the scale bytes) so that three stages fit; 256 x 192
+  // tiles 96 of an accumulator's 192.
+  static constexpr int kYRows = kBig ? 96 : (kNV ? 128 : 256);
   static constexpr uint32_t kStagingBytes = kYRows * kM * 2;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
@@ -140,16 +147,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ uint32_t sf_offset(int r) { return 16 * (r & 31) + 4 * ((r >> 5) & 3); }
 
 // kWide: each scale load covers kG stages (32 bytes per row); otherwise one
-// stage (8 or 16 bytes per row).
-template <bool kNV, bool kWide>
+// stage (8 or 16 bytes per row).  kBig: the 256 x 192 tile.
+template <bool kNV, bool kWide, bool kBig>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const uint8_t* __restrict__ x_scales, const uint8_t* __restrict__ w_scales,
                const float* __restrict__ x_global, const float* __restrict__ w_global,
                const int32_t* __restrict__ offs, int64_t T, int64_t E, int64_t N, int64_t K,
                __nv_bfloat16* __restrict__ y, int32_t* dev_status, uint64_t wait_limit_ns) {
-  using F = W4Fmt<kNV>;
+  using F = W4Fmt<kNV, kBig>;
   constexpr int kStages = F::kStages;
+  constexpr uint32_t kABytes = F::kABytes, kBBytes = F::kBBytes;
+  constexpr int kTileN = F::kTileN, kMG = F::kMG;
+  constexpr int kSfaCol = F::kSfaCol;
   constexpr uint32_t kStageBytes = F::kStageBytes;
   constexpr uint32_t kSfaBytes = F::kSfaBytes;
   constexpr int kSfbCol = F::kSfbCol;
@@ -208,16 +218,16 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort = &sh->abort;
   const int nk = (int)(K / 256);
-  const int64_t col_tiles = N / kM;
+  const int64_t col_tiles = N / F::kTileM;
   const int64_t srow = K / (kNV ? 16 : 32);  // scale bytes per row
 
   if (warp == kTmaWarp) {
     // --------------------------------------------------- TMA producer
     if (lane == 0) {
-      TileWalker walk(t_offs, E, kN, col_tiles);
+      TileWalker walk(t_offs, E, kTileN, col_tiles);
       uint32_t it = 0;
       for (int64_t tile = blockIdx.x; !*abort && walk.seek(tile); tile += gridDim.x) {
-        const int32_t wy = (int32_t)(walk.expert * N + walk.col_tile * kM);
+        const int32_t wy = (int32_t)(walk.expert * N + walk.col_tile * F::kTileM);
         const int32_t xy = (int32_t)walk.row0;
         bool ok = true;
         for (int ks = 0; ks < nk; ++ks, ++it) {
@@ -248,10 +258,10 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     constexpr int kSPR = F::kScalesPerRow;
     constexpr int kG = kWide ? 32 / kSPR : 1;      // stages per load
     constexpr int kW = kG * kSPR / 4;              // 32-bit words per row and load
-    constexpr int kRowsW = 4 / kSfWarps, kRowsX = 8 / kSfWarps;
+    constexpr int kRowsW = F::kTileM / (32 * kSfWarps), kRowsX = kTileN / (32 * kSfWarps);
     const int u = warp - kSfWarp;
     using Buf = uint32_t[kRowsW + kRowsX][kW];
-    TileWalker pwalk(t_offs, E, kN, col_tiles);
+    TileWalker pwalk(t_offs, E, kTileN, col_tiles);
     int64_t ptile = blockIdx.x;
     bool phave = pwalk.seek(ptile);
     int pg = 0;  // group within the cursor's tile
@@ -269,8 +279,9 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     };
     auto issue = [&](Buf& buf) {
       if (!phave) return;
-      const int64_t rows = pwalk.row_end - pwalk.row0 < kN ? pwalk.row_end - pwalk.row0 : kN;
-      const int64_t wrow0 = pwalk.expert * N + pwalk.col_tile * kM;
+      const int64_t rows =
+          pwalk.row_end - pwalk.row0 < kTileN ? pwalk.row_end - pwalk.row0 : kTileN;
+      const int64_t wrow0 = pwalk.expert * N + pwalk.col_tile * F::kTileM;
       const int64_t col = (int64_t)4 * kW * pg;  // first scale byte of the group
 #pragma unroll
       for (int i = 0; i < kRowsW; ++i) {
@@ -306,10 +317,13 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       uint8_t* fb = sSfb(s);
 #pragma unroll
       for (int i = 0; i < kRowsW; ++i) {
-        const uint32_t o = sf_offset(lane + 32 * (kRowsW * u + i));
+        const int m = lane + 32 * (kRowsW * u + i);  // weight row of the tile
+        const uint32_t o = sf_offset(m);
+        const int g = m >> 7;  // 128-row group
 #pragma unroll
         for (int b = 0; b < F::kBlocks; ++b)
-          *reinterpret_cast<uint32_t*>(fa + b * kSfBlock + o) = buf[i][q * F::kBlocks + b];
+          *reinterpret_cast<uint32_t*>(fa + (g * F::kBlocks + b) * kSfBlock + o) =
+              buf[i][q * F::kBlocks + b];
       }
 #pragma unroll
       for (int i = 0; i < kRowsX; ++i) {
@@ -345,7 +359,7 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     Buf ba, bb;
     issue(ba);
     issue(bb);
-    TileWalker walk(t_offs, E, kN, col_tiles);
+    TileWalker walk(t_offs, E, kTileN, col_tiles);
     uint32_t it = 0, grp = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x) {
@@ -370,22 +384,24 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      TileWalker walk(t_offs, E, kN, col_tiles);
+      TileWalker walk(t_offs, E, kTileN, col_tiles);
       uint32_t it = 0, lt = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; ok && walk.seek(tile); tile += gridDim.x, ++lt) {
         if (!(ok = mbar_wait(&sh->d_empty, (lt & 1) ^ 1, abort, wait_limit_ns))) break;
         tc_fence_after();
-        const int64_t rows = walk.row_end - walk.row0 < kN ? walk.row_end - walk.row0 : kN;
+        const int64_t rows =
+            walk.row_end - walk.row0 < kTileN ? walk.row_end - walk.row0 : kTileN;
         const int n = (int)mma_n(rows);
         for (int ks = 0; ks < nk; ++ks, ++it) {
           const int s = it % kStages;
           if (!(ok = mbar_wait(&sh->full[s], (it / kStages) & 1, abort, wait_limit_ns))) break;
           tc_fence_after();
-          // scales of the stage into TMEM (A: blocks 0,1; B: (group, block)
-          // pairs (0,0) (1,0) (0,1) (1,1), 8 columns per block index)
+          // scales of the stage into TMEM (A: (group, block) group-major,
+          // 4 columns each; B: (group, block) pairs (0,0) (1,0) (0,1) (1,1),
+          // 8 columns per block index)
 #pragma unroll
-          for (int b = 0; b < F::kBlocks; ++b)
+          for (int b = 0; b < kMG * F::kBlocks; ++b)
             tmem_cp_32x128b_warpx4(tmem + kSfaCol + 4 * b,
                                    smem_desc_noswz(smem_addr(sSfa(s) + b * kSfBlock), 128));
 #pragma unroll
@@ -401,15 +417,19 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // scales are 4kk..4kk+3 (block kk, the whole word)
             const uint32_t id = kNV ? 0u : 2u * (kk & 1);
             const uint32_t blk = kNV ? kk : kk >> 1;
-            const uint32_t sfa = (tmem + kSfaCol + 4 * blk) | (id << 30);
             const uint32_t sfb = (tmem + kSfbCol + 8 * blk) | (id << 30);
             const uint32_t idesc = idesc_mxf4(kM, n, id, id, !kNV);
-            if constexpr (kNV)
-              mma_nvf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb,
-                          (ks | kk) != 0);
-            else
-              mma_mxf4_ss(tmem + kDCol, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb,
-                          (ks | kk) != 0);
+#pragma unroll
+            for (int g = 0; g < kMG; ++g) {
+              // weight group g: rows 128g .. +128 of the A tile, accumulator g
+              const uint32_t sfa = (tmem + kSfaCol + 4 * (g * F::kBlocks + blk)) | (id << 30);
+              const uint64_t ad = adesc + ((uint64_t)(g * kM * kKB) >> 4) + 2 * kk;
+              const uint32_t d = tmem + (uint32_t)(g * kTileN);
+              if constexpr (kNV)
+                mma_nvf4_ss(d, ad, bdesc + 2 * kk, idesc, sfa, sfb, (ks | kk) != 0);
+              else
+                mma_mxf4_ss(d, ad, bdesc + 2 * kk, idesc, sfa, sfb, (ks | kk) != 0);
+            }
           }
           mma_commit(&sh->empty[s]);
         }
@@ -422,7 +442,7 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue
-    TileWalker walk(t_offs, E, kN, col_tiles);
+    TileWalker walk(t_offs, E, kTileN, col_tiles);
     uint32_t lt = 0;
     for (int64_t tile = blockIdx.x; walk.seek(tile); tile += gridDim.x, ++lt) {
       if (epi_any(*abort != 0)) break;
@@ -430,49 +450,55 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       if (epi_any(!ok)) break;
       tc_fence_after();
       const int64_t row0 = walk.row0;
-      const int64_t rows = walk.row_end - row0 < kN ? walk.row_end - row0 : kN;
-      const int col = 32 * warp + lane;  // output feature within the tile's 128
+      const int64_t rows = walk.row_end - row0 < kTileN ? walk.row_end - row0 : kTileN;
+      const int col = 32 * warp + lane;  // output feature within a weight group's 128
       // NV: the product of the two per-tensor scales, applied in f32
       const float gg = kNV ? __fmul_rn(x_global[0], w_global[walk.expert]) : 1.0f;
       constexpr int kYRows = F::kYRows;
       const int nc = (int)((rows + 31) / 32);  // 32-token chunks of D
-      __nv_bfloat16* yt = y + row0 * N + walk.col_tile * kM;
       if (rows <= 0 && lane == 0) mbar_arrive(&sh->d_empty);
-      // tokens p0 .. p0 + kYRows - 1 per pass: staged, then stored
-      for (int p0 = 0; p0 < rows; p0 += kYRows) {
-        if (p0 > 0) epi_bar();  // the previous pass's rows are stored
-        const int c_end = nc < (p0 + kYRows) / 32 ? nc : (p0 + kYRows) / 32;
+      // accumulator g (weight rows 128g .. of the tile), tokens p0 .. p0 +
+      // kYRows - 1 per pass: staged, then stored
+      bool first = true;
+      for (int g = 0; g < kMG; ++g) {
+        __nv_bfloat16* yt = y + row0 * N + walk.col_tile * F::kTileM + g * kM;
+        for (int p0 = 0; p0 < rows; p0 += kYRows) {
+          if (!first) epi_bar();  // the previous pass's rows are stored
+          first = false;
+          const int c_end = nc < (p0 + kYRows) / 32 ? nc : (p0 + kYRows) / 32;
 #pragma unroll 1
-        for (int c = p0 / 32; c < c_end; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kDCol + 32 * c, v);
-          tmem_wait_ld();
-          if constexpr (kNV) {
+          for (int c = p0 / 32; c < c_end; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + g * kTileN + 32 * c, v);
+            tmem_wait_ld();
+            if constexpr (kNV) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gg);
-          }
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gg);
+            }
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-            const int t = 32 * c + j - p0;  // token within the pass
-            if (MXQ_IN_RANGE(kChkW4Smem, (t + 1) * kM + col, kYRows * kM)) {
-              sY[t * kM + col] = (uint16_t)(pr & 0xFFFFu);
-              sY[(t + 1) * kM + col] = (uint16_t)(pr >> 16);
+            for (int j = 0; j < 32; j += 2) {
+              const uint32_t pr = pack2<kBF16>(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+              const int t = 32 * c + j - p0;  // token within the pass
+              if (MXQ_IN_RANGE(kChkW4Smem, (t + 1) * kM + col, kYRows * kM)) {
+                sY[t * kM + col] = (uint16_t)(pr & 0xFFFFu);
+                sY[(t + 1) * kM + col] = (uint16_t)(pr >> 16);
+              }
             }
           }
-        }
-        if (p0 + kYRows >= rows) {  // every chunk of D is read
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->d_empty);
-        }
-        epi_bar();  // the pass is staged
-        const int r_end = rows < p0 + kYRows ? (int)rows : p0 + kYRows;
-        for (int r = p0 + 2 * warp + (lane >> 4); r < r_end; r += 2 * kEpiWarps) {
-          const uint4 val = *reinterpret_cast<const uint4*>(sY + (r - p0) * kM + 8 * (lane & 15));
-          if (MXQ_IN_RANGE(kChkW4Out, (row0 + r) * N + walk.col_tile * kM + 8 * (lane & 15) + 7,
-                           T * N))
-            *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+          if (g == kMG - 1 && p0 + kYRows >= rows) {  // every chunk of D is read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->d_empty);
+          }
+          epi_bar();  // the pass is staged
+          const int r_end = rows < p0 + kYRows ? (int)rows : p0 + kYRows;
+          for (int r = p0 + 2 * warp + (lane >> 4); r < r_end; r += 2 * kEpiWarps) {
+            const uint4 val = *reinterpret_cast<const uint4*>(sY + (r - p0) * kM + 8 * (lane & 15));
+            if (MXQ_IN_RANGE(kChkW4Out,
+                             (row0 + r) * N + walk.col_tile * F::kTileM + g * kM + 8 * (lane & 15) + 7,
+                             T * N))
+              *reinterpret_cast<uint4*>(yt + (int64_t)r * N + 8 * (lane & 15)) = val;
+          }
         }
       }
     }
@@ -487,17 +513,17 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   if (threadIdx.x == 0 && *abort && dev_status) atomicExch(dev_status, MXQ_ERR_TIMEOUT);
 }
 
-template <bool kNV>
-int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* packed,
-                const void* scales, const float* wg, const int32_t* offs, int64_t T, int64_t E,
-                int64_t N, int64_t K, void* y, int32_t* dev_status, uint64_t wait_limit_ns,
-                cudaStream_t st) {
-  using F = W4Fmt<kNV>;
+template <bool kNV, bool kBig>
+int launch_w4a4_shape(const void* xq, const void* xs, const float* xg, const void* packed,
+                      const void* scales, const float* wg, const int32_t* offs, int64_t T,
+                      int64_t E, int64_t N, int64_t K, void* y, int32_t* dev_status,
+                      uint64_t wait_limit_ns, cudaStream_t st) {
+  using F = W4Fmt<kNV, kBig>;
   CUtensorMap xmap, wmap;
-  if (!make_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, T, K / 2, K / 2, kKB, kN,
+  if (!make_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, T, K / 2, K / 2, kKB, F::kTileN,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, E * N, K / 2, K / 2, kKB, kM,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, E * N, K / 2, K / 2, kKB,
+                    F::kTileM, CU_TENSOR_MAP_SWIZZLE_128B))
     return MXQ_ERR_CUDA;
   // Scale loads of 32 bytes per row (several stages) when every row's
   // scales start on a 16-byte boundary and the stages split into whole
@@ -505,9 +531,9 @@ int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* pac
   const int64_t srow = K / (kNV ? 16 : 32);
   const int64_t group = kNV ? 2 : 4;
   const bool wide = srow % 16 == 0 && (K / 256) % group == 0;
-  auto kernel = wide ? w4a4_tc_kernel<kNV, true> : w4a4_tc_kernel<kNV, false>;
+  auto kernel = wide ? w4a4_tc_kernel<kNV, true, kBig> : w4a4_tc_kernel<kNV, false, kBig>;
   if (allow_dynamic_smem((const void*)kernel, (int)F::kSmem) != cudaSuccess) return MXQ_ERR_CUDA;
-  const int64_t tiles = ((T + kN - 1) / kN + E) * (N / kM);
+  const int64_t tiles = ((T + F::kTileN - 1) / F::kTileN + E) * (N / F::kTileM);
   const int64_t sms = num_sms();
   const int grid = (int)(tiles < sms ? tiles : sms);
   // Programmatic stream serialization: the CTAs may start their set-up while
@@ -527,6 +553,19 @@ int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* pac
       cudaLaunchKernelEx(&cfg, kernel, xmap, wmap, (const uint8_t*)xs, (const uint8_t*)scales, xg,
                          wg, offs, T, E, N, K, (__nv_bfloat16*)y, dev_status, wait_limit_ns);
   return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+// The 256 x 192 tile where N allows it, the 128 x 256 one otherwise.
+template <bool kNV>
+int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* packed,
+                const void* scales, const float* wg, const int32_t* offs, int64_t T, int64_t E,
+                int64_t N, int64_t K, void* y, int32_t* dev_status, uint64_t wait_limit_ns,
+                cudaStream_t st) {
+  if (N % 256 == 0)
+    return launch_w4a4_shape<kNV, true>(xq, xs, xg, packed, scales, wg, offs, T, E, N, K, y,
+                                        dev_status, wait_limit_ns, st);
+  return launch_w4a4_shape<kNV, false>(xq, xs, xg, packed, scales, wg, offs, T, E, N, K, y,
+                                       dev_status, wait_limit_ns, st);
 }
 
 }  // namespace
