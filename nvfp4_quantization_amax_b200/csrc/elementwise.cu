@@ -113,7 +113,9 @@ __device__ __forceinline__ void mx_quantize_items(const void* __restrict__ x,
     // +0.0 (no sign bit for it) while a negative value that underflows
     // keeps its sign, so the code's sign bit is set iff x < 0.
 #pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = fmaf(elem_to_f32<DT>(raw_elem<DT>(raw[u], j)), inv, 0.0f);
+    for (int j = 0; j < 8; j += 2)
+      fma2_rn_zero(v[j], v[j + 1], elem_to_f32<DT>(raw_elem<DT>(raw[u], j)),
+                   elem_to_f32<DT>(raw_elem<DT>(raw[u], j + 1)), inv, inv);
     if (MXQ_IN_RANGE(kChkMxQuantOut, item, n_items)) packed[item] = e2m1x8(v);
     if ((lane & 3) == 0 && MXQ_IN_RANGE(kChkMxQuantScale, item >> 2, n_items / 4))
       scales[item >> 2] = (uint8_t)(e + 127);
@@ -171,8 +173,7 @@ __device__ __forceinline__ void mx_dequantize_items(const uint32_t* __restrict__
     for (int j = 0; j < 4; ++j) {
       uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
       // value * scale is exact; adding +0 turns the -0 of nibble 8 into +0
-      v[2 * j] = fmaf(f16lo(h2), scale, 0.0f);
-      v[2 * j + 1] = fmaf(f16hi(h2), scale, 0.0f);
+      fma2_rn_zero(v[2 * j], v[2 * j + 1], f16lo(h2), f16hi(h2), scale, scale);
     }
     store8<DT>(out, item, v);
   }
@@ -237,15 +238,14 @@ __device__ __forceinline__ void fake_quant8(float* v, float s) {
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
       uint32_t h2 = e4m3x2_to_f16x2(e4m3x2(v[j], v[j + 1]));
-      v[j] = f16lo(h2) * s;  // exact; the sign of zero is kept
-      v[j + 1] = f16hi(h2) * s;
+      mul2_rn(v[j], v[j + 1], f16lo(h2), f16hi(h2), s, s);  // exact; the sign of zero is kept
     }
   } else {
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
       uint32_t h2 = e2m1x2_to_f16x2(e2m1x2(v[j], v[j + 1]));
-      v[j] = fmaf(f16lo(h2), s, 0.0f);  // exact; zero magnitudes become +0
-      v[j + 1] = fmaf(f16hi(h2), s, 0.0f);
+      // exact; zero magnitudes become +0
+      fma2_rn_zero(v[j], v[j + 1], f16lo(h2), f16hi(h2), s, s);
     }
   }
 }
@@ -276,7 +276,9 @@ quantize_cache_kernel(const void* __restrict__ in, void* __restrict__ out, int64
       const float inv = exp2i(-k), s = exp2i(k);
       float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = elem_to_f32<DT>(raw_elem<DT>(raw[u], j)) * inv;  // exact
+      for (int j = 0; j < 8; j += 2)  // exact
+        mul2_rn(v[j], v[j + 1], elem_to_f32<DT>(raw_elem<DT>(raw[u], j)),
+                elem_to_f32<DT>(raw_elem<DT>(raw[u], j + 1)), inv, inv);
       fake_quant8<FMT>(v, s);
       if (MXQ_IN_RANGE(kChkCacheOut, item, n_items)) store8<DT>(out, item, v);
     }

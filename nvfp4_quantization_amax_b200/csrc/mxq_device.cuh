@@ -144,6 +144,32 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return r;
 }
 
+// Two binary32 products, or two fmas with a +0 addend, in one instruction
+// (sm_100 mul / fma .rn.f32x2): each lane is rounded exactly as the scalar
+// operation (mul.rn / fma.rn) rounds it, subnormals kept.
+__device__ __forceinline__ void mul2_rn(float& y0, float& y1, float a0, float a1, float b0,
+                                        float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// y = a * b + 0 per lane: a zero product becomes +0, as fmaf(a, b, 0.0f).
+__device__ __forceinline__ void fma2_rn_zero(float& y0, float& y1, float a0, float a1, float b0,
+                                             float b1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, 0;\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // ---------------------------------------------------------- exponents
 
 // floor(log2 v) of a positive finite f32 given by its bit pattern
@@ -215,8 +241,11 @@ __device__ __forceinline__ uint32_t e2m1x8_quot(const float* w, float d, float r
   uint32_t a = 0, b = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    a |= e2m1x2(w[2 * j] * r_lo, w[2 * j + 1] * r_lo) << (8 * j);
-    b |= e2m1x2(w[2 * j] * r_hi, w[2 * j + 1] * r_hi) << (8 * j);
+    float l0, l1, h0, h1;
+    mul2_rn(l0, l1, w[2 * j], w[2 * j + 1], r_lo, r_lo);
+    mul2_rn(h0, h1, w[2 * j], w[2 * j + 1], r_hi, r_hi);
+    a |= e2m1x2(l0, l1) << (8 * j);
+    b |= e2m1x2(h0, h1) << (8 * j);
   }
   return a == b ? a : e2m1x8_div(w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7], d);
 }

@@ -23,7 +23,9 @@ __device__ __forceinline__ float mx_block_scale(uint32_t s) {
 
 __device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) {
   const uint32_t h2 = e2m1x2_to_f16x2(byte);
-  return pack2<kBF16>(f16lo(h2) * scale, f16hi(h2) * scale);
+  float lo, hi;
+  mul2_rn(lo, hi, f16lo(h2), f16hi(h2), scale, scale);
+  return pack2<kBF16>(lo, hi);
 }
 
 // The same result from bf16 multiplies only.  The f16 pattern of an E2M1

@@ -108,9 +108,9 @@ __device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, fl
     const float r_lo = r * (1.0f - 0x1p-19f), r_hi = r * (1.0f + 0x1p-19f);
     float lo[8], hi[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      lo[j] = fmaf(w[j], r_lo, 0.0f);
-      hi[j] = fmaf(w[j], r_hi, 0.0f);
+    for (int j = 0; j < 8; j += 2) {
+      fma2_rn_zero(lo[j], lo[j + 1], w[j], w[j + 1], r_lo, r_lo);
+      fma2_rn_zero(hi[j], hi[j + 1], w[j], w[j + 1], r_hi, r_hi);
     }
     const uint32_t a = e2m1x8(lo);
     if (a == e2m1x8(hi)) return a;
@@ -126,7 +126,8 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
                                                      uint32_t* __restrict__ packed,
                                                      uint8_t* __restrict__ block_scales,
                                                      int64_t n_items, int64_t base, int64_t stride,
-                                                     int lane, float g, float t, bool zero) {
+                                                     int lane, float t, bool zero,
+                                                     const float* s_d, const float* s_r) {
   const int p = lane & 1;
   auto in_range = [&](int64_t item) { return kFull || item < n_items; };
   uint4 va[kNvUnroll], vb[kNvUnroll];
@@ -167,10 +168,9 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
     float q = __fdiv_rn(__uint_as_float(mk), t);
     if (q == 0.0f) q = 1.0f;
     q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
-    sm[k] = e4m3x2(q, 0.0f) & 0xFFu;
-    const float s = f16lo(e4m3x2_to_f16x2(sm[k]));
-    dm[k] = __fmul_rn(s, g);
-    rm[k] = quot_fast_ok(dm[k]) ? __frcp_rn(dm[k]) : 0.0f;
+    sm[k] = e4m3x2(q, 0.0f) & 0xFFu;  // 0x01 .. 0x7E (q is positive and clamped)
+    dm[k] = s_d[sm[k] & 0x7Fu];
+    rm[k] = s_r[sm[k] & 0x7Fu];
   }
   float d4[kNvUnroll], r4[kNvUnroll];
 #pragma unroll
@@ -212,6 +212,15 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const float g = zero ? 0.0f : __fdiv_rn(amax, 2688.0f);  // 6 * 448
   const float t = __fmul_rn(6.0f, g);
   if (blockIdx.x == 0 && threadIdx.x == 0) *global_scale = g;
+  // Per E4M3 scale code c: the divisor d = fl(s_c g) and, where the bracket
+  // applies (quot_fast_ok), r = fl(1 / d), else 0.  Looked up per block.
+  __shared__ float s_d[128], s_r[128];
+  if (threadIdx.x < 128) {
+    const float d = __fmul_rn(f16lo(e4m3x2_to_f16x2(threadIdx.x)), g);
+    s_d[threadIdx.x] = d;
+    s_r[threadIdx.x] = quot_fast_ok(d) ? __frcp_rn(d) : 0.0f;
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
   for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
@@ -219,11 +228,11 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
     // every item of this iteration exists (warp-uniform: base is the
     // warp's first item)
     if (base + (kNvUnroll - 1) * stride + 32 <= n_items)
-      nvfp4_quantize_items<DT, true>(x, packed, block_scales, n_items, base, stride, lane, g, t,
-                                     zero);
+      nvfp4_quantize_items<DT, true>(x, packed, block_scales, n_items, base, stride, lane, t, zero,
+                                     s_d, s_r);
     else
-      nvfp4_quantize_items<DT, false>(x, packed, block_scales, n_items, base, stride, lane, g, t,
-                                      zero);
+      nvfp4_quantize_items<DT, false>(x, packed, block_scales, n_items, base, stride, lane, t, zero,
+                                      s_d, s_r);
   }
 }
 
@@ -259,8 +268,9 @@ nvfp4_dequantize_kernel(const uint32_t* __restrict__ packed, const uint8_t* __re
         const uint32_t h2 = e2m1x2_to_f16x2((p[u] >> (8 * j)) & 0xFFu);
         // code * s_b is exact in binary32; times g rounds once; adding +0
         // in the same fma turns the -0 of nibble 8 into +0
-        v[2 * j] = fmaf(f16lo(h2) * s, g, 0.0f);
-        v[2 * j + 1] = fmaf(f16hi(h2) * s, g, 0.0f);
+        float c0, c1;
+        mul2_rn(c0, c1, f16lo(h2), f16hi(h2), s, s);
+        fma2_rn_zero(v[2 * j], v[2 * j + 1], c0, c1, g, g);
       }
       if (MXQ_IN_RANGE(kChkNvDeqOut, item, n_items)) store8<DT>(out, item, v);
     }
