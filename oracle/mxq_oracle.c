@@ -626,6 +626,7 @@ int orc_nvfp4_mse_code(const double* w, double g) {
 int orc_nvfp4_quantize_mse_rows(const void* x, int dtype, int64_t rows, int64_t K, double g,
                                 uint8_t* packed, uint8_t* block_scales) {
   if (K % 16 != 0 || rows < 0) return ORC_EARG;
+  ORC_PARALLEL_ROWS
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t b = 0; b < K / 16; ++b) {
       int64_t base = r * K + b * 16;

@@ -85,8 +85,10 @@ def test_mse_full_expert_weight():
     xb = bits(x)
     wg = oracle.nvfp4_global_scale(np.abs(oracle.decode(xb, "bf16")).max())
     assert float(g.item()) == wg
-    rows = np.array([0, 1, 777, 1024, 2047])
-    wp, ws, _ = oracle.nvfp4_quantize_mse(xb[rows], g=wg)
+    # the first and last row and 128 seeded ones (oracle rows on all host cores)
+    rows = np.unique(np.concatenate([[0, 2047], np.random.RandomState(11).choice(2048, 128, replace=False)]))
+    with oracle.all_cores():
+        wp, ws, _ = oracle.nvfp4_quantize_mse(xb[rows], g=wg)
     assert_equal(u8(s[torch.from_numpy(rows).to(DEV)]), ws, "sampled scales")
     assert_equal(u8(p[torch.from_numpy(rows).to(DEV)]), wp, "sampled packed")
     # every block: no worse than the max rule (the dequantized product rounds
