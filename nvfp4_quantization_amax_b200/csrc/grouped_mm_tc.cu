@@ -436,10 +436,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
               const uint4 dd = d[2 * hh + c];
               const uint32_t w[4] = {dd.x, dd.y, dd.z, dd.w};
               const uint32_t sbyte = (sb4 >> (8 * (2 * hh + c))) & 0xFFu;
-              const uint32_t flo = mx_split_factor_lo(sbyte), fhi = mx_split_factor_hi(sbyte);
+              const float sc = scale_f32(sbyte);
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                v[16 * c + i] = mx_dequant_pair_split((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, flo, fhi);
+                v[16 * c + i] = dequant_pair((w[i >> 2] >> (8 * (i & 3))) & 0xFFu, sc);
             }
             if (!waited) {
               if (!(ok = warp_wait<kPair>(&sh->empty[s], ((wi / S) & 1) ^ 1, abort, wait_limit_ns)))

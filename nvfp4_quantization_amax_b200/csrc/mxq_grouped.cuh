@@ -28,32 +28,6 @@ __device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) 
   return pack2<kBF16>(lo, hi);
 }
 
-// The same result from bf16 multiplies only.  The f16 pattern of an E2M1
-// value, its exponent and mantissa shifted down by 3 bits into bf16's layout
-// and its sign kept, is the bf16 pattern of the value times 2^-112 (a normal
-// number, or zero).  Multiplying by 2^(min(s, 142) - 15), then by
-// 2^(max(s, 142) - 142), both bf16 values, gives value * 2^(s - 127); every
-// intermediate and final product is exactly representable in bf16
-// (subnormals included) for s up to 252, so neither multiply rounds.
-constexpr uint32_t kMxSplitScale = 142;  // largest s with 2^(s - 15) a bf16 value
-__device__ __forceinline__ uint32_t mx_split_factor_lo(uint32_t s) {
-  const uint32_t e = ((s < kMxSplitScale ? s : kMxSplitScale) + 112u) << 7;
-  return e | (e << 16);  // bf16x2 of 2^(min(s, 142) - 15)
-}
-__device__ __forceinline__ uint32_t mx_split_factor_hi(uint32_t s) {
-  const uint32_t e = ((s > kMxSplitScale ? s : kMxSplitScale) - 15u) << 7;
-  return e | (e << 16);  // bf16x2 of 2^(max(s, 142) - 142)
-}
-__device__ __forceinline__ uint32_t mx_dequant_pair_split(uint32_t byte, uint32_t f_lo,
-                                                          uint32_t f_hi) {
-  const uint32_t h2 = e2m1x2_to_f16x2(byte);
-  const uint32_t t = ((h2 >> 3) & 0x0FFF0FFFu) | (h2 & 0x80008000u);
-  uint32_t r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(f_lo));
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(f_hi));
-  return r;
-}
-
 // True iff offs is non-negative, non-decreasing and ends at T.  Called by
 // every thread of a CTA (contains __syncthreads); block-uniform result.
 __device__ __forceinline__ bool offs_valid(const int32_t* offs, int64_t E, int64_t T) {

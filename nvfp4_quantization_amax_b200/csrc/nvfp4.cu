@@ -23,7 +23,10 @@ namespace mxq {
 namespace {
 
 constexpr int kNvThreads = 256;
-constexpr int kNvUnroll = 4;
+constexpr int kNvUnroll = 4;   // amax and unpack passes
+// The quantize pass keeps two items per thread: with four CTAs per SM it
+// then needs no spills, which beat four items per thread.
+constexpr int kNvQUnroll = 2;
 
 template <int DT>
 __device__ __forceinline__ uint32_t elem_bits(const uint4& a, const uint4& b, int j) {
@@ -119,7 +122,7 @@ __device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, fl
                     w[6] + 0.0f, w[7] + 0.0f, d);
 }
 
-// One iteration of the quantize pass over the warp's kNvUnroll items
+// One iteration of the quantize pass over the warp's kNvQUnroll items
 // base + u stride + lane.  kFull: all of them exist (no bounds tests).
 template <int DT, bool kFull>
 __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
@@ -130,16 +133,16 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
                                                      const float* s_d, const float* s_r) {
   const int p = lane & 1;
   auto in_range = [&](int64_t item) { return kFull || item < n_items; };
-  uint4 va[kNvUnroll], vb[kNvUnroll];
+  uint4 va[kNvQUnroll], vb[kNvQUnroll];
 #pragma unroll
-  for (int u = 0; u < kNvUnroll; ++u) {
+  for (int u = 0; u < kNvQUnroll; ++u) {
     const int64_t item = base + u * stride + lane;
     if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantIn, item, n_items))
       load_vec8<DT>(x, item, va[u], vb[u]);
   }
-  uint32_t m[kNvUnroll];
+  uint32_t m[kNvQUnroll];
 #pragma unroll
-  for (int u = 0; u < kNvUnroll; ++u) {
+  for (int u = 0; u < kNvQUnroll; ++u) {
     const int64_t item = base + u * stride + lane;
     m[u] = in_range(item) ? amax8<DT>(va[u], vb[u]) : 0u;
     m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], 1));  // the block's two lanes
@@ -148,7 +151,7 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
   // item count is even and pairs are aligned)
   if (zero) {
 #pragma unroll
-    for (int u = 0; u < kNvUnroll; ++u) {
+    for (int u = 0; u < kNvQUnroll; ++u) {
       const int64_t item = base + u * stride + lane;
       if (!in_range(item)) continue;
       if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items)) packed[item] = 0u;
@@ -158,13 +161,14 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
     return;
   }
   // The two lanes of a 16-block (lanes 2i, 2i+1) share its scale; of the
-  // four unroll slots, lane parity p derives the scales of slots 2p and
-  // 2p + 1 and the pair swaps them by shuffle.
-  float dm[2], rm[2];
-  uint32_t sm[2];
+  // kNvQUnroll unroll slots, lane parity p derives the scales of slots
+  // p kH .. p kH + kH - 1 and the pair swaps them by shuffle.
+  constexpr int kH = kNvQUnroll / 2;
+  float dm[kH], rm[kH];
+  uint32_t sm[kH];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const uint32_t mk = p ? m[2 + k] : m[k];
+  for (int k = 0; k < kH; ++k) {
+    const uint32_t mk = p ? m[kH + k] : m[k];
     float q = __fdiv_rn(__uint_as_float(mk), t);
     if (q == 0.0f) q = 1.0f;
     q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
@@ -172,18 +176,18 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
     dm[k] = s_d[sm[k] & 0x7Fu];
     rm[k] = s_r[sm[k] & 0x7Fu];
   }
-  float d4[kNvUnroll], r4[kNvUnroll];
+  float d4[kNvQUnroll], r4[kNvQUnroll];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < kH; ++k) {
     const float dk = __shfl_xor_sync(0xffffffffu, dm[k], 1);
     const float rk = __shfl_xor_sync(0xffffffffu, rm[k], 1);
     d4[k] = p ? dk : dm[k];
     r4[k] = p ? rk : rm[k];
-    d4[2 + k] = p ? dm[k] : dk;
-    r4[2 + k] = p ? rm[k] : rk;
+    d4[kH + k] = p ? dm[k] : dk;
+    r4[kH + k] = p ? rm[k] : rk;
   }
 #pragma unroll
-  for (int u = 0; u < kNvUnroll; ++u) {
+  for (int u = 0; u < kNvQUnroll; ++u) {
     const int64_t item = base + u * stride + lane;
     if (!in_range(item)) continue;
     float w[8];
@@ -193,15 +197,16 @@ __device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
       packed[item] = e2m1x8_quot_unsigned_zero(w, d4[u], r4[u]);
   }
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int64_t item = base + (2 * p + k) * stride + lane;
+  for (int k = 0; k < kH; ++k) {
+    const int64_t item = base + (kH * p + k) * stride + lane;
     if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
       block_scales[item >> 1] = (uint8_t)sm[k];
   }
 }
 
-// Four CTAs per SM for 16-bit inputs (64 registers; the extra warps hide
-// more of the pass's latency than the few spilled values cost).
+// Four CTAs per SM for 16-bit inputs (at most 64 registers; with two items
+// per thread nothing spills, and the warps hide more of the pass's latency
+// than three CTAs of four-item threads).
 template <int DT>
 __global__ void __launch_bounds__(kNvThreads, ElemTraits<DT>::kBytes == 2 ? 4 : 1)
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
@@ -224,10 +229,10 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   const int lane = threadIdx.x & 31;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
   for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
-       base += stride * kNvUnroll) {
+       base += stride * kNvQUnroll) {
     // every item of this iteration exists (warp-uniform: base is the
     // warp's first item)
-    if (base + (kNvUnroll - 1) * stride + 32 <= n_items)
+    if (base + (kNvQUnroll - 1) * stride + 32 <= n_items)
       nvfp4_quantize_items<DT, true>(x, packed, block_scales, n_items, base, stride, lane, t, zero,
                                      s_d, s_r);
     else
@@ -296,7 +301,7 @@ int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* blo
                  float* global_scale, uint32_t* amax_word, cudaStream_t st) {
   const int64_t n_items = rows * (K / 8);
   run_amax<DT>(x, n_items, amax_word, st);
-  const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items, kNvThreads * kNvUnroll);
+  const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items, kNvThreads * kNvQUnroll);
   nvfp4_quantize_kernel<DT><<<grid, kNvThreads, 0, st>>>(
       x, (uint32_t*)packed, (uint8_t*)block_scales, global_scale, amax_word, n_items);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
