@@ -541,8 +541,10 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
           const int ws = wi % kWS;
           if (!(ok = warp_wait<kPair>(&sh->wfull[ws], (wi / kWS) & 1, abort, wait_limit_ns)))
             break;
-          const uint8_t* wst = sW + ws * G::kWBytes;
-          const uint8_t* sst = sS + ws * G::kSBytes;
+          // this thread's word of row rsub; rows 8j further on share its
+          // 64-byte swizzle phase ((row >> 1) & 3 = (rsub >> 1) & 3)
+          const uint8_t* wst = sW + ws * G::kWBytes + rsub * 64 + 16 * (q ^ ((rsub >> 1) & 3)) + 4 * csub;
+          const uint8_t* sst = sS + ws * G::kSBytes + rsub * 16 + soff;
           uint32_t wd[kSubAll][4];
           float sc[kSubAll][4];
 #pragma unroll
@@ -550,13 +552,12 @@ grouped_mm_tc_kernel(const __grid_constant__ CUtensorMap tmap_act,
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int row = 32 * sub_i + 8 * j + rsub;  // n within the stage
-              wd[sub_i][j] = *reinterpret_cast<const uint32_t*>(
-                  wst + row * 64 + 16 * (q ^ ((row >> 1) & 3)) + 4 * csub);
+              wd[sub_i][j] = *reinterpret_cast<const uint32_t*>(wst + (32 * sub_i + 8 * j) * 64);
               [[maybe_unused]] const int64_t gi = e * N * (K / 32) + (m0 + 32 * q) / 32 +
                                  ((int64_t)ks * kBK + row) * (K / 32);
               const uint32_t sb =
                   scales_by_tma
-                      ? (uint32_t)sst[row * 16 + soff]
+                      ? (uint32_t)sst[(32 * sub_i + 8 * j) * 16]
                       : (MXQ_IN_RANGE(kChkGemmTcScale, gi, E * N * (K / 32))
                              ? (uint32_t)scol[((int64_t)ks * kBK + row) * (K / 32)]
                              : 0u);

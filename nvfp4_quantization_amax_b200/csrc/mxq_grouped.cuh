@@ -18,7 +18,7 @@ namespace mxq {
 // 2^(s - 127) as f32: the exponent field s for s >= 1 (255 gives +inf, as
 // exp2i(128) does), the subnormal 2^-127 for s = 0.
 __device__ __forceinline__ float mx_block_scale(uint32_t s) {
-  return __uint_as_float(s != 0u ? s << 23 : 0x00400000u);
+  return __uint_as_float(max(s << 23, 0x00400000u));  // s <= 255: s << 23 >= 2^23 unless s = 0
 }
 
 __device__ __forceinline__ uint32_t mx_dequant_pair(uint32_t byte, float scale) {
