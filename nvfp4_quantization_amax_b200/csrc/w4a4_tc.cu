@@ -33,8 +33,9 @@
 //     x 128 bits, replicated to the four lane quarters) and issues four
 //     K=64 MMAs per stage, each selecting its scales by block and byte id;
 //   * warps 0-3 drain D, round to bf16, stage the tile in shared memory
-//     (NVFP4: in two passes of 128 tokens, which leaves room for a third
-//     stage) and store the expert's rows.
+//     (in passes of 64-128 tokens for NVFP4 and for the two-accumulator
+//     tile, which leaves room for a third stage) and store the expert's
+//     rows.
 // The launch allows the CTAs to start while the previous kernel on the
 // stream finishes (programmatic stream serialization): they set up their
 // barriers and TMEM, then wait for that kernel's results before reading any
@@ -70,16 +71,17 @@ constexpr int kTmemCols = 512;
 // 8 scales per row fill 2 blocks, each MMA uses half a TMEM word) and NVFP4
 // (one UE4M3 scale per 16 K; 16 scales per row, 4 blocks, each MMA uses a
 // whole word), and two tile shapes: 128 weight rows x 256 tokens, or
-// (kBig, when N is a multiple of 256) 256 weight rows x 192 tokens, two
-// M=128 MMAs sharing each token tile: 22 % fewer operand bytes and 11 %
-// fewer scale copies per product.
+// (kBig, when N is a multiple of 256) 256 weight rows x 224 tokens, two
+// M=128 MMAs sharing each token tile (fewer operand bytes and scale copies
+// per product; 224 is what TMEM holds beside the NVFP4 scale columns, and
+// an expert of up to 1120 tokens takes five token tiles).
 template <bool kNV, bool kBig>
 struct W4Fmt {
   static constexpr int kScalesPerRow = kNV ? 16 : 8;       // per stage (256 K)
   static constexpr int kBlocks = kScalesPerRow / 4;         // per 128-row group
   static constexpr int kMG = kBig ? 2 : 1;                  // 128-row weight groups per tile
   static constexpr int kTileM = kM * kMG;                   // weight rows per tile
-  static constexpr int kTileN = kBig ? 192 : 256;           // tokens per tile (MMA N)
+  static constexpr int kTileN = kBig ? 224 : 256;           // tokens per tile (MMA N)
   static constexpr uint32_t kABytes = kTileM * kKB;
   static constexpr uint32_t kBBytes = kTileN * kKB;
   static constexpr uint32_t kSfaBytes = kMG * kBlocks * kSfBlock;
@@ -92,9 +94,9 @@ struct W4Fmt {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   // Output tokens staged in shared memory at a time (bf16, 128 features
   // each): 128 x 256 tiles stage all 256 (MXFP4) or 128 (NVFP4, whose
-  // stages carry twice the scale bytes) so that three stages fit; 256 x 192
-  // tiles 96 of an accumulator's 192.
-  static constexpr int kYRows = kBig ? 96 : (kNV ? 128 : 256);
+  // stages carry twice the scale bytes) so that three stages fit; 256 x 224
+  // tiles 96 (MXFP4) or 64 (NVFP4) of an accumulator's 224 per pass.
+  static constexpr int kYRows = kBig ? (kNV ? 64 : 96) : (kNV ? 128 : 256);
   static constexpr uint32_t kStagingBytes = kYRows * kM * 2;
   static constexpr uint32_t kSmem =
       1024 + kStages * kStageBytes + kStagingBytes + 256 + 4 * kMaxSmemExperts;
@@ -147,7 +149,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ uint32_t sf_offset(int r) { return 16 * (r & 31) + 4 * ((r >> 5) & 3); }
 
 // kWide: each scale load covers kG stages (32 bytes per row); otherwise one
-// stage (8 or 16 bytes per row).  kBig: the 256 x 192 tile.
+// stage (8 or 16 bytes per row).  kBig: the 256 x 224 tile.
 template <bool kNV, bool kWide, bool kBig>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
@@ -258,7 +260,8 @@ w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     constexpr int kSPR = F::kScalesPerRow;
     constexpr int kG = kWide ? 32 / kSPR : 1;      // stages per load
     constexpr int kW = kG * kSPR / 4;              // 32-bit words per row and load
-    constexpr int kRowsW = F::kTileM / (32 * kSfWarps), kRowsX = kTileN / (32 * kSfWarps);
+    constexpr int kRowsW = F::kTileM / (32 * kSfWarps);
+    constexpr int kRowsX = (kTileN + 32 * kSfWarps - 1) / (32 * kSfWarps);  // rows past the tile read as 0
     const int u = warp - kSfWarp;
     using Buf = uint32_t[kRowsW + kRowsX][kW];
     TileWalker pwalk(t_offs, E, kTileN, col_tiles);
@@ -555,7 +558,7 @@ int launch_w4a4_shape(const void* xq, const void* xs, const float* xg, const voi
   return err == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
-// The 256 x 192 tile where N allows it, the 128 x 256 one otherwise.
+// The 256 x 224 tile where N allows it, the 128 x 256 one otherwise.
 template <bool kNV>
 int launch_w4a4(const void* xq, const void* xs, const float* xg, const void* packed,
                 const void* scales, const float* wg, const int32_t* offs, int64_t T, int64_t E,
