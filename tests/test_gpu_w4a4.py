@@ -66,6 +66,12 @@ def test_w4a4_many_small_experts_and_one_tile_shapes():
     check([300], 384, 768)
 
 
+def test_w4a4_token_tile_boundaries():
+    # N a multiple of 256 takes 224-token tiles: experts of exactly one and
+    # two tiles, one token past each, and a single token
+    check([224, 225, 448, 449, 1], 256, 512)
+
+
 def test_w4a4_full_size_sampled():
     # the benchmark GEMM: T=32768, E=32, N=2048, K=7168, multinomial counts
     T, E, N, K = 32768, 32, 2048, 7168
@@ -147,6 +153,10 @@ def test_nvfp4_w4a4_small_ragged():
 def test_nvfp4_w4a4_many_small_experts():
     nv_check([int(c) for c in np.random.RandomState(7).randint(0, 41, size=24)], 128, 256)
     nv_check([300], 384, 768)
+
+
+def test_nvfp4_w4a4_token_tile_boundaries():
+    nv_check([224, 225, 448, 449, 1], 256, 512)
 
 
 def test_nvfp4_w4a4_full_size_sampled():
