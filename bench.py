@@ -290,14 +290,15 @@ def time_next_rows(torch, mxq, step, dev, reps=3):
 E4M3_POS_CODES = 126  # positive finite E4M3 bytes 0x01 .. 0x7E
 
 
-def mse_evaluations(torch, w, g, lanes=4):
+def mse_evaluations(torch, w, g, lanes=1):
     """(candidate, weight) evaluations the mse-rule kernel performs on the
     16-blocks of w (bf16 [rows, K]) under the global scale g, replaying its
     pruning (the measurement's work unit, not a result): each block's codes
     are visited from the top (the first code whose quotient amax / d_c is at
     most 0.25, by binary search, else 126) downwards, `lanes` interleaved
-    slots each stopping at the first code whose d underflows to 0 or whose
-    clipping error (amax - 6 d)^2 alone exceeds the slot's best sum so far.
+    slots (the kernel's lanes per block: one) each stopping at the first code
+    whose d underflows to 0 or whose clipping error (amax - 6 d)^2 alone
+    exceeds the slot's best sum so far.
     Each visit evaluates 16 weights.  Error sums are formed in float64 from
     float32 quotients as in the kernel; a sum that differs from the kernel's
     in its last bits can move a stop by one code, so the count is exact up to

@@ -17,7 +17,11 @@
 // Work split: kLanes lanes share a block, each trying every kLanes-th code
 // (only the codes that can win: see the pruning below), and combine (error,
 // code) with shuffles; the lane of the first slot then writes the block's
-// eight code bytes and its scale byte.
+// eight code bytes and its scale byte.  kLanes = 1: one thread searches a
+// block's codes alone, from the top down, so its own best sum prunes every
+// remaining code of the block, and no lane idles while another lane of its
+// block is still searching (with 2 or 4 lanes per block the sweep took 13 %
+// or 32 % longer on B200).
 // This is ALU work (126 candidates x 16 divisions and fmas per block), so
 // the grid is one thread per (block, lane slot) and the CTA scheduler
 // balances the waves.
@@ -30,7 +34,7 @@ namespace mxq {
 namespace {
 
 constexpr int kMseThreads = 256;
-constexpr int kLanes = 4;  // lanes per 16-block
+constexpr int kLanes = 1;  // lanes per 16-block
 
 __device__ __forceinline__ double f16_to_f64(uint32_t h) {
   double r;
@@ -49,7 +53,7 @@ __device__ __forceinline__ void load_block16(const void* x, int64_t blk, float* 
 }
 
 // Four CTAs per SM (64 registers, a few values spilled): the sweep is
-// issue-bound with lanes of a warp searching different numbers of codes,
+// issue-bound with the blocks of a warp needing different numbers of codes,
 // and the extra warps fill more issue slots.
 template <int DT>
 __global__ void __launch_bounds__(kMseThreads, 4)
