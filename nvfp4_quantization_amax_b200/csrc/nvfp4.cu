@@ -17,6 +17,7 @@
 
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
+#include "sm100_primitives.cuh"
 
 namespace mxq {
 
@@ -69,10 +70,19 @@ __device__ __forceinline__ void load_vec8(const void* x, int64_t item, uint4& a,
 
 __global__ void clear_word_kernel(uint32_t* w) { *w = 0u; }
 
+// The amax and quantize passes are launched with programmatic stream
+// serialization: a pass's CTAs may be scheduled while the kernel before it
+// finishes (each pass allows it for its successor at once), and wait for
+// that kernel's results (sm100::griddep_wait) before touching what it wrote.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // max |x| over the tensor as binary32 bits, accumulated with atomicMax.
 template <int DT>
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restrict__ amax_word) {
+  griddep_launch_dependents();
   __shared__ uint32_t s_max[kNvThreads / 32];
   uint32_t m = 0;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
@@ -96,6 +106,7 @@ nvfp4_amax_kernel(const void* __restrict__ x, int64_t n_items, uint32_t* __restr
   if (threadIdx.x < 32) {
     m = threadIdx.x < kNvThreads / 32 ? s_max[threadIdx.x] : 0u;
     m = __reduce_max_sync(0xffffffffu, m);
+    sm100::griddep_wait();  // the cleared word (x itself was complete before the clear)
     if (threadIdx.x == 0 && m != 0u) atomicMax(amax_word, m);
   }
 }
@@ -212,6 +223,8 @@ __global__ void __launch_bounds__(kNvThreads, ElemTraits<DT>::kBytes == 2 ? 4 : 
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
                       uint8_t* __restrict__ block_scales, float* __restrict__ global_scale,
                       const uint32_t* __restrict__ amax_word, int64_t n_items) {
+  griddep_launch_dependents();
+  sm100::griddep_wait();  // the amax pass has completed
   const float amax = __uint_as_float(*amax_word);
   const bool zero = amax == 0.0f;
   const float g = zero ? 0.0f : __fdiv_rn(amax, 2688.0f);  // 6 * 448
@@ -287,12 +300,27 @@ int grid_for(Kernel kernel, int64_t n_units, int per_block) {
   return wave_grid((const void*)kernel, kNvThreads, n_units, per_block);
 }
 
+// Launch with programmatic stream serialization (see griddep_launch_dependents).
+template <class... Params, class... Args>
+void launch_dependent(void (*kernel)(Params...), int grid, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kNvThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int DT>
 void run_amax(const void* x, int64_t n_items, uint32_t* amax_word, cudaStream_t st) {
   clear_word_kernel<<<1, 1, 0, st>>>(amax_word);
   if (n_items > 0) {
     const int grid = grid_for(nvfp4_amax_kernel<DT>, n_items, kNvThreads * kNvUnroll);
-    nvfp4_amax_kernel<DT><<<grid, kNvThreads, 0, st>>>(x, n_items, amax_word);
+    launch_dependent(nvfp4_amax_kernel<DT>, grid, st, x, n_items, amax_word);
   }
 }
 
@@ -302,8 +330,8 @@ int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* blo
   const int64_t n_items = rows * (K / 8);
   run_amax<DT>(x, n_items, amax_word, st);
   const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items, kNvThreads * kNvQUnroll);
-  nvfp4_quantize_kernel<DT><<<grid, kNvThreads, 0, st>>>(
-      x, (uint32_t*)packed, (uint8_t*)block_scales, global_scale, amax_word, n_items);
+  launch_dependent(nvfp4_quantize_kernel<DT>, grid, st, x, (uint32_t*)packed,
+                   (uint8_t*)block_scales, global_scale, (const uint32_t*)amax_word, n_items);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
