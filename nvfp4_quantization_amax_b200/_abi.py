@@ -193,6 +193,9 @@ def _ptr(t):
 # together).  The results equal one call on the whole tensor: these
 # operations treat every row on its own.
 HOST_CHUNK_BYTES = 64 << 20
+# A tensor of less than two such chunks still streams, in four chunks of at
+# least this many bytes (smaller tensors take one round trip).
+HOST_MIN_CHUNK_BYTES = 4 << 20
 _HOST_DEPTH = 3  # device buffer sets in rotation
 
 
@@ -229,7 +232,10 @@ def _stream_rows(inputs, outputs, rows, launch, what):
     ins = [t.view(rows, -1) for t in inputs]
     outs = [t.view(rows, -1) for t in outputs]
     in_row = sum(t.shape[1] * t.element_size() for t in ins)
-    chunk = max(1, HOST_CHUNK_BYTES // max(1, in_row))
+    chunk_bytes = HOST_CHUNK_BYTES
+    if rows * in_row < 2 * HOST_CHUNK_BYTES:
+        chunk_bytes = max(min(HOST_MIN_CHUNK_BYTES, HOST_CHUNK_BYTES), rows * in_row // 4)
+    chunk = max(1, chunk_bytes // max(1, in_row))
     n_chunks = (rows + chunk - 1) // chunk
     if n_chunks < 2:
         return False
