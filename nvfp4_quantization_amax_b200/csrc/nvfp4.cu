@@ -7,8 +7,8 @@
 // Three launches on the caller's stream: clear the amax word of the
 // workspace, a grid-wide amax (warp and CTA reductions, one atomicMax per
 // CTA on the magnitude bits, which order like the values), then the
-// streaming quantize pass (same item/lane layout as the MXFP4 pack, with a
-// block of 16 held by two lanes).  Every binary32 operation the recipe names
+// streaming quantize pass (one 16-block per lane: its maximum, scale and
+// codes need no exchange between lanes).  Every binary32 operation the recipe names
 // (the divisions and products) is the IEEE-rounded one (div.rn / mul.rn), or
 // gives provably the same E2M1 code (the guarded reciprocal quotient of
 // e2m1x8_quot), so the codes match a plain float32 implementation bit for
@@ -25,9 +25,8 @@ namespace {
 
 constexpr int kNvThreads = 256;
 constexpr int kNvUnroll = 4;   // amax and unpack passes
-// The quantize pass keeps two items per thread: with four CTAs per SM it
-// then needs no spills, which beat four items per thread.
-constexpr int kNvQUnroll = 2;
+// The quantize pass: one 16-block per lane and iteration (40 registers).
+constexpr int kNvQUnroll = 1;
 
 template <int DT>
 __device__ __forceinline__ uint32_t elem_bits(const uint4& a, const uint4& b, int j) {
@@ -133,91 +132,79 @@ __device__ __forceinline__ uint32_t e2m1x8_quot_unsigned_zero(const float* w, fl
                     w[6] + 0.0f, w[7] + 0.0f, d);
 }
 
-// One iteration of the quantize pass over the warp's kNvQUnroll items
-// base + u stride + lane.  kFull: all of them exist (no bounds tests).
-template <int DT, bool kFull>
-__device__ __forceinline__ void nvfp4_quantize_items(const void* __restrict__ x,
-                                                     uint32_t* __restrict__ packed,
-                                                     uint8_t* __restrict__ block_scales,
-                                                     int64_t n_items, int64_t base, int64_t stride,
-                                                     int lane, float t, bool zero,
-                                                     const float* s_d, const float* s_r) {
-  const int p = lane & 1;
-  auto in_range = [&](int64_t item) { return kFull || item < n_items; };
-  uint4 va[kNvQUnroll], vb[kNvQUnroll];
-#pragma unroll
-  for (int u = 0; u < kNvQUnroll; ++u) {
-    const int64_t item = base + u * stride + lane;
-    if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantIn, item, n_items))
-      load_vec8<DT>(x, item, va[u], vb[u]);
-  }
-  uint32_t m[kNvQUnroll];
-#pragma unroll
-  for (int u = 0; u < kNvQUnroll; ++u) {
-    const int64_t item = base + u * stride + lane;
-    m[u] = in_range(item) ? amax8<DT>(va[u], vb[u]) : 0u;
-    m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], 1));  // the block's two lanes
-  }
-  // both lanes of a block are in range or out of range together (the
-  // item count is even and pairs are aligned)
-  if (zero) {
-#pragma unroll
-    for (int u = 0; u < kNvQUnroll; ++u) {
-      const int64_t item = base + u * stride + lane;
-      if (!in_range(item)) continue;
-      if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items)) packed[item] = 0u;
-      if (p == 0 && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
-        block_scales[item >> 1] = 0x38u;  // E4M3 1.0
-    }
-    return;
-  }
-  // The two lanes of a 16-block (lanes 2i, 2i+1) share its scale; of the
-  // kNvQUnroll unroll slots, lane parity p derives the scales of slots
-  // p kH .. p kH + kH - 1 and the pair swaps them by shuffle.
-  constexpr int kH = kNvQUnroll / 2;
-  float dm[kH], rm[kH];
-  uint32_t sm[kH];
-#pragma unroll
-  for (int k = 0; k < kH; ++k) {
-    const uint32_t mk = p ? m[kH + k] : m[k];
-    float q = __fdiv_rn(__uint_as_float(mk), t);
-    if (q == 0.0f) q = 1.0f;
-    q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
-    sm[k] = e4m3x2(q, 0.0f) & 0xFFu;  // 0x01 .. 0x7E (q is positive and clamped)
-    dm[k] = s_d[sm[k] & 0x7Fu];
-    rm[k] = s_r[sm[k] & 0x7Fu];
-  }
-  float d4[kNvQUnroll], r4[kNvQUnroll];
-#pragma unroll
-  for (int k = 0; k < kH; ++k) {
-    const float dk = __shfl_xor_sync(0xffffffffu, dm[k], 1);
-    const float rk = __shfl_xor_sync(0xffffffffu, rm[k], 1);
-    d4[k] = p ? dk : dm[k];
-    r4[k] = p ? rk : rm[k];
-    d4[kH + k] = p ? dm[k] : dk;
-    r4[kH + k] = p ? rm[k] : rk;
-  }
-#pragma unroll
-  for (int u = 0; u < kNvQUnroll; ++u) {
-    const int64_t item = base + u * stride + lane;
-    if (!in_range(item)) continue;
-    float w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(va[u], vb[u], j));
-    if (MXQ_IN_RANGE(kChkNvQuantOut, item, n_items))
-      packed[item] = e2m1x8_quot_unsigned_zero(w, d4[u], r4[u]);
-  }
-#pragma unroll
-  for (int k = 0; k < kH; ++k) {
-    const int64_t item = base + (kH * p + k) * stride + lane;
-    if (in_range(item) && MXQ_IN_RANGE(kChkNvQuantScale, item >> 1, n_items / 2))
-      block_scales[item >> 1] = (uint8_t)sm[k];
+// 16 elements of block blk as two items (16-byte loads kept in L1: the
+// lane's second load reads the other half of the sectors its first one
+// brought in).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+template <int DT>
+__device__ __forceinline__ void load_block16v(const void* x, int64_t blk, uint4& a0, uint4& b0,
+                                              uint4& a1, uint4& b1) {
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    a0 = ld_nc_v4((const char*)x + blk * 32);
+    a1 = ld_nc_v4((const char*)x + blk * 32 + 16);
+  } else {
+    a0 = ld_nc_v4((const char*)x + blk * 64);
+    b0 = ld_nc_v4((const char*)x + blk * 64 + 16);
+    a1 = ld_nc_v4((const char*)x + blk * 64 + 32);
+    b1 = ld_nc_v4((const char*)x + blk * 64 + 48);
   }
 }
 
-// Four CTAs per SM for 16-bit inputs (at most 64 registers; with two items
-// per thread nothing spills, and the warps hide more of the pass's latency
-// than three CTAs of four-item threads).
+// One iteration of the quantize pass: each lane one 16-block (two items) of
+// kNvQUnroll slots base + u stride + lane.  kFull: all of them exist.
+template <int DT, bool kFull>
+__device__ __forceinline__ void nvfp4_quantize_blocks(const void* __restrict__ x,
+                                                      uint2* __restrict__ packed,
+                                                      uint8_t* __restrict__ block_scales,
+                                                      int64_t n_blocks, int64_t base,
+                                                      int64_t stride, int lane, float t, bool zero,
+                                                      const float* s_d, const float* s_r) {
+  auto in_range = [&](int64_t blk) { return kFull || blk < n_blocks; };
+  uint4 a0[kNvQUnroll], b0[kNvQUnroll], a1[kNvQUnroll], b1[kNvQUnroll];
+#pragma unroll
+  for (int u = 0; u < kNvQUnroll; ++u) {
+    const int64_t blk = base + u * stride + lane;
+    if (in_range(blk) && MXQ_IN_RANGE(kChkNvQuantIn, 2 * blk + 1, 2 * n_blocks))
+      load_block16v<DT>(x, blk, a0[u], b0[u], a1[u], b1[u]);
+  }
+  if (zero) {
+#pragma unroll
+    for (int u = 0; u < kNvQUnroll; ++u) {
+      const int64_t blk = base + u * stride + lane;
+      if (!in_range(blk)) continue;
+      if (MXQ_IN_RANGE(kChkNvQuantOut, 2 * blk + 1, 2 * n_blocks)) packed[blk] = make_uint2(0u, 0u);
+      if (MXQ_IN_RANGE(kChkNvQuantScale, blk, n_blocks)) block_scales[blk] = 0x38u;  // E4M3 1.0
+    }
+    return;
+  }
+#pragma unroll
+  for (int u = 0; u < kNvQUnroll; ++u) {
+    const int64_t blk = base + u * stride + lane;
+    if (!in_range(blk)) continue;
+    const uint32_t m = max(amax8<DT>(a0[u], b0[u]), amax8<DT>(a1[u], b1[u]));
+    float q = __fdiv_rn(__uint_as_float(m), t);
+    if (q == 0.0f) q = 1.0f;
+    q = fminf(fmaxf(q, 0.001953125f), 448.0f);  // [2^-9, 448]
+    const uint32_t sc = e4m3x2(q, 0.0f) & 0xFFu;  // 0x01 .. 0x7E
+    const float d = s_d[sc & 0x7Fu], r = s_r[sc & 0x7Fu];
+    float w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(a0[u], b0[u], j));
+    const uint32_t c0 = e2m1x8_quot_unsigned_zero(w, d, r);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = elem_to_f32<DT>(elem_bits<DT>(a1[u], b1[u], j));
+    const uint32_t c1 = e2m1x8_quot_unsigned_zero(w, d, r);
+    if (MXQ_IN_RANGE(kChkNvQuantOut, 2 * blk + 1, 2 * n_blocks)) packed[blk] = make_uint2(c0, c1);
+    if (MXQ_IN_RANGE(kChkNvQuantScale, blk, n_blocks)) block_scales[blk] = (uint8_t)sc;
+  }
+}
+
+// At least four CTAs per SM for 16-bit inputs (at most 64 registers; the
+// one-block-per-lane pass needs 40, and the occupancy query sizes the grid).
 template <int DT>
 __global__ void __launch_bounds__(kNvThreads, ElemTraits<DT>::kBytes == 2 ? 4 : 1)
 nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
@@ -240,17 +227,16 @@ nvfp4_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
+  const int64_t n_blocks = n_items / 2;
   const int64_t stride = (int64_t)gridDim.x * kNvThreads;
-  for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_items;
+  for (int64_t base = (int64_t)blockIdx.x * kNvThreads + (threadIdx.x & ~31); base < n_blocks;
        base += stride * kNvQUnroll) {
-    // every item of this iteration exists (warp-uniform: base is the
-    // warp's first item)
-    if (base + (kNvQUnroll - 1) * stride + 32 <= n_items)
-      nvfp4_quantize_items<DT, true>(x, packed, block_scales, n_items, base, stride, lane, t, zero,
-                                     s_d, s_r);
+    if (base + (kNvQUnroll - 1) * stride + 32 <= n_blocks)
+      nvfp4_quantize_blocks<DT, true>(x, (uint2*)packed, block_scales, n_blocks, base, stride,
+                                      lane, t, zero, s_d, s_r);
     else
-      nvfp4_quantize_items<DT, false>(x, packed, block_scales, n_items, base, stride, lane, t, zero,
-                                      s_d, s_r);
+      nvfp4_quantize_blocks<DT, false>(x, (uint2*)packed, block_scales, n_blocks, base, stride,
+                                       lane, t, zero, s_d, s_r);
   }
 }
 
@@ -329,7 +315,7 @@ int run_quantize(const void* x, int64_t rows, int64_t K, void* packed, void* blo
                  float* global_scale, uint32_t* amax_word, cudaStream_t st) {
   const int64_t n_items = rows * (K / 8);
   run_amax<DT>(x, n_items, amax_word, st);
-  const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items, kNvThreads * kNvQUnroll);
+  const int grid = grid_for(nvfp4_quantize_kernel<DT>, n_items / 2, kNvThreads * kNvQUnroll);
   launch_dependent(nvfp4_quantize_kernel<DT>, grid, st, x, (uint32_t*)packed,
                    (uint8_t*)block_scales, global_scale, (const uint32_t*)amax_word, n_items);
   return cudaGetLastError() == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
