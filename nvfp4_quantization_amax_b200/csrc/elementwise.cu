@@ -2,11 +2,14 @@
 // and cache fake quantization (quantize_cache) for sm_100a.
 //
 // All three are streaming passes.  The work unit ("item") is 8 consecutive
-// elements of one row: one 16-byte load of bf16/f16 input.  A block of B
+// elements of one row: one 16-byte load of bf16/f16 input.  The pack gives
+// each lane one whole 32-element block (four items, loads kept in L1), so a
+// block's maximum, scale, code bytes and scale byte need no exchange between
+// lanes.  In the unpack and the cache fake quantization a block of B
 // channels is B/8 consecutive items, handled by B/8 consecutive lanes of one
-// warp, which combine their block maximum with xor-shuffles.  Each thread
+// warp, which combine their block maximum with xor-shuffles; each thread
 // keeps kUnroll independent items in flight (coalesced 16-byte loads with
-// L1 no-allocate), and the grid is a whole number of waves over the SMs.
+// L1 no-allocate).  The grid is a whole number of waves over the SMs.
 //
 // Page references (title, then section):
 //  "nemo_automodel.components.quantization.mxfp4": quantize_mxfp4 (scale
@@ -82,60 +85,70 @@ __device__ __forceinline__ int mx_scale_exp(uint32_t amax_f32bits) {
   return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
-// One iteration of the pack over the warp's kUnroll items base + u stride
-// + lane.  kFull: all of them exist (no bounds tests).
-template <int DT, bool kFull>
-__device__ __forceinline__ void mx_quantize_items(const void* __restrict__ x,
-                                                  uint32_t* __restrict__ packed,
-                                                  uint8_t* __restrict__ scales, int64_t n_items,
-                                                  int64_t base, int64_t stride, int lane) {
-  auto in_range = [&](int64_t item) { return kFull || item < n_items; };
-  Raw8<DT> raw[kUnroll];
-#pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const int64_t item = base + u * stride + lane;
-    if (in_range(item) && MXQ_IN_RANGE(kChkMxQuantIn, item, n_items))
-      raw[u] = load_raw8<DT>(x, item);
+// A 32-element block of the pack's input: its four items, read with 16-byte
+// loads kept in L1 (a lane's loads read the halves of the same sectors).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+template <int DT>
+__device__ __forceinline__ Raw8<DT> load_raw8_l1(const void* base, int64_t item) {
+  Raw8<DT> r;
+  if constexpr (ElemTraits<DT>::kBytes == 2) {
+    r.a = ld_nc_v4((const char*)base + item * 16);
+  } else {
+    r.a = ld_nc_v4((const char*)base + item * 32);
+    r.b = ld_nc_v4((const char*)base + item * 32 + 16);
   }
+  return r;
+}
+
+// One iteration of the pack: each lane one 32-element block (four items) at
+// base + lane, with its maximum, scale, 16 code bytes and scale byte.
+template <int DT, bool kFull>
+__device__ __forceinline__ void mx_quantize_block(const void* __restrict__ x,
+                                                  uint4* __restrict__ packed,
+                                                  uint8_t* __restrict__ scales, int64_t n_blocks,
+                                                  int64_t blk) {
+  if (!kFull && blk >= n_blocks) return;
+  if (!MXQ_IN_RANGE(kChkMxQuantIn, 4 * blk + 3, 4 * n_blocks)) return;
+  Raw8<DT> raw[4];
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const int64_t item = base + u * stride + lane;
-    const bool valid = in_range(item);
-    // Block amax over the four lanes that hold one 32-element block.
-    uint32_t m = valid ? raw_amax<DT>(raw[u]) : 0u;
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    if (!valid) continue;
-    const int e = mx_scale_exp(m);
-    const float inv = exp2i(-e);  // exact power of two
+  for (int i = 0; i < 4; ++i) raw[i] = load_raw8_l1<DT>(x, 4 * blk + i);
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, raw_amax<DT>(raw[i]));
+  const int e = mx_scale_exp(m);
+  const float inv = exp2i(-e);  // exact power of two
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
     float v[8];
     // x * 2^-e is exact; adding +0 in the same rounding turns -0.0 into
     // +0.0 (no sign bit for it) while a negative value that underflows
     // keeps its sign, so the code's sign bit is set iff x < 0.
 #pragma unroll
     for (int j = 0; j < 8; j += 2)
-      fma2_rn_zero(v[j], v[j + 1], elem_to_f32<DT>(raw_elem<DT>(raw[u], j)),
-                   elem_to_f32<DT>(raw_elem<DT>(raw[u], j + 1)), inv, inv);
-    if (MXQ_IN_RANGE(kChkMxQuantOut, item, n_items)) packed[item] = e2m1x8(v);
-    if ((lane & 3) == 0 && MXQ_IN_RANGE(kChkMxQuantScale, item >> 2, n_items / 4))
-      scales[item >> 2] = (uint8_t)(e + 127);
+      fma2_rn_zero(v[j], v[j + 1], elem_to_f32<DT>(raw_elem<DT>(raw[i], j)),
+                   elem_to_f32<DT>(raw_elem<DT>(raw[i], j + 1)), inv, inv);
+    c[i] = e2m1x8(v);
   }
+  if (MXQ_IN_RANGE(kChkMxQuantOut, 4 * blk + 3, 4 * n_blocks))
+    packed[blk] = make_uint4(c[0], c[1], c[2], c[3]);
+  if (MXQ_IN_RANGE(kChkMxQuantScale, blk, n_blocks)) scales[blk] = (uint8_t)(e + 127);
 }
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads)
 mx_quantize_kernel(const void* __restrict__ x, uint32_t* __restrict__ packed,
                    uint8_t* __restrict__ scales, int64_t n_items) {
-  const int lane = threadIdx.x & 31;
+  const int64_t n_blocks = n_items / 4;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < n_items;
-       base += stride * kUnroll) {
-    // warp-uniform: base is the warp's first item
-    if (base + (kUnroll - 1) * stride + 32 <= n_items)
-      mx_quantize_items<DT, true>(x, packed, scales, n_items, base, stride, lane);
-    else
-      mx_quantize_items<DT, false>(x, packed, scales, n_items, base, stride, lane);
-  }
+  for (int64_t blk = (int64_t)blockIdx.x * kThreads + threadIdx.x; blk < n_blocks; blk += stride)
+    mx_quantize_block<DT, true>(x, (uint4*)packed, scales, n_blocks, blk);
 }
 
 // -------------------------------------------------------- mx_dequantize
@@ -347,7 +360,7 @@ static int grid_for(Kernel kernel, int64_t n_units, int per_block) {
 int launch_mx_quantize(const void* x, int dt, int64_t rows, int64_t K, void* packed, void* scales,
                        cudaStream_t st) {
   const int64_t n_items = rows * (K / 8);
-  const int per = kThreads * kUnroll;
+  const int per = kThreads * 4;  // items: one 32-block per thread and iteration
   auto* p = (uint32_t*)packed;
   auto* s = (uint8_t*)scales;
   switch (dt) {
