@@ -239,7 +239,8 @@ int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
  *  packed        device, [rows, K/2] bytes (output), 16-byte aligned: E2M1
  *                codes, low nibble = even column.
  *  block_scales  device, [rows, K/16] E4M3 bytes (output), one per 16 values.
- *  global_scale  device, one float (output): g = max|x| / (6 * 448).
+ *  global_scale  device, one float (output), 4-byte aligned: g = max|x| /
+ *                (6 * 448).
  *  workspace     device, MXQ_NVFP4_WORKSPACE_BYTES bytes of scratch, owned by
  *                the caller, clobbered; calls that overlap on the GPU must not
  *                share it.
@@ -250,15 +251,15 @@ int nvfp4_w4a4_grouped_mm(const void* x_packed, const void* x_block_scales,
  *  sign bit iff x < 0).  An all-zero tensor gives g = 0, codes 0 and block
  *  scales 1.0.  Precondition: max|x| is 0 or at least 2^-126.
  *  Errors: K % 16 != 0 -> MXQ_ERR_SHAPE; null -> MXQ_ERR_INVALID_ARG;
- *  misaligned x/packed/workspace -> MXQ_ERR_ALIGNMENT. */
+ *  misaligned x/packed/workspace/global_scale -> MXQ_ERR_ALIGNMENT. */
 int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* packed,
                    void* block_scales, float* global_scale, void* workspace, void* stream);
 
 /* NVFP4 unpack: out[r][k] = round_dtype(fl32(E2M1(nibble) * s_b * g)) (the
  * binary32 product, rounded once more to out_dtype).  Nibble 8 gives +0.0.
  *  packed [rows, K/2] (16-byte aligned), block_scales [rows, K/16] E4M3,
- *  global_scale device float, out [rows, K] (16-byte aligned).
- *  Errors as for nvfp4_quantize. */
+ *  global_scale device float (4-byte aligned), out [rows, K] (16-byte
+ *  aligned).  Errors as for nvfp4_quantize. */
 int nvfp4_dequantize(const void* packed, const void* block_scales, const float* global_scale,
                      int64_t rows, int64_t K, void* out, int out_dtype, void* stream);
 

@@ -300,7 +300,8 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, void* pa
   if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
   if (!fits(rows, K)) return MXQ_ERR_SHAPE;
-  if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
+  if (!aligned16(workspace) || !word_aligned(global_scale) ||
+      (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
     return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4},
                  {workspace, MXQ_NVFP4_WORKSPACE_BYTES}},
@@ -317,7 +318,8 @@ int nvfp4_quantize_mse(const void* x, int x_dtype, int64_t rows, int64_t K, void
   if (!global_scale || !workspace) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
   if (!fits(rows, K)) return MXQ_ERR_SHAPE;
-  if (!aligned16(workspace) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
+  if (!aligned16(workspace) || !word_aligned(global_scale) ||
+      (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
     return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4},
                  {workspace, MXQ_NVFP4_WORKSPACE_BYTES}},
@@ -334,7 +336,8 @@ int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t rows, int64_t K, 
   if (!global_scale) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && K > 0 && (!x || !packed || !block_scales)) return MXQ_ERR_INVALID_ARG;
   if (!fits(rows, K)) return MXQ_ERR_SHAPE;
-  if (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))) return MXQ_ERR_ALIGNMENT;
+  if (!word_aligned(global_scale) || (rows > 0 && K > 0 && (!aligned16(x) || !aligned16(packed))))
+    return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4}},
                 {{x, rows * K * elem_bytes(x_dtype)}}))
     return MXQ_ERR_INVALID_ARG;
@@ -352,7 +355,8 @@ int nvfp4_dequantize(const void* packed, const void* block_scales, const float* 
   if (rows == 0 || K == 0) return MXQ_OK;
   if (!packed || !block_scales || !global_scale || !out) return MXQ_ERR_INVALID_ARG;
   if (!fits(rows, K)) return MXQ_ERR_SHAPE;
-  if (!aligned16(packed) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  if (!aligned16(packed) || !aligned16(out) || !word_aligned(global_scale))
+    return MXQ_ERR_ALIGNMENT;
   if (!no_alias({{out, rows * K * elem_bytes(out_dtype)}},
                 {{packed, rows * K / 2}, {block_scales, rows * K / 16}, {global_scale, 4}}))
     return MXQ_ERR_INVALID_ARG;

@@ -136,10 +136,15 @@ def test_nvfp4_validation(L):
     assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, NULL, A1, NULL) == EARG  # global scale
     assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, A2, BAD, NULL) == EALIGN
     assert L.nvfp4_quantize(BAD, 0, 4, 64, A2, A2, A2, A1, NULL) == EALIGN
+    # the global scale is one float the kernels read or write: 4-byte aligned
+    assert L.nvfp4_quantize(A1, 0, 4, 64, A2, A2, BAD, A1, NULL) == EALIGN
+    assert L.nvfp4_quantize(NULL, 0, 0, 64, NULL, NULL, BAD, A1, NULL) == EALIGN
+    assert L.nvfp4_quantize_mse(A1, 0, 4, 64, A2, A2, BAD, A1, NULL) == EALIGN
     assert L.nvfp4_quantize(A1, 9, 4, 64, A2, A2, A2, A1, NULL) == EARG
     assert L.nvfp4_dequantize(A1, A2, A2, 4, 24, A1, 0, NULL) == ESHAPE
     assert L.nvfp4_dequantize(A1, A2, NULL, 4, 32, A1, 0, NULL) == EARG
     assert L.nvfp4_dequantize(BAD, A2, A2, 4, 32, A1, 0, NULL) == EALIGN
+    assert L.nvfp4_dequantize(A1, A2, BAD, 4, 32, A1, 0, NULL) == EALIGN
     assert L.nvfp4_dequantize(NULL, NULL, NULL, 0, 32, NULL, 0, NULL) == OK
 
 
@@ -148,6 +153,7 @@ def test_nvfp4_noalloc_validation_needs_no_gpu(L):
     assert L.nvfp4_quantize_noalloc(A1, 0, 4, 40, A2, A2, A2, NULL) == ESHAPE
     assert L.nvfp4_quantize_noalloc(A1, 0, 4, 64, A2, A2, NULL, NULL) == EARG
     assert L.nvfp4_quantize_noalloc(BAD, 0, 4, 64, A2, A2, A2, NULL) == EALIGN
+    assert L.nvfp4_quantize_noalloc(A1, 0, 4, 64, A2, A2, BAD, NULL) == EALIGN
     assert L.nvfp4_quantize_noalloc(A1, 5, 4, 64, A2, A2, A2, NULL) == EARG
 
 
