@@ -304,3 +304,60 @@ def test_plain_c_program_builds_against_the_header_and_links(tmp_path, L):
                            "-lmxq", "-Wl,-rpath," + libdir, "-o", str(exe_cc)])
     out_cc = subprocess.run([str(exe_cc)], capture_output=True, text=True, timeout=60)
     assert out_cc.returncode == 0 and out_cc.stdout == out.stdout
+
+
+def _base(i):
+    # distinct, widely spaced stand-in device addresses (never dereferenced)
+    return (i + 1) << 24
+
+
+# Every pointer the header documents as aligned: (entry point, argument
+# template with ("P", i) for the i-th stand-in pointer, {argument index:
+# the boundary it must sit on}).  Sizes are small and valid, so each call
+# below fails only on the one pointer moved off its boundary.
+_ALIGNED_POINTERS = [
+    ("mx_quantize", [("P", 0), 0, 4, 64, ("P", 1), ("P", 2), NULL], {0: 16, 4: 16}),
+    ("mx_dequantize", [("P", 0), ("P", 1), 4, 64, ("P", 2), 0, NULL], {0: 16, 4: 16}),
+    ("quantize_cache", [("P", 0), ("P", 1), 0, 4, 64, 0, 32, NULL], {0: 2, 1: 2}),
+    ("quantize_cache", [("P", 0), ("P", 1), 2, 4, 64, 1, 32, NULL], {0: 4, 1: 4}),
+    ("quantize_cache_packed", [("P", 0), 0, 4, 64, 1, 32, ("P", 1), ("P", 2), NULL], {0: 2}),
+    ("dequantize_cache_packed", [("P", 0), ("P", 1), 4, 64, 1, 32, ("P", 2), 0, NULL], {6: 2}),
+    ("mxfp4_grouped_mm",
+     [("P", 0), ("P", 1), ("P", 2), ("P", 3), 8, 1, 128, 256, 0, ("P", 4), ("P", 5), NULL],
+     {0: 2, 3: 4, 9: 2, 10: 4}),
+    ("mxfp4_w4a4_grouped_mm",
+     [("P", 0), ("P", 1), ("P", 2), ("P", 3), ("P", 4), 8, 1, 128, 256, ("P", 5), ("P", 6), NULL],
+     {0: 16, 1: 16, 2: 16, 3: 16, 4: 4, 9: 16, 10: 4}),
+    ("nvfp4_w4a4_grouped_mm",
+     [("P", 0), ("P", 1), ("P", 2), ("P", 3), ("P", 4), ("P", 5), ("P", 6), 8, 1, 128, 256,
+      ("P", 7), ("P", 8), NULL],
+     {0: 16, 1: 16, 2: 4, 3: 16, 4: 16, 5: 4, 6: 4, 11: 16, 12: 4}),
+    ("nvfp4_quantize", [("P", 0), 0, 4, 64, ("P", 1), ("P", 2), ("P", 3), ("P", 4), NULL],
+     {0: 16, 4: 16, 6: 4, 7: 16}),
+    ("nvfp4_quantize_mse", [("P", 0), 0, 4, 64, ("P", 1), ("P", 2), ("P", 3), ("P", 4), NULL],
+     {0: 16, 4: 16, 6: 4, 7: 16}),
+    ("nvfp4_quantize_noalloc", [("P", 0), 0, 4, 64, ("P", 1), ("P", 2), ("P", 3), NULL],
+     {0: 16, 4: 16, 6: 4}),
+    ("nvfp4_dequantize", [("P", 0), ("P", 1), ("P", 2), 4, 64, ("P", 3), 0, NULL],
+     {0: 16, 2: 4, 5: 16}),
+    ("mxq_debug_selftest", [("P", 0), NULL], {0: 4}),
+]
+
+
+@pytest.mark.parametrize("name,template,rules", _ALIGNED_POINTERS,
+                         ids=["%s-%d" % (e[0], i) for i, e in enumerate(_ALIGNED_POINTERS)])
+def test_every_aligned_pointer_is_checked_before_launch(L, name, template, rules):
+    fn = getattr(L, name)
+    for idx, boundary in rules.items():
+        # every offset that leaves the boundary, at one byte and at half of it
+        for off in sorted({1, boundary // 2}):
+            if off == 0:
+                continue
+            args = []
+            for k, a in enumerate(template):
+                if isinstance(a, tuple):
+                    addr = _base(a[1]) + (off if k == idx else 0)
+                    args.append(ctypes.c_void_p(addr))
+                else:
+                    args.append(a)
+            assert fn(*args) == EALIGN, (name, idx, off)
