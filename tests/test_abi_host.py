@@ -361,3 +361,26 @@ def test_every_aligned_pointer_is_checked_before_launch(L, name, template, rules
                 else:
                     args.append(a)
             assert fn(*args) == EALIGN, (name, idx, off)
+
+
+# The pointers each call needs (all but the optional status word and the
+# stream), by argument index, for the same templates: on a non-empty shape a
+# null in any of them is MXQ_ERR_INVALID_ARG before a launch.
+_REQUIRED_POINTERS = {
+    "mx_quantize": (0, 4, 5), "mx_dequantize": (0, 1, 4), "quantize_cache": (0, 1),
+    "quantize_cache_packed": (0, 6, 7), "dequantize_cache_packed": (0, 1, 6),
+    "mxfp4_grouped_mm": (0, 1, 2, 3, 9), "mxfp4_w4a4_grouped_mm": (0, 1, 2, 3, 4, 9),
+    "nvfp4_w4a4_grouped_mm": (0, 1, 2, 3, 4, 5, 6, 11), "nvfp4_quantize": (0, 4, 5, 6, 7),
+    "nvfp4_quantize_mse": (0, 4, 5, 6, 7), "nvfp4_quantize_noalloc": (0, 4, 5, 6),
+    "nvfp4_dequantize": (0, 1, 2, 5), "mxq_debug_selftest": (0,),
+}
+
+
+@pytest.mark.parametrize("name,template,rules", _ALIGNED_POINTERS,
+                         ids=["%s-%d" % (e[0], i) for i, e in enumerate(_ALIGNED_POINTERS)])
+def test_every_required_pointer_is_checked_before_launch(L, name, template, rules):
+    fn = getattr(L, name)
+    for idx in _REQUIRED_POINTERS[name]:
+        args = [ctypes.c_void_p(0 if k == idx else _base(a[1])) if isinstance(a, tuple) else a
+                for k, a in enumerate(template)]
+        assert fn(*args) == EARG, (name, idx)
