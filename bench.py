@@ -123,7 +123,7 @@ class ClockSampler:
 
     def __enter__(self):
         cmd = ["nvidia-smi", "-i", str(self.index),
-               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--query-gpu=timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
                "--format=csv,noheader,nounits", "-lms", "20"]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
@@ -148,26 +148,40 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
+    def summary(self, t0=None, t1=None):
+        """Clocks while the GPU ran the timed region: the samples whose
+        nvidia-smi timestamp falls in [t0, t1] (host wall-clock seconds of
+        the region's start and of its closing synchronize)."""
+        samples = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 4:
+            if len(parts) < 5:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-                mask = int(parts[3], 16)
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx, mask = float(parts[1]), float(parts[2]), int(parts[4], 16)
             except ValueError:
                 continue
-            for bit, name in REASON_BITS.items():
-                if mask & bit and name != "gpu_idle":
-                    reasons.add(name)
-        if not sm:
+            try:
+                watts = float(parts[3])
+            except ValueError:  # "[N/A]"
+                watts = None
+            samples.append((ts, sm, mx, watts, mask))
+        if not samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        loaded = sorted(sm)[len(sm) // 2:] if len(sm) > 3 else sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        window = [x for x in samples if t0 is not None and t0 <= x[0] <= t1]
+        used = window if window else samples
+        reasons = set()
+        for x in used:
+            for bit, name in REASON_BITS.items():
+                if x[4] & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x[1] for x in used),
+                "sm_min_mhz": min(x[1] for x in used), "sm_max_mhz": used[-1][2],
+                "power_w_median": (round(statistics.median(w), 1)
+                                   if (w := [x[3] for x in used if x[3] is not None]) else None),
+                "reasons": sorted(reasons), "samples": len(used),
+                "window": "timed region" if window else "whole sampler run (no sample in the region)"}
 
 
 # ------------------------------------------------------------ GPU arm
@@ -361,8 +375,9 @@ def mse_roofline(evals_s, clocks):
     an ncu count (profiles/mse_issue.json: smsp__thread_inst_executed.sum of
     one launch over the evaluations the replay counts for that launch); the
     peak is every SM sub-partition issuing one full warp instruction per
-    clock: 148 x 4 x 32 thread instructions per cycle at the SM clock
-    sampled during the benchmark."""
+    clock: 148 x 4 x 32 thread instructions per cycle at the maximum SM
+    clock (the sweep runs outside the timed step, whose sampled clock may
+    sit lower under the power cap)."""
     path = os.path.join(ROOT, "profiles", "mse_issue.json")
     if not os.path.exists(path):
         return None
@@ -370,7 +385,7 @@ def mse_roofline(evals_s, clocks):
         prof = json.load(f)
     if prof.get("source_sha") != source_hash("nvfp4_mse.cu"):
         return None
-    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
     per_eval = prof["thread_inst_per_eval"]
     peak = 148 * 4 * 32 * mhz * 1e6 / per_eval
     return {"bound": "issue", "unit": "G evaluations/s", "achieved": round(evals_s / 1e9, 2),
@@ -469,11 +484,13 @@ def run_gpu(args, rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(gpu_id(torch, dev)) as clk:
+        t_region = time.time()
         start.record()
         for k in range(args.steps):
             step.run(ev[k])
         stop.record()
         torch.cuda.synchronize()
+        t_region = (t_region, time.time())
     if world > 1:
         dist.barrier()
     if int(step.status.item()) != 0:
@@ -499,7 +516,8 @@ def run_gpu(args, rank, world):
             extra["sweep"] = time_sweep(torch, mxq, gen, dev, args.sweep_max_log2)
 
     if rank == 0:
-        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary(), next_ms, extra)
+        report(args, world, total_ms, kern_ms, e2e_dt, h2d, d2h, clk.summary(*t_region), next_ms,
+               extra)
     if world > 1:
         dist.destroy_process_group()
 

@@ -75,3 +75,30 @@ def test_report_line_has_the_contract_keys(world):
         3 * bench.algorithmic_bytes()["quantize_cache"]
     per_gpu = qd_bytes / ((0.45 + 0.44 + 0.06) * 1e-3) / 1e9
     assert abs(line["value"] - world * per_gpu) / (world * per_gpu) < 1e-3
+
+
+def _smi_line(ts, sm, watts, mask):
+    import datetime
+
+    stamp = datetime.datetime.fromtimestamp(ts).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    return "%s, %s, 1965, %s, 0x%016x" % (stamp, sm, watts, mask)
+
+
+def test_clock_summary_takes_only_the_timed_region():
+    # idle samples at the boost clock before and after the region, power-capped
+    # ones inside it: the summary must describe the region alone
+    t0 = 1_800_000_000.0
+    clk = bench.ClockSampler(0)
+    clk.lines = ([_smi_line(t0 - 0.2 + 0.02 * i, 1965, 300.0, 0x1) for i in range(10)] +
+                 [_smi_line(t0 + 0.01 + 0.02 * i, 1500 + i, 990.0, 0x4) for i in range(5)] +
+                 [_smi_line(t0 + 0.2 + 0.02 * i, 1965, "[N/A]", 0x0) for i in range(10)] +
+                 ["garbage", ""])
+    s = clk.summary(t0, t0 + 0.1)
+    assert s["samples"] == 5 and s["window"] == "timed region"
+    assert s["sm_mhz"] == 1502 and s["sm_min_mhz"] == 1500 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_median"] == 990.0
+    # no sample inside the region: every sample, and the summary says so
+    s = clk.summary(t0 + 5.0, t0 + 5.001)
+    assert s["samples"] == 25 and s["window"].startswith("whole sampler run")
+    assert s["sm_mhz"] == 1965 and s["power_w_median"] == 300.0
+    assert bench.ClockSampler(0).summary(t0, t0 + 1)["reasons"] == ["unavailable"]
