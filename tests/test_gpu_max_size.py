@@ -8,7 +8,8 @@ whole-tensor calls, as the sweep times them, and the oracle checks sampled
 rows: the first and the last, 16 seeded ones, and the rows around the places
 where a 32-bit index or byte offset would wrap (element 2^31 of x and of the
 bf16 outputs, byte 2^32 of the packed codes).  Inputs are those rows as the
-GPU received them, copied back.
+GPU received them, copied back.  The NVFP4 max-rule quantize and unpack are
+checked the same way at the size the benchmark times them, [64, 2048, 7168].
 """
 import numpy as np
 import pytest
@@ -76,4 +77,31 @@ def test_streaming_kernels_at_the_largest_benchmark_size():
         _same(_bits(out[rows]), oracle.quantize_cache(xr, fmt, B), "%s B=%d rows" % (fmt, B))
 
     del x, packed, scales, out, rows
+    torch.cuda.empty_cache()
+
+
+def test_nvfp4_max_rule_at_the_benchmark_size():
+    # NVFP4 quantize (max rule) and unpack of the expert weights bf16
+    # [64, 2048, 7168], the size the benchmark times them at.  The per-tensor
+    # scale needs max |x| over the whole tensor: taken on the host from every
+    # element's magnitude bits (for finite bf16 they order like the values),
+    # then the oracle gives g, and the codes, block scales and unpacked values
+    # of the first, the last and 32 seeded rows.
+    W = gen.expert_weights(device=DEV)
+    p, s, g = mxq.nvfp4_quantize(W)
+    y = mxq.nvfp4_dequantize(p, s, g)
+    hb = _bits(W).reshape(-1, C)
+    amax_bits = np.array([int((hb & 0x7FFF).max())], np.uint16)
+    want_g = oracle.nvfp4_global_scale(oracle.decode(amax_bits, "bf16")[0])
+    assert float(g.item()) == want_g
+    n = hb.shape[0]
+    seeded = np.random.default_rng(5).choice(n, 32, replace=False)
+    rows = sorted({0, n - 1} | {int(r) for r in seeded})
+    want_p, want_s = oracle.nvfp4_quantize_rows(hb[rows], want_g)
+    idx = torch.tensor(rows, device=DEV)
+    _same(_u8(p.view(-1, C // 2)[idx]), want_p, "packed rows")
+    _same(_u8(s.view(-1, C // 16)[idx]), want_s, "block scale rows")
+    _same(_bits(y.view(-1, C)[idx]), oracle.nvfp4_dequantize(want_p, want_s, want_g),
+          "unpacked rows")
+    del W, p, s, g, y
     torch.cuda.empty_cache()
