@@ -852,19 +852,56 @@ def run_sweep(args):
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the scalar CPU oracle, as it stands, single-threaded
+    on the host.  One step is one bounded sample of the quant/dequant part of
+    the workload (the same generators, so the same values): mx_quantize and
+    mx_dequantize of the first 16 expert-weight rows of [64,2048,7168] and
+    quantize_cache in the three formats of the first 64 KV rows of
+    [4,8192,512]; W untimed steps, then K timed ones.  Rank 0 alone runs."""
     if rank != 0:
         return
-    cb = cpu_baseline(max(4.0, min(30.0, 2.0 * args.steps)))
-    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+    import numpy as np
+    import torch
+
+    import oracle
+    import synthetic as gen
+
+    def bf16_bits(t):
+        return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+    w_rows, kv_rows = 16, 64
+    wb = bf16_bits(gen.expert_weights(1, w_rows, 7168).view(w_rows, 7168))
+    kv = bf16_bits(gen.kv_cache((1, kv_rows, 512)).view(kv_rows, 512))
+    e_w, e_kv = w_rows * 7168, kv_rows * 512
+    step_bytes = 2 * (e_w * 2 + e_w // 2 + e_w // 32) + len(CACHE_RUNS) * e_kv * 4
+
+    def one_step():
+        pk, sc = oracle.mx_quantize(wb)
+        oracle.mx_dequantize(pk, sc)
+        for f, b in CACHE_RUNS:
+            oracle.quantize_cache(kv, f, b)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = time.perf_counter() - t0
+    value = round(step_bytes * args.steps / dt / 1e9, 4)
+    sample = ("each step: mx_quantize and mx_dequantize of [16,7168] expert-weight rows and "
+              "quantize_cache (fp8/128, mxfp4/32, nvfp4/16) of [64,512] KV rows, %d bytes of the "
+              "GPU metric's algorithmic traffic; %d timed steps after %d untimed, one thread"
+              % (step_bytes, args.steps, args.warmup))
+    cores, model = host_cpu()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD,
-                       "sample": "each step times the scalar CPU oracle on a bounded sample of "
-                                 "this workload (rows of the same tensors), single thread; "
-                                 "cpu_baseline also gives the all-core figures"},
-            "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample, "cpu_model": model, "cores_available": cores},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -102,3 +102,23 @@ def test_clock_summary_takes_only_the_timed_region():
     assert s["samples"] == 25 and s["window"].startswith("whole sampler run")
     assert s["sm_mhz"] == 1965 and s["power_w_median"] == 300.0
     assert bench.ClockSampler(0).summary(t0, t0 + 1)["reasons"] == ["unavailable"]
+
+
+def test_reference_arm_line():
+    # the oracle arm: W untimed and K timed steps on rank 0, nothing elsewhere
+    args = types.SimpleNamespace(steps=2, warmup=3)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(args, 1, 2)
+    assert buf.getvalue() == ""
+    with redirect_stdout(buf):
+        bench.run_reference(args, 0, 1)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["steps"] == 2 and line["warmup"] == 3 and line["ms_per_step"] > 0
+    assert line["value"] > 0 and line["unit"] == "GB/s" and line["higher_is_better"] is True
+    cb = line["cpu_baseline"]
+    assert cb["value"] == line["value"] and cb["kind"] == "oracle" and cb["cores"] == 1
+    assert cb["sample"] and line["config"]["workload"] == bench.WORKLOAD
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
