@@ -7,8 +7,9 @@ failure (check id, index, extent) and skips the access, so nothing traps and
 no out-of-range address is touched.  Here a child process loads it in place
 of libmxq.so and runs the small parity cases of every entry point: results
 must still equal the oracle's, and after every test no check may have
-failed (tests/conftest.py).  A second child runs the self-test, a checked
-store one element past its declared extent, and reads the record back.
+failed (tests/conftest.py).  A second child does the same for the
+maximum-size cases.  A third runs the self-test, a checked store one element
+past its declared extent, and reads the record back.
 """
 import os
 import subprocess
@@ -40,6 +41,16 @@ def test_debug_variant_passes_the_small_parity_cases_without_a_failed_check():
                        cwd=ROOT, env=debug_env(), capture_output=True, text=True, timeout=1500)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
     assert " passed" in r.stdout
+
+
+def test_debug_variant_at_the_largest_benchmark_size_without_a_failed_check():
+    # the maximum-size cases (element indices past 2^31 in one call) with
+    # every indexed access checked; both must run, not skip
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "gpu",
+                        "tests/test_gpu_max_size.py"],
+                       cwd=ROOT, env=debug_env(), capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+    assert "2 passed" in r.stdout, r.stdout[-2000:]
 
 
 SELFTEST = """
